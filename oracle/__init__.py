@@ -57,9 +57,9 @@ def lib():
         L.oracle_max_finite.argtypes = [i32]
         L.oracle_max_finite.restype = dbl
         L.oracle_padded_extents.argtypes = [i32, i32, i64, i64, ctypes.POINTER(i64), ctypes.POINTER(i64)]
-        L.oracle_codes_bytes.argtypes = [i32, i32, i32, i64, i64, i64, i64]
+        L.oracle_codes_bytes.argtypes = [i32, i32, i64, i64, i64, i64]
         L.oracle_codes_bytes.restype = i64
-        L.oracle_scales_bytes.argtypes = [i32, i32, i64, i64, i64, i64]
+        L.oracle_scales_bytes.argtypes = [i32, i32, i32, i64, i64, i64, i64]
         L.oracle_scales_bytes.restype = i64
         L.oracle_quantize.argtypes = [vp, i64, i64, i64, i64, vp, i32, i32, i32, vp, vp]
         L.oracle_dequantize.argtypes = [vp, vp, i64, i64, i64, i64, i32, i32, i32, vp]
@@ -117,18 +117,19 @@ def max_finite(fmt: int) -> float:
 # --------------------------------------------------------------------------
 # quantized layout
 # --------------------------------------------------------------------------
-def padded_extents(block: int, order: int, A: int, B: int) -> tuple[int, int]:
+def padded_extents(fmt: int, order: int, A: int, B: int) -> tuple[int, int]:
+    """(Ap, Bp): only the innermost axis is padded, to whole 16-byte rows."""
     ap, bp = ctypes.c_int64(), ctypes.c_int64()
-    lib().oracle_padded_extents(block, order, A, B, ctypes.byref(ap), ctypes.byref(bp))
+    lib().oracle_padded_extents(fmt, order, A, B, ctypes.byref(ap), ctypes.byref(bp))
     return ap.value, bp.value
 
 
-def codes_bytes(fmt, block, order, d0, d1, d2, d3) -> int:
-    return int(lib().oracle_codes_bytes(fmt, block, order, d0, d1, d2, d3))
+def codes_bytes(fmt, order, d0, d1, d2, d3) -> int:
+    return int(lib().oracle_codes_bytes(fmt, order, d0, d1, d2, d3))
 
 
-def scales_bytes(block, order, d0, d1, d2, d3) -> int:
-    return int(lib().oracle_scales_bytes(block, order, d0, d1, d2, d3))
+def scales_bytes(fmt, block, order, d0, d1, d2, d3) -> int:
+    return int(lib().oracle_scales_bytes(fmt, block, order, d0, d1, d2, d3))
 
 
 def quantize(x: np.ndarray, fmt: int, block: int, order: int) -> tuple[np.ndarray, np.ndarray]:
@@ -136,8 +137,8 @@ def quantize(x: np.ndarray, fmt: int, block: int, order: int) -> tuple[np.ndarra
     assert x.dtype == np.float32 and x.ndim == 4
     d0, d1, d2, d3 = x.shape
     strides = np.array([s // 4 for s in x.strides], dtype=np.int64)
-    codes = np.zeros(codes_bytes(fmt, block, order, d0, d1, d2, d3), dtype=np.uint8)
-    scales = np.zeros(scales_bytes(block, order, d0, d1, d2, d3), dtype=np.uint8)
+    codes = np.zeros(codes_bytes(fmt, order, d0, d1, d2, d3), dtype=np.uint8)
+    scales = np.zeros(scales_bytes(fmt, block, order, d0, d1, d2, d3), dtype=np.uint8)
     lib().oracle_quantize(_p(x), d0, d1, d2, d3, _p(strides), fmt, block, order, _p(codes), _p(scales))
     return codes, scales
 
@@ -170,11 +171,12 @@ def im2col_fp32(x: np.ndarray, R, S, sh, sw, ph, pw) -> np.ndarray:
 def im2col_cbf(codes, scales, N, C, H, W, R, S, sh, sw, ph, pw, fmt, block, order):
     """Channel-batch-first im2col on quantized X; returns (codes, scales) of the
     expanded tensor (spatial P x Q, B = N, A = R*S*Ap)."""
-    Ap, Bp = padded_extents(block, order, C, N)
+    Ap, Bp = padded_extents(fmt, order, C, N)
     P, Q = out_hw(H, W, R, S, sh, sw, ph, pw)
-    Ae = R * S * Ap
-    co = np.zeros(codes_bytes(fmt, block, order, Bp, Ae, P, Q), dtype=np.uint8)
-    so = np.zeros(scales_bytes(block, order, Bp, Ae, P, Q), dtype=np.uint8)
+    nsa = Ap if block == B32 else -(-Ap // 32)
+    nsb = Bp if block == A32 else -(-Bp // 32)
+    co = np.zeros(codes_bytes(fmt, order, Bp, R * S * Ap, P, Q), dtype=np.uint8)
+    so = np.zeros(P * Q * nsb * R * S * nsa, dtype=np.uint8)
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
     lib().oracle_im2col_cbf(_p(codes), _p(scales), N, C, H, W, R, S, sh, sw, ph, pw,

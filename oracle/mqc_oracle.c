@@ -169,39 +169,41 @@ int oracle_scale_code(int fmt, double amax)
  *   order AB (B innermost): codes[((h*d3 + w)*Ap + a)*Bp + b]
  * 4-bit codes are packed two per byte, even element in the low nibble.
  *
- * Padded extents: a blocked axis is rounded up to 32, and so is the innermost
- * axis (for 16-byte row pitches); an axis that is neither keeps its size.
- * Scales (one byte per block):
- *   A32 : scales[(pix*Bp + b)*(Ap/32) + a/32]
- *   B32 : scales[(pix*(Bp/32) + b/32)*Ap + a]
- *   SQ32: scales[(pix*(Bp/32) + b/32)*(Ap/32) + a/32]
+ * Padded extents: only the innermost axis is padded, to a whole number of
+ * 16-byte rows (16 FP8 codes or 32 FP4 codes), so that every row starts on a
+ * 16-byte boundary; the other axis keeps its size.  A block that runs past
+ * the end of its axis is short: it covers only the real elements (zeros never
+ * raise a block's absolute maximum, so this equals zero-padding the block).
+ * Scales (one byte per block; nb(x) = ceil(x / 32)):
+ *   A32 : scales[(pix*Bp + b)*nb(Ap) + a/32]
+ *   B32 : scales[(pix*nb(Bp) + b/32)*Ap + a]
+ *   SQ32: scales[(pix*nb(Bp) + b/32)*nb(Ap) + a/32]
  */
-static int64_t up32(int64_t x) { return (x + 31) / 32 * 32; }
+static int64_t nb32(int64_t x) { return (x + 31) / 32; }
 
-void oracle_padded_extents(int block, int order, int64_t A, int64_t B, int64_t *Ap, int64_t *Bp)
+void oracle_padded_extents(int fmt, int order, int64_t A, int64_t B, int64_t *Ap, int64_t *Bp)
 {
-    int padA = (block == OR_A32 || block == OR_SQ32 || order == OR_ORDER_BA);
-    int padB = (block == OR_B32 || block == OR_SQ32 || order == OR_ORDER_AB);
-    *Ap = padA ? up32(A) : A;
-    *Bp = padB ? up32(B) : B;
+    int64_t row = fmt_bits(fmt) == 4 ? 32 : 16;      /* elements per 16 bytes */
+    *Ap = (order == OR_ORDER_BA) ? (A + row - 1) / row * row : A;
+    *Bp = (order == OR_ORDER_AB) ? (B + row - 1) / row * row : B;
 }
 
-int64_t oracle_codes_bytes(int fmt, int block, int order, int64_t d0, int64_t d1, int64_t d2, int64_t d3)
+int64_t oracle_codes_bytes(int fmt, int order, int64_t d0, int64_t d1, int64_t d2, int64_t d3)
 {
     int64_t Ap, Bp;
-    oracle_padded_extents(block, order, d1, d0, &Ap, &Bp);
+    oracle_padded_extents(fmt, order, d1, d0, &Ap, &Bp);
     int64_t n = d2 * d3 * Ap * Bp;
     return fmt_bits(fmt) == 4 ? n / 2 : n;
 }
 
-int64_t oracle_scales_bytes(int block, int order, int64_t d0, int64_t d1, int64_t d2, int64_t d3)
+int64_t oracle_scales_bytes(int fmt, int block, int order, int64_t d0, int64_t d1, int64_t d2, int64_t d3)
 {
     int64_t Ap, Bp;
-    oracle_padded_extents(block, order, d1, d0, &Ap, &Bp);
+    oracle_padded_extents(fmt, order, d1, d0, &Ap, &Bp);
     int64_t pix = d2 * d3;
-    if (block == OR_A32) return pix * Bp * (Ap / 32);
-    if (block == OR_B32) return pix * (Bp / 32) * Ap;
-    return pix * (Bp / 32) * (Ap / 32);
+    if (block == OR_A32) return pix * Bp * nb32(Ap);
+    if (block == OR_B32) return pix * nb32(Bp) * Ap;
+    return pix * nb32(Bp) * nb32(Ap);
 }
 
 static int64_t code_index(int order, int64_t pix, int64_t b, int64_t a, int64_t Ap, int64_t Bp)
@@ -211,9 +213,9 @@ static int64_t code_index(int order, int64_t pix, int64_t b, int64_t a, int64_t 
 
 static int64_t scale_index(int block, int64_t pix, int64_t b, int64_t a, int64_t Ap, int64_t Bp)
 {
-    if (block == OR_A32) return (pix * Bp + b) * (Ap / 32) + a / 32;
-    if (block == OR_B32) return (pix * (Bp / 32) + b / 32) * Ap + a;
-    return (pix * (Bp / 32) + b / 32) * (Ap / 32) + a / 32;
+    if (block == OR_A32) return (pix * Bp + b) * nb32(Ap) + a / 32;
+    if (block == OR_B32) return (pix * nb32(Bp) + b / 32) * Ap + a;
+    return (pix * nb32(Bp) + b / 32) * nb32(Ap) + a / 32;
 }
 
 static void put_code(uint8_t *codes, int fmt, int64_t idx, int code)
@@ -247,8 +249,8 @@ void oracle_quantize(const float *src, int64_t d0, int64_t d1, int64_t d2, int64
                      uint8_t *codes, uint8_t *scales)
 {
     int64_t Ap, Bp;
-    oracle_padded_extents(block, order, d1, d0, &Ap, &Bp);
-    int64_t nbytes = oracle_codes_bytes(fmt, block, order, d0, d1, d2, d3);
+    oracle_padded_extents(fmt, order, d1, d0, &Ap, &Bp);
+    int64_t nbytes = oracle_codes_bytes(fmt, order, d0, d1, d2, d3);
     memset(codes, 0, (size_t)nbytes);
     /* block extent along B and along A */
     int64_t eb = (block == OR_A32) ? 1 : 32;
@@ -259,17 +261,18 @@ void oracle_quantize(const float *src, int64_t d0, int64_t d1, int64_t d2, int64
         int64_t h = pix / d3, w = pix % d3;
         for (int64_t b0 = 0; b0 < Bp; b0 += eb)
             for (int64_t a0 = 0; a0 < Ap; a0 += ea) {
+                int64_t b1 = b0 + eb < Bp ? b0 + eb : Bp, a1 = a0 + ea < Ap ? a0 + ea : Ap;
                 double amax = 0.0;
-                for (int64_t b = b0; b < b0 + eb; ++b)
-                    for (int64_t a = a0; a < a0 + ea; ++a) {
+                for (int64_t b = b0; b < b1; ++b)
+                    for (int64_t a = a0; a < a1; ++a) {
                         double x = fabs(src_at(src, d0, d1, strides, b, a, h, w));
                         if (x > amax || x != x) amax = x;
                     }
                 int sc = oracle_scale_code(fmt, amax);
                 scales[scale_index(block, pix, b0, a0, Ap, Bp)] = (uint8_t)sc;
                 double inv = ldexp(1.0, 127 - sc);       /* 2^-e, exact */
-                for (int64_t b = b0; b < b0 + eb; ++b)
-                    for (int64_t a = a0; a < a0 + ea; ++a) {
+                for (int64_t b = b0; b < b1; ++b)
+                    for (int64_t a = a0; a < a1; ++a) {
                         double x = src_at(src, d0, d1, strides, b, a, h, w);
                         int code = oracle_encode(fmt, x * inv);
                         put_code(codes, fmt, code_index(order, pix, b, a, Ap, Bp), code);
@@ -284,7 +287,7 @@ void oracle_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t d0, 
                        int64_t d2, int64_t d3, int fmt, int block, int order, double *out)
 {
     int64_t Ap, Bp;
-    oracle_padded_extents(block, order, d1, d0, &Ap, &Bp);
+    oracle_padded_extents(fmt, order, d1, d0, &Ap, &Bp);
 #pragma omp parallel for schedule(static)
     for (int64_t b = 0; b < d0; ++b)
         for (int64_t a = 0; a < d1; ++a)
@@ -341,14 +344,14 @@ void oracle_im2col_cbf(const uint8_t *codes, const uint8_t *scales,
                        int fmt, int block, int order, uint8_t *codes_out, uint8_t *scales_out)
 {
     int64_t Ap, Bp;
-    oracle_padded_extents(block, order, Cin, N, &Ap, &Bp);
+    oracle_padded_extents(fmt, order, Cin, N, &Ap, &Bp);
     int64_t Ho = out_size(Hin, Kh, sh, ph), Wo = out_size(Win, Kw, sw, pw);
-    int64_t Ae = Kh * Kw * Ap;              /* expanded A extent (already padded) */
-    int64_t nb = oracle_codes_bytes(fmt, block, order, Bp, Ae, Ho, Wo);
+    int64_t Ae = Kh * Kw * Ap;              /* expanded A extent: Ap per tap */
+    int64_t nb = oracle_codes_bytes(fmt, order, Bp, Ae, Ho, Wo);
     memset(codes_out, 0, (size_t)nb);
-    int64_t n_sb = (block == OR_A32) ? Bp : Bp / 32;       /* scale rows per pixel */
-    int64_t n_sa = (block == OR_B32) ? Ap : Ap / 32;       /* scale cols per tap */
-    int64_t n_sa_e = (block == OR_B32) ? Ae : Ae / 32;
+    int64_t n_sb = (block == OR_A32) ? Bp : nb32(Bp);       /* scale rows per pixel */
+    int64_t n_sa = (block == OR_B32) ? Ap : nb32(Ap);       /* scale cols per tap */
+    int64_t n_sa_e = Kh * Kw * n_sa;
 #pragma omp parallel for schedule(static)
     for (int64_t p = 0; p < Ho; ++p)
         for (int64_t q = 0; q < Wo; ++q)

@@ -1,0 +1,487 @@
+// conv_gemm.cuh -- block-scaled tcgen05 implicit GEMM for the three
+// convolution GEMMs of the MicroQonv paper (arXiv:2609.28358, section II-C3
+// and section IV-B):
+//     forward        Y_f{Cout,N}   = W_f{Cout,Cin}   . X'_{Cin,N}
+//     input grad.    G_X'{Cin,N}   = W_f^T{Cout,Cin} . G_Yf{Cout,N}
+//     weight grad.   G_Wf{Cout,Cin} = G_Yf{Cout,N}   . X'^T_{Cin,N}
+// with the channel-batch-first im2col (section IV-A) folded into the operand
+// staging: the expanded X' is never written.  Each K-block of 32 elements of
+// an operand row is one OCP MX block with its own E8M0 scale, and the tensor
+// core applies both operands' scales per K-block (Eq. 7: the quantization
+// direction matches the dot-product direction).
+//
+// Two kinds share one kernel:
+//   CONV  (forward, input gradient): GEMM rows = output pixels (q, p, n),
+//         columns = output channels, reduction = (kernel tap, channel).  The
+//         A tile of a tap is one TMA box of the activation tensor at shifted
+//         coordinates (out-of-range rows are zero-filled: the padding);
+//         strided convolutions use one tensor map per stride phase.
+//   WGRAD (weight gradient): rows = C_out, columns = C_in of one tap,
+//         reduction = (output pixel, batch) with N contiguous; split over K.
+//
+// CTA layout (persistent, one CTA per SM, 10 warps):
+//   warp 0      TMA producer (codes of A and B, one elected thread)
+//   warp 1      TMEM allocator + MMA issuer (one thread): scale factors
+//               smem -> TMEM with tcgen05.cp, then tcgen05.mma block_scale
+//   warps 2-5   scale-factor gather: E8M0 bytes of every operand row and
+//               K-block into the 128x4 shared-memory atom the MMA expects
+//   warps 6-9   epilogue: TMEM -> registers -> fp32 global stores
+// Every wait is bounded in time; a wait that runs out records a device error
+// and the CTA winds down without hanging.
+#pragma once
+
+#include "common.cuh"
+
+namespace mqc {
+
+constexpr int kMaxTaps = 64;
+constexpr int kGemmThreads = 320;
+constexpr int kTmemCols = 512;
+constexpr int kSfTmemBase = 256;
+
+enum GemmKind : int { kConv = 0, kWgrad = 1 };
+
+// Where the E8M0 scale of (row, K-block) of an operand lives:
+//   base + pixel*pix_pitch + (row/row_div)*row_pitch + kblock*kb_pitch (+ tap*tap_pitch)
+struct ScaleSrc {
+    const uint8_t *base;
+    int64_t pix_pitch;
+    int64_t tap_pitch;
+    int32_t row_div;
+    int32_t row_pitch;
+    int32_t kb_pitch;
+    int32_t rows;
+    int32_t H, W;
+};
+
+struct ConvTap {
+    int16_t dh, dw;        // offsets of the A (CONV) or B (WGRAD) tensor-map coordinates
+    int16_t sf_dh, sf_dw;  // offsets of the pixel whose scales apply
+    int16_t map;           // tensor map (stride phase) of the shifted operand
+    int16_t btap;          // CONV: tap index of W; WGRAD: output offset r*S + s
+};
+
+struct alignas(64) GemmParams {
+    CUtensorMap amap[4];
+    CUtensorMap bmap[4];
+    ScaleSrc sfa, sfb;
+    ConvTap taps[kMaxTaps];
+    int32_t ntaps;
+    int32_t n_amaps, n_bmaps;    // tensor maps in use
+    int32_t BN, nb_atoms, wkb, stages, nacc;
+    uint32_t idesc;
+    uint64_t timeout_ns;
+    int32_t num_units;
+    int32_t a_box_bytes, b_box_bytes;
+    // CONV kind
+    int32_t rows_nfirst;         // A map dims (C, N, W, H) instead of (C, W, H, N)
+    int32_t bq, bp, bn;          // A box extents along q, p, n
+    int32_t TQ, TP, TN, NT;      // tile counts
+    int32_t Qe, Pe, Ne;          // output extents (row masks)
+    int32_t CB, total_kb;        // K-blocks per tap, K-blocks per tile
+    int32_t a_st_h, a_st_w;      // output coordinate -> scale pixel multiplier
+    int32_t Ncols;               // GEMM columns (output channels)
+    // WGRAD kind
+    int32_t MT, Mrows, splits, kiters_total, QG, NC, bqk, P, Q;
+    int32_t x_st_h, x_st_w;      // stride of X pixels per output pixel
+    // output
+    float *out;
+    int64_t out_base, os_q, os_p, os_n, os_c, os_m, split_pitch;
+};
+
+struct UnitInfo {
+    int nk;                 // K iterations (stages) of this unit
+    int kbase;              // WGRAD: first global K iteration
+    int q0, p0, n0;         // CONV: tile origin
+    int m0;                 // WGRAD: first output channel row
+    int col0;               // first GEMM column
+    int tap;                // WGRAD: tap of this unit
+    int split;              // WGRAD: split index
+};
+
+template <int KIND>
+__device__ __forceinline__ UnitInfo decode_unit(const GemmParams &p, int u) {
+    UnitInfo I{};
+    if (KIND == kConv) {
+        const int nt = u % p.NT;
+        const int mt = u / p.NT;
+        const int tq = mt % p.TQ;
+        const int tp = (mt / p.TQ) % p.TP;
+        const int tn = mt / (p.TQ * p.TP);
+        I.q0 = tq * p.bq;
+        I.p0 = tp * p.bp;
+        I.n0 = tn * p.bn;
+        I.col0 = nt * p.BN;
+        I.nk = (p.total_kb + 3) / 4;
+    } else {
+        int r = u;
+        const int mt = r % p.MT;
+        r /= p.MT;
+        const int nt = r % p.NT;
+        r /= p.NT;
+        I.tap = r % p.ntaps;
+        I.split = r / p.ntaps;
+        I.m0 = mt * 128;
+        I.col0 = nt * p.BN;
+        const int64_t k0 = static_cast<int64_t>(I.split) * p.kiters_total / p.splits;
+        const int64_t k1 = static_cast<int64_t>(I.split + 1) * p.kiters_total / p.splits;
+        I.kbase = static_cast<int>(k0);
+        I.nk = static_cast<int>(k1 - k0);
+    }
+    return I;
+}
+
+// Row m (0..127) of a CONV tile -> output coordinates within the tile.
+__device__ __forceinline__ void conv_row(const GemmParams &p, int m, int &iq, int &ip, int &in) {
+    if (p.rows_nfirst) {
+        in = m % p.bn;
+        iq = (m / p.bn) % p.bq;
+        ip = m / (p.bn * p.bq);
+    } else {
+        iq = m % p.bq;
+        ip = (m / p.bq) % p.bp;
+        in = m / (p.bq * p.bp);
+    }
+}
+
+__device__ __forceinline__ uint32_t swizzle_of(int wkb) {
+    return wkb == 4 ? kSwizzle128B : (wkb == 2 ? kSwizzle64B : kSwizzle32B);
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    // swizzled operand tiles need 1024-byte alignment
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int S = p.stages;
+    const int a_stage = 128 * 128;
+    const int b_stage = p.BN * 128;
+    const int sfb_stage = 512 * p.nb_atoms;
+    uint8_t *sA = smem;
+    uint8_t *sB = sA + S * a_stage;
+    uint8_t *sSFA = sB + S * b_stage;
+    uint8_t *sSFB = sSFA + S * 512;
+    uint64_t *full_tma = reinterpret_cast<uint64_t *>(sSFB + S * sfb_stage);
+    uint64_t *full_sf = full_tma + S;
+    uint64_t *empty = full_sf + S;
+    uint64_t *acc_full = empty + S;
+    uint64_t *acc_empty = acc_full + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_tma[s], 1);
+            mbar_init(&full_sf[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < p.n_amaps; ++i) prefetch_tensormap(&p.amap[i]);
+        for (int i = 0; i < p.n_bmaps; ++i) prefetch_tensormap(&p.bmap[i]);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint64_t lim = p.timeout_ns;
+    const int sf_cols = 4 + 4 * p.nb_atoms;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const UnitInfo I = decode_unit<KIND>(p, u);
+                for (int ki = 0; ki < I.nk; ++ki, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *a_dst = sA + s * a_stage;
+                    uint8_t *b_dst = sB + s * b_stage;
+                    if (KIND == kConv) {
+                        const int nkb = min(4, p.total_kb - 4 * ki);
+                        const int nbox = (nkb + p.wkb - 1) / p.wkb;
+                        mbar_arrive_expect_tx(&full_tma[s],
+                                              static_cast<uint32_t>(nbox * (p.a_box_bytes + p.b_box_bytes)));
+                        for (int j = 0; j < nbox; ++j) {
+                            const int g = 4 * ki + j * p.wkb;
+                            const int tap = g / p.CB;
+                            const int cb = g % p.CB;
+                            const ConvTap T = p.taps[tap];
+                            const int cx = cb * 32;
+                            if (p.rows_nfirst)
+                                tma_load_4d(a_dst + j * 128 * 32 * p.wkb, &p.amap[T.map], &full_tma[s], cx, I.n0,
+                                            I.q0 + T.dw, I.p0 + T.dh);
+                            else
+                                tma_load_4d(a_dst + j * 128 * 32 * p.wkb, &p.amap[T.map], &full_tma[s], cx,
+                                            I.q0 + T.dw, I.p0 + T.dh, I.n0);
+                            tma_load_3d(b_dst + j * p.BN * 32 * p.wkb, &p.bmap[0], &full_tma[s], cx, I.col0,
+                                        T.btap);
+                        }
+                    } else {
+                        const int kg = I.kbase + ki;
+                        const int nc = kg % p.NC;
+                        const int qg = (kg / p.NC) % p.QG;
+                        const int pp = kg / (p.NC * p.QG);
+                        const ConvTap T = p.taps[I.tap];
+                        mbar_arrive_expect_tx(&full_tma[s], static_cast<uint32_t>(p.a_box_bytes + p.b_box_bytes));
+                        const int nx = nc * 32 * p.wkb;
+                        tma_load_4d(a_dst, &p.amap[0], &full_tma[s], nx, I.m0, qg * p.bqk, pp);
+                        tma_load_4d(b_dst, &p.bmap[T.map], &full_tma[s], nx, I.col0, qg * p.bqk + T.dw, pp + T.dh);
+                    }
+                }
+            }
+            if (!ok) {
+                // let the copies already in flight land before the CTA exits
+                const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0u;
+                for (uint32_t c = first; c < it; ++c)
+                    mbar_wait(&full_tma[c % S], (c / S) & 1u, 100000000ull, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, tcount = 0;
+            bool ok = true;
+            const uint32_t swz = swizzle_of(p.wkb);
+            const uint32_t row_bytes = 32u * p.wkb;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const UnitInfo I = decode_unit<KIND>(p, u);
+                if (I.nk == 0) continue;
+                const uint32_t acc = tcount % p.nacc;
+                const uint32_t aph = (tcount / p.nacc) & 1u;
+                if (!mbar_wait(&acc_empty[acc], aph ^ 1u, lim, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + acc * p.BN;
+                for (int ki = 0; ki < I.nk; ++ki, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait(&full_tma[s], ph, lim, abort_flag) || !mbar_wait(&full_sf[s], ph, lim, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfa_t = tmem + kSfTmemBase + s * sf_cols;
+                    const uint32_t sfb_t = sfa_t + 4;
+                    tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(smem_u32(sSFA + s * 512), 0, 128, kSwizzleNone));
+                    for (int a = 0; a < p.nb_atoms; ++a)
+                        tc_cp_32x128b_warpx4(sfb_t + 4 * a, make_smem_desc(smem_u32(sSFB + s * sfb_stage + a * 512),
+                                                                           0, 128, kSwizzleNone));
+                    const int nkb = KIND == kConv ? min(4, p.total_kb - 4 * ki) : 4;
+                    const uint32_t a_base = smem_u32(sA + s * a_stage);
+                    const uint32_t b_base = smem_u32(sB + s * b_stage);
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        const int j = kb / p.wkb, within = kb % p.wkb;
+                        const uint64_t adesc =
+                            make_smem_desc(a_base + j * 128 * row_bytes + within * 32, 16, 8 * row_bytes, swz);
+                        const uint64_t bdesc =
+                            make_smem_desc(b_base + j * p.BN * row_bytes + within * 32, 16, 8 * row_bytes, swz);
+                        const uint32_t idesc = p.idesc | (static_cast<uint32_t>(kb) << 29) |
+                                               (static_cast<uint32_t>(kb) << 4);
+                        tc_mma_mxf8f6f4(d_tmem, adesc, bdesc, idesc, sfa_t | (static_cast<uint32_t>(kb) << 30),
+                                        sfb_t | (static_cast<uint32_t>(kb) << 30), (ki > 0 || kb > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
+                }
+                if (!ok) break;
+                tc_commit(&acc_full[acc]);
+                ++tcount;
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ scale-factor gather
+        const int sfw = warp - 2;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const UnitInfo I = decode_unit<KIND>(p, u);
+            // A rows of this lane: m = lane + 32 j
+            int ra_h[4], ra_w[4], ra_off[4];
+            bool ra_ok[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int m = lane + 32 * j;
+                if (KIND == kConv) {
+                    int iq, ip, in;
+                    conv_row(p, m, iq, ip, in);
+                    const int q = I.q0 + iq, pr = I.p0 + ip, n = I.n0 + in;
+                    ra_ok[j] = m < p.bq * p.bp * p.bn && q < p.Qe && pr < p.Pe && n < p.Ne;
+                    ra_h[j] = p.a_st_h * pr;
+                    ra_w[j] = p.a_st_w * q;
+                    ra_off[j] = (n / p.sfa.row_div) * p.sfa.row_pitch;
+                } else {
+                    const int k = I.m0 + m;
+                    ra_ok[j] = k < p.sfa.rows;
+                    ra_h[j] = 0;
+                    ra_w[j] = 0;
+                    ra_off[j] = (k / p.sfa.row_div) * p.sfa.row_pitch;
+                }
+            }
+            for (int ki = 0; ki < I.nk; ++ki, ++it) {
+                if (static_cast<int>(it & 3u) != sfw) continue;
+                const int s = static_cast<int>(it % S);
+                const uint32_t ph = (it / S) & 1u;
+                uint32_t wa[4] = {0u, 0u, 0u, 0u};      // A atom bytes: row lane+32j, byte kb
+                uint32_t wb[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+                if (KIND == kConv) {
+                    const int nkb = min(4, p.total_kb - 4 * ki);
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        const int g = 4 * ki + kb;
+                        const int tap = g / p.CB, cb = g % p.CB;
+                        const ConvTap T = p.taps[tap];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
+                            if (ra_ok[j] && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W) {
+                                const uint8_t *src = p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
+                                                     ra_off[j] + cb * p.sfa.kb_pitch;
+                                wa[j] |= static_cast<uint32_t>(__ldg(src)) << (8 * kb);
+                            }
+                        }
+                        const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
+                        for (int at = 0; at < p.nb_atoms; ++at)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int r = I.col0 + 128 * at + 32 * j + lane;
+                                if (128 * at + 32 * j + lane < p.BN && r < p.sfb.rows)
+                                    wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + (r / p.sfb.row_div) * p.sfb.row_pitch))
+                                                 << (8 * kb);
+                            }
+                    }
+                } else {
+                    const int kg = I.kbase + ki;
+                    const int nc = kg % p.NC;
+                    const int qg = (kg / p.NC) % p.QG;
+                    const int pp = kg / (p.NC * p.QG);
+                    const ConvTap T = p.taps[I.tap];
+                    for (int kb = 0; kb < 4; ++kb) {
+                        const int q = qg * p.bqk + kb / p.wkb;
+                        const int nb = nc * p.wkb + kb % p.wkb;
+                        if (q >= p.Q) continue;
+                        const uint8_t *asrc = p.sfa.base + (static_cast<int64_t>(pp) * p.Q + q) * p.sfa.pix_pitch +
+                                              nb * p.sfa.kb_pitch;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (ra_ok[j]) wa[j] |= static_cast<uint32_t>(__ldg(asrc + ra_off[j])) << (8 * kb);
+                        const int hh = p.x_st_h * pp + T.sf_dh, ww = p.x_st_w * q + T.sf_dw;
+                        if (hh < 0 || hh >= p.sfb.H || ww < 0 || ww >= p.sfb.W) continue;
+                        const uint8_t *bsrc = p.sfb.base + (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
+                                              nb * p.sfb.kb_pitch;
+                        for (int at = 0; at < p.nb_atoms; ++at)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int r = I.col0 + 128 * at + 32 * j + lane;
+                                if (128 * at + 32 * j + lane < p.BN && r < p.sfb.rows)
+                                    wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + (r / p.sfb.row_div) * p.sfb.row_pitch))
+                                                 << (8 * kb);
+                            }
+                    }
+                }
+                if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                *reinterpret_cast<uint4 *>(sSFA + s * 512 + lane * 16) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+                for (int at = 0; at < p.nb_atoms; ++at)
+                    *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + at * 512 + lane * 16) =
+                        make_uint4(wb[at][0], wb[at][1], wb[at][2], wb[at][3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_sf[s]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int qd = warp & 3;               // TMEM lane quadrant of this warp
+        const int m = qd * 32 + lane;
+        uint32_t tcount = 0;
+        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+            const UnitInfo I = decode_unit<KIND>(p, u);
+            bool row_ok;
+            int64_t row_off;
+            if (KIND == kConv) {
+                int iq, ip, in;
+                conv_row(p, m, iq, ip, in);
+                const int q = I.q0 + iq, pr = I.p0 + ip, n = I.n0 + in;
+                row_ok = m < p.bq * p.bp * p.bn && q < p.Qe && pr < p.Pe && n < p.Ne;
+                row_off = p.out_base + n * p.os_n + pr * p.os_p + q * p.os_q;
+            } else {
+                const int k = I.m0 + m;
+                row_ok = k < p.Mrows;
+                row_off = p.out_base + I.split * p.split_pitch + k * p.os_m + p.taps[I.tap].btap;
+            }
+            if (I.nk == 0) {
+                if (row_ok)
+                    for (int c = I.col0; c < min(I.col0 + p.BN, p.Ncols); ++c) p.out[row_off + c * p.os_c] = 0.0f;
+                continue;
+            }
+            const uint32_t acc = tcount % p.nacc;
+            const uint32_t aph = (tcount / p.nacc) & 1u;
+            if (!mbar_wait(&acc_full[acc], aph, lim, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16) + acc * p.BN;
+            for (int c16 = 0; c16 < p.BN / 16; ++c16) {
+                uint32_t r[16];
+                tc_ld_32x32b_x16(t_row + c16 * 16, r);
+                tc_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int c = I.col0 + c16 * 16 + jj;
+                        if (c < p.Ncols) p.out[row_off + c * p.os_c] = __uint_as_float(r[jj]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            ++tcount;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Deterministic split-K reduction: out[i] = sum over s (in order) of part[s][i].
+__global__ void splitk_reduce_kernel(const float *__restrict__ part, float *__restrict__ out, int64_t n, int splits) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float acc = 0.0f;
+        for (int s = 0; s < splits; ++s) acc += part[s * n + i];
+        out[i] = acc;
+    }
+}
+
+// One thread waits on a barrier that nothing signals, with a time limit, so
+// that the bounded wait runs out and records the device error.
+__global__ void expire_wait_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_wait(&bar, 0u, limit_ns, nullptr);
+    }
+}
+
+}  // namespace mqc

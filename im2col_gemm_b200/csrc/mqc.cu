@@ -1,0 +1,821 @@
+// mqc.cu -- host side of libmqc: the C ABI declared in include/mqc.h.
+// Validates arguments, encodes TMA tensor maps, chooses tile shapes and
+// launches the kernels of quantize.cuh, im2col.cuh and conv_gemm.cuh.  It
+// never allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mqc.h"
+#include "common.cuh"
+#include "conv_gemm.cuh"
+#include "im2col.cuh"
+#include "quantize.cuh"
+
+using namespace mqc;
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+mqc_status fail(mqc_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+mqc_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(MQC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+int64_t nb32(int64_t x) { return ceil_div(x, 32); }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool fmt_ok(int f) { return f == MQC_E4M3 || f == MQC_E5M2 || f == MQC_E2M1; }
+bool mx_ok(const mqc_mx *m) {
+    return m != nullptr && fmt_ok(m->fmt) && m->block >= 0 && m->block <= 2 && (m->order == 0 || m->order == 1);
+}
+int64_t row_elems(int fmt) { return fmt == MQC_E2M1 ? 32 : 16; }   // elements per 16-byte row unit
+int emax_elem(int fmt) { return fmt == MQC_E4M3 ? 8 : (fmt == MQC_E5M2 ? 15 : 2); }
+
+// Padded extents of the channel-batch-first layout: only the innermost axis
+// is padded, to whole 16-byte rows.
+void padded(int fmt, int order, int64_t A, int64_t B, int64_t &Ap, int64_t &Bp) {
+    const int64_t r = row_elems(fmt);
+    Ap = order == MQC_ORDER_BA ? round_up(A, r) : A;
+    Bp = order == MQC_ORDER_AB ? round_up(B, r) : B;
+}
+
+int64_t codes_bytes(int fmt, int order, int64_t d0, int64_t d1, int64_t d2, int64_t d3) {
+    int64_t Ap, Bp;
+    padded(fmt, order, d1, d0, Ap, Bp);
+    const int64_t n = d2 * d3 * Ap * Bp;
+    return fmt == MQC_E2M1 ? n / 2 : n;
+}
+
+int64_t scales_bytes(int fmt, int block, int order, int64_t d0, int64_t d1, int64_t d2, int64_t d3) {
+    int64_t Ap, Bp;
+    padded(fmt, order, d1, d0, Ap, Bp);
+    const int64_t pix = d2 * d3;
+    if (block == MQC_BLOCK_A32) return pix * Bp * nb32(Ap);
+    if (block == MQC_BLOCK_B32) return pix * nb32(Bp) * Ap;
+    return pix * nb32(Bp) * nb32(Ap);
+}
+
+bool conv_ok(const mqc_conv *c) {
+    if (c == nullptr) return false;
+    if (c->N <= 0 || c->C <= 0 || c->H <= 0 || c->W <= 0 || c->K <= 0 || c->R <= 0 || c->S <= 0) return false;
+    if (c->stride_h <= 0 || c->stride_w <= 0 || c->pad_h < 0 || c->pad_w < 0) return false;
+    if (c->H + 2 * c->pad_h < c->R || c->W + 2 * c->pad_w < c->S) return false;
+    return true;
+}
+int conv_P(const mqc_conv *c) { return (c->H + 2 * c->pad_h - c->R) / c->stride_h + 1; }
+int conv_Q(const mqc_conv *c) { return (c->W + 2 * c->pad_w - c->S) / c->stride_w + 1; }
+
+// ---------------------------------------------------------------- device info
+struct DevInfo {
+    int sms = 0;
+    int max_smem = 0;
+    bool gemm_attr[2] = {false, false};
+};
+std::mutex g_dev_mu;
+DevInfo g_dev[64];
+
+mqc_status dev_info(DevInfo *&out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(MQC_ERR_CUDA, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo &d = g_dev[dev];
+    if (d.sms == 0) {
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (major != 10 || minor != 0)
+            return fail(MQC_ERR_UNSUPPORTED, "libmqc is built for sm_100a; device %d is sm_%d%d", dev, major, minor);
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+        e = cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(smem)");
+    }
+    out = &d;
+    return MQC_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+mqc_status get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode ? MQC_OK : fail(MQC_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+}
+
+// Encode a tiled map over 1-byte codes.  dims[0] is contiguous; strides are
+// the byte strides of dims[1..rank-1]; the inner box is 32*wkb bytes with the
+// matching shared-memory swizzle.
+mqc_status encode_codes_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                            const uint64_t *strides, const uint32_t *box, int wkb) {
+    mqc_status st = get_encoder();
+    if (st != MQC_OK) return st;
+    cuuint64_t gd[5], gs[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        gd[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (dims[i] == 0 || dims[i] > (1ull << 32)) return fail(MQC_ERR_INVALID, "tensor extent %llu out of range",
+                                                                (unsigned long long)dims[i]);
+        if (box[i] == 0 || box[i] > 256) return fail(MQC_ERR_INVALID, "box extent %u out of range", box[i]);
+    }
+    for (int i = 0; i < rank - 1; ++i) {
+        gs[i] = strides[i];
+        if (strides[i] % 16 != 0) return fail(MQC_ERR_ALIGNMENT, "tensor stride %llu not a multiple of 16 bytes",
+                                              (unsigned long long)strides[i]);
+    }
+    const CUtensorMapSwizzle sw = wkb == 4 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                           : (wkb == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void *>(base), gd, gs, bx, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MQC_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return MQC_OK;
+}
+
+int largest_wkb(int64_t nblocks) { return nblocks % 4 == 0 ? 4 : (nblocks % 2 == 0 ? 2 : 1); }
+
+// Output-tile geometry of the CONV kind: a box of bq x bp x bn output
+// positions (q fastest) with at most 128 rows, chosen to minimise the rows
+// computed over the whole problem, with a preference for long runs along q
+// (contiguous fp32 stores in NCHW).
+void choose_rows(int Qe, int Pe, int Ne, int &bq, int &bp, int &bn) {
+    double best = 1e300;
+    bq = bp = bn = 1;
+    for (int q = 1; q <= std::min(Qe, 128); ++q)
+        for (int n = 1; n <= std::min(Ne, 128 / q); ++n) {
+            const int pr = std::min(Pe, 128 / (q * n));
+            if (pr < 1) continue;
+            const double tiles = double(ceil_div(Qe, q)) * ceil_div(Pe, pr) * ceil_div(Ne, n);
+            double cost = tiles * 128.0;
+            const int want = std::min(32, Qe);
+            if (q < want) cost *= 1.0 + 0.25 * (1.0 - double(q) / want);
+            if (cost < best - 1e-9) {
+                best = cost;
+                bq = q;
+                bp = pr;
+                bn = n;
+            }
+        }
+}
+
+int choose_bn(int ncols) {
+    if (ncols <= 128) return static_cast<int>(round_up(ncols, 32));
+    return 128;
+}
+
+uint32_t mma_fmt(int f) { return f == MQC_E4M3 ? 0u : (f == MQC_E5M2 ? 1u : 5u); }
+
+const uint64_t kDefaultTimeoutNs = 4000000000ull;
+
+template <int KIND>
+mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
+    const int per_stage = 128 * 128 + P.BN * 128 + 512 + 512 * P.nb_atoms;
+    const int sf_cols = 4 + 4 * P.nb_atoms;
+    const int fixed = 1024 + 64 * 8 + 64;
+    int S = std::min(8, (d.max_smem - fixed) / per_stage);
+    S = std::min(S, (kTmemCols - kSfTmemBase) / sf_cols);
+    if (S < 2) return fail(MQC_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+    P.stages = S;
+    P.nacc = (P.BN <= 128) ? 2 : 1;
+    P.timeout_ns = kDefaultTimeoutNs;
+    const int smem = fixed + S * per_stage;
+    if (!d.gemm_attr[KIND]) {
+        cudaError_t e = cudaFuncSetAttribute(conv_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             d.max_smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        const_cast<DevInfo &>(d).gemm_attr[KIND] = true;
+    }
+    const int grid = std::max(1, std::min(P.num_units, d.sms));
+    conv_gemm_kernel<KIND><<<grid, kGemmThreads, smem, stream>>>(P);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "conv_gemm_kernel launch");
+    return MQC_OK;
+}
+
+// Tap of a strided operand: r - pad = st*d + phase with 0 <= phase < st.
+void split_tap(int off, int st, int &d, int &ph) {
+    ph = ((off % st) + st) % st;
+    d = (off - ph) / st;
+}
+
+bool gemm_fmt_ok(const mqc_mx *m) { return m->fmt == MQC_E4M3 || m->fmt == MQC_E5M2; }
+
+mqc_status check_gemm_operand(const char *name, const void *q, const uint8_t *s, const mqc_mx *m, int want_order,
+                              bool along_first) {
+    if (q == nullptr || s == nullptr || !mx_ok(m)) return fail(MQC_ERR_INVALID, "%s: null pointer or bad mx", name);
+    if (!aligned16(q)) return fail(MQC_ERR_ALIGNMENT, "%s codes not 16-byte aligned", name);
+    if (!gemm_fmt_ok(m)) return fail(MQC_ERR_UNSUPPORTED, "%s: only E4M3/E5M2 operands in the GEMMs of this build", name);
+    if (m->order != want_order)
+        return fail(MQC_ERR_UNSUPPORTED, "%s: code order must be %s", name, want_order == 0 ? "BA" : "AB");
+    const int want_block = along_first ? MQC_BLOCK_A32 : MQC_BLOCK_B32;
+    if (m->block != want_block && m->block != MQC_BLOCK_SQ32)
+        return fail(MQC_ERR_UNSUPPORTED, "%s: block mode must be %s or SQ32", name, along_first ? "A32" : "B32");
+    return MQC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mqc_version(void) { return 100; }
+
+const char *mqc_status_string(mqc_status s) {
+    switch (s) {
+    case MQC_OK: return "ok";
+    case MQC_ERR_INVALID: return "invalid argument";
+    case MQC_ERR_UNSUPPORTED: return "unsupported";
+    case MQC_ERR_CUDA: return "CUDA error";
+    case MQC_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case MQC_ERR_ALIGNMENT: return "misaligned pointer";
+    case MQC_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+const char *mqc_last_error_message(void) { return g_msg; }
+
+int64_t mqc_codes_bytes(const mqc_mx *mx, int32_t d0, int32_t d1, int32_t d2, int32_t d3) {
+    if (!mx_ok(mx) || d0 <= 0 || d1 <= 0 || d2 <= 0 || d3 <= 0) return -1;
+    return codes_bytes(mx->fmt, mx->order, d0, d1, d2, d3);
+}
+
+int64_t mqc_scales_bytes(const mqc_mx *mx, int32_t d0, int32_t d1, int32_t d2, int32_t d3) {
+    if (!mx_ok(mx) || d0 <= 0 || d1 <= 0 || d2 <= 0 || d3 <= 0) return -1;
+    return scales_bytes(mx->fmt, mx->block, mx->order, d0, d1, d2, d3);
+}
+
+mqc_status mqc_tensor_dims(mqc_role role, const mqc_conv *c, int32_t dims[4]) {
+    if (!conv_ok(c) || dims == nullptr) return fail(MQC_ERR_INVALID, "bad conv descriptor");
+    switch (role) {
+    case MQC_ROLE_X: dims[0] = c->N; dims[1] = c->C; dims[2] = c->H; dims[3] = c->W; return MQC_OK;
+    case MQC_ROLE_W: dims[0] = c->K; dims[1] = c->C; dims[2] = c->R; dims[3] = c->S; return MQC_OK;
+    case MQC_ROLE_G: dims[0] = c->N; dims[1] = c->K; dims[2] = conv_P(c); dims[3] = conv_Q(c); return MQC_OK;
+    }
+    return fail(MQC_ERR_INVALID, "bad role %d", (int)role);
+}
+
+// ------------------------------------------------------------------ quantize
+mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, void *codes, uint8_t *scales,
+                           void *codes_alt, void *stream) {
+    if (src == nullptr || d == nullptr || codes == nullptr || scales == nullptr || !mx_ok(mx))
+        return fail(MQC_ERR_INVALID, "quantize: null pointer or bad mx descriptor");
+    if (d->d0 <= 0 || d->d1 <= 0 || d->d2 <= 0 || d->d3 <= 0)
+        return fail(MQC_ERR_INVALID, "quantize: extents must be positive");
+    if ((reinterpret_cast<uintptr_t>(src) & 3u) != 0) return fail(MQC_ERR_ALIGNMENT, "quantize: src not 4-byte aligned");
+    if (!aligned16(codes) || (codes_alt != nullptr && !aligned16(codes_alt)))
+        return fail(MQC_ERR_ALIGNMENT, "quantize: codes not 16-byte aligned");
+    if (static_cast<int64_t>(d->d2) * d->d3 > (int64_t(1) << 31) - 64)
+        return fail(MQC_ERR_INVALID, "quantize: too many spatial positions");
+    DevInfo *dv;
+    mqc_status st = dev_info(dv);
+    if (st != MQC_OK) return st;
+
+    QuantParams p{};
+    p.src = src;
+    p.sb = d->s0;
+    p.sa = d->s1;
+    p.sh = d->s2;
+    p.sw = d->s3;
+    p.B = d->d0;
+    p.A = d->d1;
+    p.H = d->d2;
+    p.W = d->d3;
+    p.npix = d->d2 * d->d3;
+    int64_t Ap, Bp;
+    padded(mx->fmt, mx->order, p.A, p.B, Ap, Bp);
+    p.Ap1 = static_cast<int32_t>(Ap);
+    p.Bp1 = static_cast<int32_t>(Bp);
+    const bool map_a = mx->order == MQC_ORDER_BA;
+    const int64_t r = row_elems(mx->fmt);
+    p.I = map_a ? p.A : p.B;
+    p.O = map_a ? p.B : p.A;
+    p.I1 = static_cast<int32_t>(map_a ? Ap : Bp);
+    p.O1 = p.O;
+    p.codes = static_cast<uint8_t *>(codes);
+    p.codes_alt = static_cast<uint8_t *>(codes_alt);
+    p.O2 = static_cast<int32_t>(round_up(p.O, r));
+    p.scales = scales;
+    p.block = mx->block;
+    p.fmt = mx->fmt;
+    p.emax = emax_elem(mx->fmt);
+    p.nIT = static_cast<int32_t>(ceil_div(p.I1, 32));
+    p.nOT = static_cast<int32_t>(ceil_div(codes_alt ? p.O2 : p.O, 32));
+    const int64_t tiles = ceil_div(p.npix, 32) * p.nOT * p.nIT;
+    if (tiles > (int64_t(1) << 31) - 1) return fail(MQC_ERR_INVALID, "quantize: tensor too large");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool fp4 = mx->fmt == MQC_E2M1;
+    if (map_a && !fp4) mx_quantize_kernel<true, false><<<static_cast<unsigned>(tiles), 256, 0, s>>>(p);
+    else if (map_a && fp4) mx_quantize_kernel<true, true><<<static_cast<unsigned>(tiles), 256, 0, s>>>(p);
+    else if (!fp4) mx_quantize_kernel<false, false><<<static_cast<unsigned>(tiles), 256, 0, s>>>(p);
+    else mx_quantize_kernel<false, true><<<static_cast<unsigned>(tiles), 256, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "mx_quantize_kernel launch");
+    return MQC_OK;
+}
+
+// ------------------------------------------------------------------ im2col
+static void im2col_geometry(const mqc_conv *c, const mqc_mx *mx, int64_t &Ap, int64_t &Bp, int64_t &chunk_codes,
+                            int64_t &rows_codes, int64_t &chunk_sc, int64_t &rows_sc) {
+    padded(mx->fmt, mx->order, c->C, c->N, Ap, Bp);
+    const int64_t bytes_per = mx->fmt == MQC_E2M1 ? 2 : 1;   // elements per byte
+    if (mx->order == MQC_ORDER_BA) {
+        chunk_codes = Ap / bytes_per;
+        rows_codes = Bp;
+    } else {
+        chunk_codes = Ap * Bp / bytes_per;
+        rows_codes = 1;
+    }
+    if (mx->block == MQC_BLOCK_A32) {
+        rows_sc = Bp;
+        chunk_sc = nb32(Ap);
+    } else if (mx->block == MQC_BLOCK_B32) {
+        rows_sc = nb32(Bp);
+        chunk_sc = Ap;
+    } else {
+        rows_sc = nb32(Bp);
+        chunk_sc = nb32(Ap);
+    }
+}
+
+int64_t mqc_im2col_cbf_codes_bytes(const mqc_conv *c, const mqc_mx *mx) {
+    if (!conv_ok(c) || !mx_ok(mx)) return -1;
+    int64_t Ap, Bp, cc, rc, cs, rs;
+    im2col_geometry(c, mx, Ap, Bp, cc, rc, cs, rs);
+    return int64_t(conv_P(c)) * conv_Q(c) * rc * c->R * c->S * cc;
+}
+
+int64_t mqc_im2col_cbf_scales_bytes(const mqc_conv *c, const mqc_mx *mx) {
+    if (!conv_ok(c) || !mx_ok(mx)) return -1;
+    int64_t Ap, Bp, cc, rc, cs, rs;
+    im2col_geometry(c, mx, Ap, Bp, cc, rc, cs, rs);
+    return int64_t(conv_P(c)) * conv_Q(c) * rs * c->R * c->S * cs;
+}
+
+mqc_status mqc_im2col_cbf(const void *codes, const uint8_t *scales, const mqc_conv *c, const mqc_mx *mx,
+                          void *codes_out, uint8_t *scales_out, void *stream) {
+    if (codes == nullptr || scales == nullptr || codes_out == nullptr || scales_out == nullptr || !conv_ok(c) ||
+        !mx_ok(mx))
+        return fail(MQC_ERR_INVALID, "im2col: null pointer or bad descriptor");
+    if (!aligned16(codes) || !aligned16(codes_out)) return fail(MQC_ERR_ALIGNMENT, "im2col: codes not 16-byte aligned");
+    DevInfo *dv;
+    mqc_status st = dev_info(dv);
+    if (st != MQC_OK) return st;
+    int64_t Ap, Bp, cc, rc, cs, rs;
+    im2col_geometry(c, mx, Ap, Bp, cc, rc, cs, rs);
+    Im2colParams p{};
+    p.RS = c->R * c->S;
+    p.S = c->S;
+    p.P = conv_P(c);
+    p.Q = conv_Q(c);
+    p.H = c->H;
+    p.W = c->W;
+    p.st_h = c->stride_h;
+    p.st_w = c->stride_w;
+    p.pad_h = c->pad_h;
+    p.pad_w = c->pad_w;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int blocks = dv->sms * 8;
+    p.src = static_cast<const uint8_t *>(codes);
+    p.dst = static_cast<uint8_t *>(codes_out);
+    p.chunk = cc;
+    p.per_pix = rc;
+    p.n_out = int64_t(p.P) * p.Q * rc * p.RS * cc / 16;
+    im2col_gather_kernel<true><<<blocks, 256, 0, s>>>(p);
+    p.src = scales;
+    p.dst = scales_out;
+    p.chunk = cs;
+    p.per_pix = rs;
+    p.n_out = int64_t(p.P) * p.Q * rs * p.RS * cs;
+    im2col_gather_kernel<false><<<blocks, 256, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "im2col_gather_kernel launch");
+    return MQC_OK;
+}
+
+// ------------------------------------------------------------------ forward
+mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, const void *wq, const uint8_t *ws,
+                          const mqc_mx *wf, const mqc_conv *c, float *y, void *stream) {
+    if (!conv_ok(c) || y == nullptr) return fail(MQC_ERR_INVALID, "conv2d_fwd: bad conv descriptor or null output");
+    mqc_status st = check_gemm_operand("X", xq, xs, xf, MQC_ORDER_BA, true);
+    if (st != MQC_OK) return st;
+    st = check_gemm_operand("W", wq, ws, wf, MQC_ORDER_BA, true);
+    if (st != MQC_OK) return st;
+    if (c->R * c->S > kMaxTaps) return fail(MQC_ERR_UNSUPPORTED, "conv2d_fwd: at most %d kernel taps", kMaxTaps);
+    DevInfo *dv;
+    if ((st = dev_info(dv)) != MQC_OK) return st;
+
+    const int N = c->N, C = c->C, H = c->H, W = c->W, K = c->K, R = c->R, S = c->S;
+    const int sh = c->stride_h, sw = c->stride_w, P = conv_P(c), Q = conv_Q(c);
+    const int64_t Cp = round_up(C, 16);
+    GemmParams G;
+    memset(&G, 0, sizeof G);
+    G.CB = static_cast<int32_t>(nb32(Cp));
+    G.wkb = largest_wkb(G.CB);
+    choose_rows(Q, P, N, G.bq, G.bp, G.bn);
+    G.BN = choose_bn(K);
+    G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
+    G.Qe = Q;
+    G.Pe = P;
+    G.Ne = N;
+    G.TQ = static_cast<int32_t>(ceil_div(Q, G.bq));
+    G.TP = static_cast<int32_t>(ceil_div(P, G.bp));
+    G.TN = static_cast<int32_t>(ceil_div(N, G.bn));
+    G.NT = static_cast<int32_t>(ceil_div(K, G.BN));
+    G.Ncols = K;
+    G.a_st_h = sh;
+    G.a_st_w = sw;
+    G.idesc = make_idesc_mx(mma_fmt(xf->fmt), mma_fmt(wf->fmt), 128, G.BN);
+    if (sh * sw > 4) return fail(MQC_ERR_UNSUPPORTED, "conv2d_fwd: stride product above 4");
+    // A: one map per stride phase; dims (C, W', H', N) so that rows run along q
+    bool phase_ok[16] = {};
+    for (int attempt = 0; attempt < 2; ++attempt) {
+        G.rows_nfirst = attempt;
+        st = MQC_OK;
+        for (int a = 0; a < sh && st == MQC_OK; ++a)
+            for (int b = 0; b < sw && st == MQC_OK; ++b) {
+                const int64_t Hh = ceil_div(H - a, sh), Ww = ceil_div(W - b, sw);
+                phase_ok[a * sw + b] = Hh > 0 && Ww > 0;
+                if (!phase_ok[a * sw + b]) continue;
+                const uint8_t *base = static_cast<const uint8_t *>(xq) + (int64_t(a) * W + b) * N * Cp;
+                if (!G.rows_nfirst) {
+                    const uint64_t dims[4] = {uint64_t(Cp), uint64_t(Ww), uint64_t(Hh), uint64_t(N)};
+                    const uint64_t strd[3] = {uint64_t(sw) * N * Cp, uint64_t(sh) * W * N * Cp, uint64_t(Cp)};
+                    const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bq), uint32_t(G.bp), uint32_t(G.bn)};
+                    st = encode_codes_map(&G.amap[a * sw + b], base, 4, dims, strd, box, G.wkb);
+                } else {
+                    const uint64_t dims[4] = {uint64_t(Cp), uint64_t(N), uint64_t(Ww), uint64_t(Hh)};
+                    const uint64_t strd[3] = {uint64_t(Cp), uint64_t(sw) * N * Cp, uint64_t(sh) * W * N * Cp};
+                    const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bn), uint32_t(G.bq), uint32_t(G.bp)};
+                    st = encode_codes_map(&G.amap[a * sw + b], base, 4, dims, strd, box, G.wkb);
+                }
+            }
+        if (st == MQC_OK) break;
+    }
+    if (st != MQC_OK) return st;
+    {
+        const uint64_t dims[3] = {uint64_t(Cp), uint64_t(K), uint64_t(R) * S};
+        const uint64_t strd[2] = {uint64_t(Cp), uint64_t(K) * Cp};
+        const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(G.BN), 1u};
+        if ((st = encode_codes_map(&G.bmap[0], wq, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
+    }
+    G.ntaps = 0;
+    for (int r = 0; r < R; ++r)
+        for (int s = 0; s < S; ++s) {
+            int dh, ph, dw, pw;
+            split_tap(r - c->pad_h, sh, dh, ph);
+            split_tap(s - c->pad_w, sw, dw, pw);
+            ConvTap &T = G.taps[G.ntaps++];
+            T.btap = static_cast<int16_t>(r * S + s);
+            T.sf_dh = static_cast<int16_t>(r - c->pad_h);
+            T.sf_dw = static_cast<int16_t>(s - c->pad_w);
+            if (phase_ok[ph * sw + pw]) {
+                T.map = static_cast<int16_t>(ph * sw + pw);
+                T.dh = static_cast<int16_t>(dh);
+                T.dw = static_cast<int16_t>(dw);
+            } else {           // a phase with no rows: read far outside (zeros)
+                T.map = 0;
+                T.dh = T.dw = -30000;
+                T.sf_dh = T.sf_dw = -30000;
+            }
+        }
+    G.total_kb = G.ntaps * G.CB;
+    for (int i = 0; i < sh * sw; ++i)          // unused phases get a valid copy (never read)
+        if (!phase_ok[i]) G.amap[i] = G.amap[0];
+    G.n_amaps = sh * sw;
+    G.n_bmaps = 1;
+    G.a_box_bytes = 32 * G.wkb * G.bq * G.bp * G.bn;
+    G.b_box_bytes = 32 * G.wkb * G.BN;
+    const bool sqx = xf->block == MQC_BLOCK_SQ32, sqw = wf->block == MQC_BLOCK_SQ32;
+    G.sfa.base = xs;
+    G.sfa.pix_pitch = (sqx ? nb32(N) : N) * nb32(Cp);
+    G.sfa.row_div = sqx ? 32 : 1;
+    G.sfa.row_pitch = static_cast<int32_t>(nb32(Cp));
+    G.sfa.kb_pitch = 1;
+    G.sfa.rows = N;
+    G.sfa.H = H;
+    G.sfa.W = W;
+    G.sfb.base = ws;
+    G.sfb.tap_pitch = (sqw ? nb32(K) : K) * nb32(Cp);
+    G.sfb.row_div = sqw ? 32 : 1;
+    G.sfb.row_pitch = static_cast<int32_t>(nb32(Cp));
+    G.sfb.kb_pitch = 1;
+    G.sfb.rows = K;
+    G.out = y;
+    G.out_base = 0;
+    G.os_q = 1;
+    G.os_p = Q;
+    G.os_n = int64_t(K) * P * Q;
+    G.os_c = int64_t(P) * Q;
+    G.num_units = G.TQ * G.TP * G.TN * G.NT;
+    return launch_gemm<kConv>(G, *dv, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ input gradient
+mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *wf, const void *gq, const uint8_t *gs,
+                               const mqc_mx *gf, const mqc_conv *c, float *gx, void *stream) {
+    if (!conv_ok(c) || gx == nullptr) return fail(MQC_ERR_INVALID, "conv2d_bwd_data: bad conv descriptor or null output");
+    mqc_status st = check_gemm_operand("W", wq, ws, wf, MQC_ORDER_AB, false);
+    if (st != MQC_OK) return st;
+    st = check_gemm_operand("G_Y", gq, gs, gf, MQC_ORDER_BA, true);
+    if (st != MQC_OK) return st;
+    if (c->R * c->S > kMaxTaps) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_data: at most %d kernel taps", kMaxTaps);
+    DevInfo *dv;
+    if ((st = dev_info(dv)) != MQC_OK) return st;
+    const int N = c->N, C = c->C, H = c->H, W = c->W, K = c->K, R = c->R, S = c->S;
+    const int sh = c->stride_h, sw = c->stride_w, P = conv_P(c), Q = conv_Q(c);
+    const int64_t Kp = round_up(K, 16);
+    const bool sqg = gf->block == MQC_BLOCK_SQ32, sqw = wf->block == MQC_BLOCK_SQ32;
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    for (int ah = 0; ah < sh; ++ah)
+        for (int aw = 0; aw < sw; ++aw) {
+            const int Pe = static_cast<int>(ceil_div(H - ah, sh)), Qe = static_cast<int>(ceil_div(W - aw, sw));
+            if (Pe <= 0 || Qe <= 0) continue;
+            GemmParams G;
+            memset(&G, 0, sizeof G);
+            G.CB = static_cast<int32_t>(nb32(Kp));
+            G.wkb = largest_wkb(G.CB);
+            choose_rows(Qe, Pe, N, G.bq, G.bp, G.bn);
+            G.BN = choose_bn(C);
+            G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
+            G.Qe = Qe;
+            G.Pe = Pe;
+            G.Ne = N;
+            G.TQ = static_cast<int32_t>(ceil_div(Qe, G.bq));
+            G.TP = static_cast<int32_t>(ceil_div(Pe, G.bp));
+            G.TN = static_cast<int32_t>(ceil_div(N, G.bn));
+            G.NT = static_cast<int32_t>(ceil_div(C, G.BN));
+            G.Ncols = C;
+            G.a_st_h = 1;
+            G.a_st_w = 1;
+            G.idesc = make_idesc_mx(mma_fmt(gf->fmt), mma_fmt(wf->fmt), 128, G.BN);
+            st = MQC_ERR_CUDA;
+            for (int attempt = 0; attempt < 2 && st != MQC_OK; ++attempt) {
+                G.rows_nfirst = attempt;
+                if (!G.rows_nfirst) {
+                    const uint64_t dims[4] = {uint64_t(Kp), uint64_t(Q), uint64_t(P), uint64_t(N)};
+                    const uint64_t strd[3] = {uint64_t(N) * Kp, uint64_t(Q) * N * Kp, uint64_t(Kp)};
+                    const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bq), uint32_t(G.bp), uint32_t(G.bn)};
+                    st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
+                } else {
+                    const uint64_t dims[4] = {uint64_t(Kp), uint64_t(N), uint64_t(Q), uint64_t(P)};
+                    const uint64_t strd[3] = {uint64_t(Kp), uint64_t(N) * Kp, uint64_t(Q) * N * Kp};
+                    const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bn), uint32_t(G.bq), uint32_t(G.bp)};
+                    st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
+                }
+            }
+            if (st != MQC_OK) return st;
+            {
+                const uint64_t dims[3] = {uint64_t(Kp), uint64_t(C), uint64_t(R) * S};
+                const uint64_t strd[2] = {uint64_t(Kp), uint64_t(C) * Kp};
+                const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(G.BN), 1u};
+                if ((st = encode_codes_map(&G.bmap[0], wq, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
+            }
+            G.ntaps = 0;
+            for (int r = 0; r < R; ++r) {
+                if (((ah + c->pad_h - r) % sh + sh) % sh != 0) continue;
+                const int dr = (ah + c->pad_h - r) / sh;
+                for (int s = 0; s < S; ++s) {
+                    if (((aw + c->pad_w - s) % sw + sw) % sw != 0) continue;
+                    const int ds = (aw + c->pad_w - s) / sw;
+                    ConvTap &T = G.taps[G.ntaps++];
+                    T.dh = T.sf_dh = static_cast<int16_t>(dr);
+                    T.dw = T.sf_dw = static_cast<int16_t>(ds);
+                    T.map = 0;
+                    T.btap = static_cast<int16_t>(r * S + s);
+                }
+            }
+            G.total_kb = G.ntaps * G.CB;
+            G.n_amaps = 1;
+            G.n_bmaps = 1;
+            G.a_box_bytes = 32 * G.wkb * G.bq * G.bp * G.bn;
+            G.b_box_bytes = 32 * G.wkb * G.BN;
+            G.sfa.base = gs;
+            G.sfa.pix_pitch = (sqg ? nb32(N) : N) * nb32(Kp);
+            G.sfa.row_div = sqg ? 32 : 1;
+            G.sfa.row_pitch = static_cast<int32_t>(nb32(Kp));
+            G.sfa.kb_pitch = 1;
+            G.sfa.rows = N;
+            G.sfa.H = P;
+            G.sfa.W = Q;
+            G.sfb.base = ws;
+            G.sfb.tap_pitch = nb32(Kp) * (sqw ? nb32(C) : C);
+            G.sfb.row_div = sqw ? 32 : 1;
+            G.sfb.row_pitch = 1;
+            G.sfb.kb_pitch = static_cast<int32_t>(sqw ? nb32(C) : C);
+            G.sfb.rows = C;
+            G.out = gx;
+            G.out_base = int64_t(ah) * W + aw;
+            G.os_q = sw;
+            G.os_p = int64_t(sh) * W;
+            G.os_n = int64_t(C) * H * W;
+            G.os_c = int64_t(H) * W;
+            G.num_units = G.TQ * G.TP * G.TN * G.NT;
+            if ((st = launch_gemm<kConv>(G, *dv, strm)) != MQC_OK) return st;
+        }
+    return MQC_OK;
+}
+
+// ------------------------------------------------------------------ weight gradient
+static void wgrad_plan(const mqc_conv *c, const DevInfo &d, int &BN, int &splits, int64_t &kiters) {
+    const int P = conv_P(c), Q = conv_Q(c);
+    const int64_t Np = round_up(c->N, 16);
+    const int64_t NB = nb32(Np);
+    const int wkb = largest_wkb(NB);
+    const int bqk = 4 / wkb;
+    kiters = int64_t(P) * ceil_div(Q, bqk) * (NB / wkb);
+    BN = choose_bn(c->C);
+    const int64_t base = ceil_div(c->K, 128) * ceil_div(c->C, BN) * int64_t(c->R) * c->S;
+    int64_t sp = base >= d.sms ? 1 : d.sms / base;
+    sp = std::min<int64_t>(sp, std::max<int64_t>(1, kiters / 8));
+    splits = static_cast<int>(std::max<int64_t>(1, sp));
+}
+
+size_t mqc_conv2d_bwd_weight_workspace_bytes(const mqc_conv *c, const mqc_mx *gf, const mqc_mx *xf) {
+    (void)gf;
+    (void)xf;
+    if (!conv_ok(c)) return 0;
+    DevInfo *dv;
+    if (dev_info(dv) != MQC_OK) return 0;
+    int BN, splits;
+    int64_t kiters;
+    wgrad_plan(c, *dv, BN, splits, kiters);
+    if (splits <= 1) return 0;
+    return size_t(splits) * size_t(c->K) * c->C * c->R * c->S * sizeof(float);
+}
+
+mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx *gf, const void *xq,
+                                 const uint8_t *xs, const mqc_mx *xf, const mqc_conv *c, float *gw, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    if (!conv_ok(c) || gw == nullptr) return fail(MQC_ERR_INVALID, "conv2d_bwd_weight: bad conv descriptor or null output");
+    mqc_status st = check_gemm_operand("G_Y", gq, gs, gf, MQC_ORDER_AB, false);
+    if (st != MQC_OK) return st;
+    st = check_gemm_operand("X", xq, xs, xf, MQC_ORDER_AB, false);
+    if (st != MQC_OK) return st;
+    if (c->R * c->S > kMaxTaps) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_weight: at most %d kernel taps", kMaxTaps);
+    DevInfo *dv;
+    if ((st = dev_info(dv)) != MQC_OK) return st;
+    const int N = c->N, C = c->C, H = c->H, W = c->W, K = c->K, R = c->R, S = c->S;
+    const int sh = c->stride_h, sw = c->stride_w, P = conv_P(c), Q = conv_Q(c);
+    const int64_t Np = round_up(N, 16);
+    GemmParams G;
+    memset(&G, 0, sizeof G);
+    int64_t kiters;
+    if (sh * sw > 4) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_weight: stride product above 4");
+    wgrad_plan(c, *dv, G.BN, G.splits, kiters);
+    const size_t need = G.splits > 1 ? size_t(G.splits) * K * C * R * S * sizeof(float) : 0;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return fail(MQC_ERR_WORKSPACE, "conv2d_bwd_weight: needs %zu workspace bytes", need);
+    if (need > 0 && !aligned16(workspace)) return fail(MQC_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+    const int64_t NB = nb32(Np);
+    G.wkb = largest_wkb(NB);
+    G.bqk = 4 / G.wkb;
+    G.NC = static_cast<int32_t>(NB / G.wkb);
+    G.QG = static_cast<int32_t>(ceil_div(Q, G.bqk));
+    G.kiters_total = static_cast<int32_t>(kiters);
+    G.P = P;
+    G.Q = Q;
+    G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
+    G.MT = static_cast<int32_t>(ceil_div(K, 128));
+    G.NT = static_cast<int32_t>(ceil_div(C, G.BN));
+    G.Mrows = K;
+    G.Ncols = C;
+    G.x_st_h = sh;
+    G.x_st_w = sw;
+    G.idesc = make_idesc_mx(mma_fmt(gf->fmt), mma_fmt(xf->fmt), 128, G.BN);
+    {
+        const uint64_t dims[4] = {uint64_t(Np), uint64_t(K), uint64_t(Q), uint64_t(P)};
+        const uint64_t strd[3] = {uint64_t(Np), uint64_t(K) * Np, uint64_t(Q) * K * Np};
+        const uint32_t box[4] = {uint32_t(32 * G.wkb), 128u, uint32_t(G.bqk), 1u};
+        if ((st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb)) != MQC_OK) return st;
+    }
+    bool phase_ok[16] = {};
+    for (int a = 0; a < sh; ++a)
+        for (int b = 0; b < sw; ++b) {
+            const int64_t Hh = ceil_div(H - a, sh), Ww = ceil_div(W - b, sw);
+            phase_ok[a * sw + b] = Hh > 0 && Ww > 0;
+            if (!phase_ok[a * sw + b]) continue;
+            const uint8_t *base = static_cast<const uint8_t *>(xq) + (int64_t(a) * W + b) * C * Np;
+            const uint64_t dims[4] = {uint64_t(Np), uint64_t(C), uint64_t(Ww), uint64_t(Hh)};
+            const uint64_t strd[3] = {uint64_t(Np), uint64_t(sw) * C * Np, uint64_t(sh) * W * C * Np};
+            const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.BN), uint32_t(G.bqk), 1u};
+            if ((st = encode_codes_map(&G.bmap[a * sw + b], base, 4, dims, strd, box, G.wkb)) != MQC_OK) return st;
+        }
+    G.ntaps = 0;
+    for (int r = 0; r < R; ++r)
+        for (int s = 0; s < S; ++s) {
+            int dh, ph, dw, pw;
+            split_tap(r - c->pad_h, sh, dh, ph);
+            split_tap(s - c->pad_w, sw, dw, pw);
+            ConvTap &T = G.taps[G.ntaps++];
+            T.btap = static_cast<int16_t>(r * S + s);
+            T.sf_dh = static_cast<int16_t>(r - c->pad_h);
+            T.sf_dw = static_cast<int16_t>(s - c->pad_w);
+            if (phase_ok[ph * sw + pw]) {
+                T.map = static_cast<int16_t>(ph * sw + pw);
+                T.dh = static_cast<int16_t>(dh);
+                T.dw = static_cast<int16_t>(dw);
+            } else {
+                T.map = 0;
+                for (int i = 0; i < sh * sw; ++i)
+                    if (phase_ok[i]) { T.map = static_cast<int16_t>(i); break; }
+                T.dh = T.dw = -30000;
+                T.sf_dh = T.sf_dw = -30000;
+            }
+        }
+    for (int i = 0; i < sh * sw; ++i)
+        if (!phase_ok[i])
+            for (int j = 0; j < sh * sw; ++j)
+                if (phase_ok[j]) { G.bmap[i] = G.bmap[j]; break; }
+    G.n_amaps = 1;
+    G.n_bmaps = sh * sw;
+    G.a_box_bytes = 32 * G.wkb * 128 * G.bqk;
+    G.b_box_bytes = 32 * G.wkb * G.BN * G.bqk;
+    const bool sqg = gf->block == MQC_BLOCK_SQ32, sqx = xf->block == MQC_BLOCK_SQ32;
+    G.sfa.base = gs;
+    G.sfa.pix_pitch = nb32(Np) * (sqg ? nb32(K) : K);
+    G.sfa.kb_pitch = static_cast<int32_t>(sqg ? nb32(K) : K);
+    G.sfa.row_div = sqg ? 32 : 1;
+    G.sfa.row_pitch = 1;
+    G.sfa.rows = K;
+    G.sfa.H = P;
+    G.sfa.W = Q;
+    G.sfb.base = xs;
+    G.sfb.pix_pitch = nb32(Np) * (sqx ? nb32(C) : C);
+    G.sfb.kb_pitch = static_cast<int32_t>(sqx ? nb32(C) : C);
+    G.sfb.row_div = sqx ? 32 : 1;
+    G.sfb.row_pitch = 1;
+    G.sfb.rows = C;
+    G.sfb.H = H;
+    G.sfb.W = W;
+    G.out = G.splits > 1 ? static_cast<float *>(workspace) : gw;
+    G.out_base = 0;
+    G.os_m = int64_t(C) * R * S;
+    G.os_c = int64_t(R) * S;
+    G.split_pitch = int64_t(K) * C * R * S;
+    G.num_units = G.MT * G.NT * G.ntaps * G.splits;
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    if ((st = launch_gemm<kWgrad>(G, *dv, strm)) != MQC_OK) return st;
+    if (G.splits > 1) {
+        const int64_t n = int64_t(K) * C * R * S;
+        const int blocks = static_cast<int>(std::min<int64_t>(ceil_div(n, 256), int64_t(dv->sms) * 8));
+        splitk_reduce_kernel<<<blocks, 256, 0, strm>>>(static_cast<const float *>(workspace), gw, n, G.splits);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "splitk_reduce_kernel launch");
+    }
+    return MQC_OK;
+}
+
+// ------------------------------------------------------------------ status
+mqc_status mqc_get_device_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, g_mqc_device_error, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+    if (v != 0) {
+        e = cudaMemcpyToSymbol(g_mqc_device_error, &zero, sizeof zero);
+        if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+        return fail(MQC_ERR_DEVICE_TIMEOUT, "a kernel-side wait ran out of time (device error %d)", v);
+    }
+    return MQC_OK;
+}
+
+mqc_status mqc_debug_expire_wait(int64_t limit_ns, void *stream) {
+    if (limit_ns < 1000 || limit_ns > 10000000000ll) return fail(MQC_ERR_INVALID, "limit_ns out of range");
+    DevInfo *dv;
+    mqc_status st = dev_info(dv);
+    if (st != MQC_OK) return st;
+    expire_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "expire_wait_kernel launch");
+    return MQC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,151 @@
+"""Parity of the block-scaled tensor-core convolutions with the oracle.
+
+The CUDA path quantizes the fp32 inputs with its own quantizer and runs its
+GEMM; the oracle quantizes the same inputs, dequantizes them and evaluates
+Eq. 1-3 directly in double, with sum |a*b| alongside.  Every output element
+must satisfy |err| <= 1e-3 * sum|a*b| + 1e-6.
+"""
+import numpy as np
+import pytest
+
+import synth
+
+pytestmark = pytest.mark.gpu
+RTOL, ATOL = 1e-3, 1e-6
+
+
+@pytest.fixture(scope="module")
+def mqc():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import im2col_gemm_b200
+    return im2col_gemm_b200
+
+
+def _dev(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _host(t):
+    import torch
+    torch.cuda.synchronize()
+    return t.cpu().numpy().astype(np.float64)
+
+
+def _check(name, got, ref, refabs):
+    err = np.abs(got - ref)
+    bound = RTOL * refabs + ATOL
+    bad = ~(err <= bound)
+    if bad.any():
+        idx = np.argwhere(bad)
+        first = [tuple(int(v) for v in i) for i in idx[:6]]
+        vals = [(float(got[tuple(i)]), float(ref[tuple(i)])) for i in idx[:6]]
+        raise AssertionError(f"{name}: {bad.sum()} of {bad.size} outside tolerance; max err/bound "
+                             f"{float((err / bound).max()):.3g}; first {first} got/want {vals}")
+
+
+# (N, C, H, W, K, R, S, stride, pad)
+FWD_CASES = [
+    (2, 32, 8, 8, 32, 3, 3, 1, 1),        # the single-conv workload
+    (64, 64, 4, 4, 64, 1, 1, 1, 0),       # plain GEMM: 1x1 conv
+    (4, 48, 9, 11, 40, 3, 3, 2, 1),       # ragged, stride 2
+    (16, 16, 20, 20, 32, 3, 3, 2, 1),     # C = 16 (half a block), stride 2
+    (3, 128, 10, 9, 160, 3, 3, 1, 1),     # two column tiles, 4-block boxes
+    (8, 96, 7, 6, 256, 1, 1, 1, 0),       # C with 3 blocks
+    (5, 32, 12, 12, 24, 2, 3, 1, 0),      # non-square kernel, K < 32
+]
+
+
+@pytest.mark.parametrize("case", FWD_CASES)
+@pytest.mark.parametrize("blocks", [(0, 0), (2, 2)])
+def test_conv_fwd_parity(mqc, orc, case, blocks):
+    N, C, H, W, K, R, S, st, pad = case
+    bx, bw = blocks
+    x = synth.random_tensor((N, C, H, W), seed=700 + N + C, dist="student_t")
+    w = synth.random_tensor((K, C, R, S), seed=701 + K, scale=0.05)
+    fx, fw = 0, (1 if (K // 8) % 2 else 0)
+    cv = mqc.conv_desc(N, C, H, W, K, R, S, st, pad)
+    y = mqc.conv2d_fwd(mqc.quantize_mx(_dev(x), fx, bx, 0), mqc.quantize_mx(_dev(w), fw, bw, 0), cv)
+    xd = orc.dequantize(*orc.quantize(x, fx, bx, 0), x.shape, fx, bx, 0)
+    wd = orc.dequantize(*orc.quantize(w, fw, bw, 0), w.shape, fw, bw, 0)
+    ref, refabs = orc.conv_fwd(xd, wd, st, st, pad, pad)
+    _check(f"fwd {case} blocks {blocks}", _host(y), ref, refabs)
+
+
+BWD_CASES = [
+    (2, 32, 8, 8, 32, 3, 3, 1, 1),
+    (32, 64, 6, 5, 64, 1, 1, 1, 0),
+    (4, 40, 9, 11, 48, 3, 3, 2, 1),
+    (16, 16, 12, 12, 32, 3, 3, 2, 1),
+    (40, 96, 5, 6, 130, 3, 3, 1, 1),
+    (64, 32, 6, 6, 32, 3, 3, 1, 0),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES)
+@pytest.mark.parametrize("sq", [False, True])
+def test_conv_bwd_data_parity(mqc, orc, case, sq):
+    N, C, H, W, K, R, S, st, pad = case
+    P, Q = orc.out_hw(H, W, R, S, st, st, pad, pad)
+    w = synth.random_tensor((K, C, R, S), seed=801 + K, scale=0.05)
+    g = synth.random_tensor((N, K, P, Q), seed=802 + N, scale=1e-3)
+    bw, bg = (2, 2) if sq else (1, 0)
+    cv = mqc.conv_desc(N, C, H, W, K, R, S, st, pad)
+    gx = mqc.conv2d_bwd_data(mqc.quantize_mx(_dev(w), 0, bw, 1), mqc.quantize_mx(_dev(g), 1, bg, 0), cv)
+    wd = orc.dequantize(*orc.quantize(w, 0, bw, 1), w.shape, 0, bw, 1)
+    gd = orc.dequantize(*orc.quantize(g, 1, bg, 0), g.shape, 1, bg, 0)
+    ref, refabs = orc.conv_dgrad(wd, gd, H, W, st, st, pad, pad)
+    _check(f"dgrad {case} sq={sq}", _host(gx), ref, refabs)
+
+
+@pytest.mark.parametrize("case", BWD_CASES)
+@pytest.mark.parametrize("sq", [False, True])
+def test_conv_bwd_weight_parity(mqc, orc, case, sq):
+    N, C, H, W, K, R, S, st, pad = case
+    P, Q = orc.out_hw(H, W, R, S, st, st, pad, pad)
+    x = synth.random_tensor((N, C, H, W), seed=901 + C, dist="student_t")
+    g = synth.random_tensor((N, K, P, Q), seed=902 + K, scale=1e-3)
+    b = 2 if sq else 1
+    cv = mqc.conv_desc(N, C, H, W, K, R, S, st, pad)
+    gw = mqc.conv2d_bwd_weight(mqc.quantize_mx(_dev(g), 1, b, 1), mqc.quantize_mx(_dev(x), 0, b, 1), cv)
+    gd = orc.dequantize(*orc.quantize(g, 1, b, 1), g.shape, 1, b, 1)
+    xd = orc.dequantize(*orc.quantize(x, 0, b, 1), x.shape, 0, b, 1)
+    ref, refabs = orc.conv_wgrad(gd, xd, R, S, st, st, pad, pad)
+    _check(f"wgrad {case} sq={sq}", _host(gw), ref, refabs)
+
+
+def test_training_step_shares_one_quantization(mqc, orc):
+    """SQ32: each tensor is quantized once, in both code orders, and the
+    three GEMMs read those copies (paper, section IV-B: quantized once)."""
+    N, C, H, W, K, R, S, st, pad = 32, 64, 10, 10, 96, 3, 3, 1, 1
+    P, Q = orc.out_hw(H, W, R, S, st, st, pad, pad)
+    x = synth.random_tensor((N, C, H, W), seed=11, dist="student_t")
+    w = synth.random_tensor((K, C, R, S), seed=12, scale=0.02)
+    g = synth.random_tensor((N, K, P, Q), seed=13, scale=1e-3)
+    cv = mqc.conv_desc(N, C, H, W, K, R, S, st, pad)
+    xq = mqc.quantize_mx(_dev(x), 0, 2, 0, both_orders=True)
+    wq = mqc.quantize_mx(_dev(w), 0, 2, 0, both_orders=True)
+    gq = mqc.quantize_mx(_dev(g), 1, 2, 0, both_orders=True)
+    y = mqc.conv2d_fwd(xq, wq, cv)
+    gx = mqc.conv2d_bwd_data(wq.other_order(), gq, cv)
+    gw = mqc.conv2d_bwd_weight(gq.other_order(), xq.other_order(), cv)
+    xd = orc.dequantize(*orc.quantize(x, 0, 2, 0), x.shape, 0, 2, 0)
+    wd = orc.dequantize(*orc.quantize(w, 0, 2, 0), w.shape, 0, 2, 0)
+    gd = orc.dequantize(*orc.quantize(g, 1, 2, 0), g.shape, 1, 2, 0)
+    _check("step fwd", _host(y), *orc.conv_fwd(xd, wd, st, st, pad, pad))
+    _check("step dgrad", _host(gx), *orc.conv_dgrad(wd, gd, H, W, st, st, pad, pad))
+    _check("step wgrad", _host(gw), *orc.conv_wgrad(gd, xd, R, S, st, st, pad, pad))
+
+
+def test_device_wait_timeout_is_reported(mqc):
+    """A bounded kernel-side wait that runs out sets the device error flag; the
+    host reads and clears it and the context stays usable."""
+    import torch
+    assert mqc.get_device_status() == 0
+    mqc.debug_expire_wait(2_000_000)          # 2 ms
+    assert mqc.get_device_status() == -4
+    assert mqc.get_device_status() == 0
+    t = torch.ones(4, device="cuda")
+    assert float(t.sum()) == 4.0

@@ -31,7 +31,9 @@ STATUS = {0: "MQC_OK", -1: "MQC_ERR_INVALID", -2: "MQC_ERR_UNSUPPORTED", -3: "MQ
 EXPORTS = ("mqc_codes_bytes", "mqc_scales_bytes", "mqc_tensor_dims", "mqc_quantize_mx", "mqc_im2col_cbf",
            "mqc_im2col_cbf_scales_bytes", "mqc_im2col_cbf_codes_bytes", "mqc_conv2d_fwd", "mqc_conv2d_bwd_data",
            "mqc_conv2d_bwd_weight", "mqc_conv2d_bwd_weight_workspace_bytes", "mqc_get_device_status",
-           "mqc_debug_expire_wait", "mqc_status_string", "mqc_last_error_message", "mqc_version")
+           "mqc_debug_expire_wait", "mqc_status_string", "mqc_last_error_message", "mqc_version",
+           "mqc_conv2d_bwd_weight_noalloc")
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class MqcError(RuntimeError):
@@ -73,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "mqc_conv2d_bwd_data": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp]),
         "mqc_conv2d_bwd_weight": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp, sz, vp]),
         "mqc_conv2d_bwd_weight_workspace_bytes": (sz, [P(Conv), P(MX), P(MX)]),
+        "mqc_conv2d_bwd_weight_noalloc": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp]),
         "mqc_get_device_status": (i32, [vp]),
         "mqc_debug_expire_wait": (i32, [i64, vp]),
         "mqc_status_string": (ctypes.c_char_p, [i32]),
@@ -130,6 +133,13 @@ def mqc_conv2d_bwd_weight(gq, gs, gf: MX, xq, xs, xf: MX, conv: Conv, gw, worksp
 
 def mqc_conv2d_bwd_weight_workspace_bytes(conv: Conv, gf: MX, xf: MX) -> int:
     return lib.mqc_conv2d_bwd_weight_workspace_bytes(ctypes.byref(conv), ctypes.byref(gf), ctypes.byref(xf))
+
+
+def mqc_conv2d_bwd_weight_noalloc(gq, gs, gf: MX, xq, xs, xf: MX, conv: Conv, gw, stream) -> int:
+    """Weight gradient with the library's static split-K scratch: no workspace
+    argument and no allocation (see include/mqc.h)."""
+    return lib.mqc_conv2d_bwd_weight_noalloc(gq, gs, ctypes.byref(gf), xq, xs, ctypes.byref(xf),
+                                             ctypes.byref(conv), gw, stream)
 
 
 def mqc_get_device_status(stream) -> int:

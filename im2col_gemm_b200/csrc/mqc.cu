@@ -792,6 +792,49 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     return MQC_OK;
 }
 
+// ------------------------------------------------------------------ weight gradient, no allocation
+// Split-K scratch owned by the library: one copy per device, alive until the
+// process exits.  Host code must not use the symbol itself as a device
+// address; it looks the address up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MQC_NOALLOC_SCRATCH_BYTES];
+
+static std::mutex g_noalloc_mu;
+static void *g_noalloc_ptr[64];
+
+mqc_status mqc_conv2d_bwd_weight_noalloc(const void *gq, const uint8_t *gs, const mqc_mx *gf, const void *xq,
+                                         const uint8_t *xs, const mqc_mx *xf, const mqc_conv *c, float *gw,
+                                         void *stream) {
+    if (!conv_ok(c) || gw == nullptr)
+        return fail(MQC_ERR_INVALID, "conv2d_bwd_weight_noalloc: bad conv descriptor or null output");
+    mqc_status st = check_gemm_operand("G_Y", gq, gs, gf, MQC_ORDER_AB, false);
+    if (st != MQC_OK) return st;
+    st = check_gemm_operand("X", xq, xs, xf, MQC_ORDER_AB, false);
+    if (st != MQC_OK) return st;
+    const size_t need = mqc_conv2d_bwd_weight_workspace_bytes(c, gf, xf);
+    if (need > MQC_NOALLOC_SCRATCH_BYTES)
+        return fail(MQC_ERR_WORKSPACE,
+                    "conv2d_bwd_weight_noalloc: needs %zu bytes of split-K scratch, above the %u-byte static "
+                    "maximum; use mqc_conv2d_bwd_weight with a workspace",
+                    need, MQC_NOALLOC_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    if (need > 0) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+        if (dev < 0 || dev >= 64) return fail(MQC_ERR_CUDA, "device ordinal %d out of range", dev);
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (g_noalloc_ptr[dev] == nullptr) {
+            void *p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(split-K scratch)");
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    return mqc_conv2d_bwd_weight(gq, gs, gf, xq, xs, xf, c, gw, scratch, scratch ? MQC_NOALLOC_SCRATCH_BYTES : 0,
+                                 stream);
+}
+
 // ------------------------------------------------------------------ status
 mqc_status mqc_get_device_status(void *stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -186,6 +186,36 @@ MQC_API mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, cons
                                  void *workspace, size_t workspace_bytes, void *stream);
 MQC_API size_t mqc_conv2d_bwd_weight_workspace_bytes(const mqc_conv *conv, const mqc_mx *gf, const mqc_mx *xf);
 
+/* Size of the library's own split-K scratch array used by
+ * mqc_conv2d_bwd_weight_noalloc (16 MiB, held on every GPU that loads the
+ * library until the process exits). */
+#define MQC_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* Weight gradient that allocates nothing and takes no workspace.  (The paper
+ * has no counterpart: this is a deployment convenience of this library.)
+ * Same arguments, operand requirements and result as mqc_conv2d_bwd_weight,
+ * but the split-K partial sums go to a fixed array inside the library
+ * instead of caller memory.  It is meant for callers that cannot call
+ * cudaMalloc or hand out scratch at the call site: plugin hosts whose device
+ * memory is owned by someone else and frozen after start-up, and
+ * latency-critical loops that cannot afford an allocation (and the device
+ * synchronization cudaMalloc may imply) per call.
+ *   - The first call on each device looks up that device's copy of the array
+ *     (with the device current) and caches its address; make that first call
+ *     before any stream capture.
+ *   - A problem whose split-K scratch (mqc_conv2d_bwd_weight_workspace_bytes)
+ *     exceeds MQC_NOALLOC_SCRATCH_BYTES is rejected with MQC_ERR_WORKSPACE
+ *     and nothing is launched.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's partial sums; each call overwrites every partial it later reads,
+ *     so nothing needs to start at zero.  Calls that can overlap on the GPU
+ *     (different streams, or different host threads) race on the array and
+ *     must be serialized by the caller.
+ * Errors: as mqc_conv2d_bwd_weight. */
+MQC_API mqc_status mqc_conv2d_bwd_weight_noalloc(const void *gq, const uint8_t *gs, const mqc_mx *gf,
+                                         const void *xq, const uint8_t *xs, const mqc_mx *xf,
+                                         const mqc_conv *conv, float *gw, void *stream);
+
 /* Synchronizes `stream`, then reads and clears the device error flag set by a
  * bounded wait that ran out.  MQC_OK if none; MQC_ERR_DEVICE_TIMEOUT if one
  * did; MQC_ERR_CUDA if the synchronization itself failed. */

@@ -60,23 +60,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint (ns): the thread sleeps until the phase
+// completes or the hint elapses, whichever comes first.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed, for at most
-// `limit_ns` nanoseconds.  Gives up early when *abort becomes non-zero (some
-// other role of the CTA already gave up).  On running out it records
-// kDevTimeout in the device error word, raises *abort and returns false.
+// about `limit_ns` nanoseconds (measured with the SM clock, taken as <= 2 GHz).
+// Gives up early when *abort becomes non-zero (some other role of the CTA
+// already gave up).  On running out it records kDevTimeout in the device
+// error word, raises *abort and returns false.  The common case (phase
+// already complete) costs one try_wait.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns,
                                           volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 31u) == 0) {
-            if (abort != nullptr && *abort) return false;
-            if (globaltimer_ns() - t0 > limit_ns) {
-                record_device_error(kDevTimeout);
-                if (abort != nullptr) *abort = 1;
-                return false;
-            }
+    const long long c0 = clock64();
+    const long long lim = static_cast<long long>(limit_ns) * 2;
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+        if (abort != nullptr && *abort) return false;
+        if (clock64() - c0 > lim) {
+            record_device_error(kDevTimeout);
+            if (abort != nullptr) *abort = 1;
+            return false;
         }
     }
 }

@@ -148,12 +148,25 @@ __device__ __forceinline__ uint32_t swizzle_of(int wkb) {
     return wkb == 4 ? kSwizzle128B : (wkb == 2 ? kSwizzle64B : kSwizzle32B);
 }
 
+// Walks K-blocks g = 0, 1, 2, ... of a CONV tile as (tap, channel block)
+// without divisions.
+struct KbWalker {
+    int tap, cb;
+    __device__ __forceinline__ void advance(int n, int CB) {
+        cb += n;
+        while (cb >= CB) {
+            cb -= CB;
+            ++tap;
+        }
+    }
+};
+
 template <int KIND>
 __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int S = p.stages;
+    const int S = p.stages;                 // at least 4
     const int a_stage = 128 * 128;
     const int b_stage = p.BN * 128;
     const int sfb_stage = 512 * p.nb_atoms;
@@ -199,17 +212,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     const uint32_t tmem = *tmem_holder;
     const uint64_t lim = p.timeout_ns;
     const int sf_cols = 4 + 4 * p.nb_atoms;
+    const int row_bytes = 32 * p.wkb;          // bytes of one operand row of a TMA box
+    const int lg_wkb = p.wkb == 4 ? 2 : (p.wkb == 2 ? 1 : 0);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             uint32_t it = 0;
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
                 const UnitInfo I = decode_unit<KIND>(p, u);
-                for (int ki = 0; ki < I.nk; ++ki, ++it) {
-                    const int s = static_cast<int>(it % S);
-                    const uint32_t ph = (it / S) & 1u;
+                KbWalker kw{0, 0};
+                int kg = I.kbase, nc = 0, qg = 0, pp = 0;
+                if (KIND == kWgrad) {
+                    nc = kg % p.NC;
+                    qg = (kg / p.NC) % p.QG;
+                    pp = kg / (p.NC * p.QG);
+                }
+                for (int ki = 0; ki < I.nk; ++ki, ++it, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) {
                         ok = false;
                         break;
@@ -218,34 +240,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     uint8_t *b_dst = sB + s * b_stage;
                     if (KIND == kConv) {
                         const int nkb = min(4, p.total_kb - 4 * ki);
-                        const int nbox = (nkb + p.wkb - 1) / p.wkb;
+                        const int nbox = nkb >> lg_wkb;
                         mbar_arrive_expect_tx(&full_tma[s],
                                               static_cast<uint32_t>(nbox * (p.a_box_bytes + p.b_box_bytes)));
                         for (int j = 0; j < nbox; ++j) {
-                            const int g = 4 * ki + j * p.wkb;
-                            const int tap = g / p.CB;
-                            const int cb = g % p.CB;
-                            const ConvTap T = p.taps[tap];
-                            const int cx = cb * 32;
+                            const ConvTap T = p.taps[kw.tap];
+                            const int cx = kw.cb * 32;
                             if (p.rows_nfirst)
-                                tma_load_4d(a_dst + j * 128 * 32 * p.wkb, &p.amap[T.map], &full_tma[s], cx, I.n0,
+                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full_tma[s], cx, I.n0,
                                             I.q0 + T.dw, I.p0 + T.dh);
                             else
-                                tma_load_4d(a_dst + j * 128 * 32 * p.wkb, &p.amap[T.map], &full_tma[s], cx,
+                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full_tma[s], cx,
                                             I.q0 + T.dw, I.p0 + T.dh, I.n0);
-                            tma_load_3d(b_dst + j * p.BN * 32 * p.wkb, &p.bmap[0], &full_tma[s], cx, I.col0,
-                                        T.btap);
+                            tma_load_3d(b_dst + j * p.BN * row_bytes, &p.bmap[0], &full_tma[s], cx, I.col0, T.btap);
+                            kw.advance(p.wkb, p.CB);
                         }
                     } else {
-                        const int kg = I.kbase + ki;
-                        const int nc = kg % p.NC;
-                        const int qg = (kg / p.NC) % p.QG;
-                        const int pp = kg / (p.NC * p.QG);
                         const ConvTap T = p.taps[I.tap];
                         mbar_arrive_expect_tx(&full_tma[s], static_cast<uint32_t>(p.a_box_bytes + p.b_box_bytes));
-                        const int nx = nc * 32 * p.wkb;
+                        const int nx = nc * row_bytes;
                         tma_load_4d(a_dst, &p.amap[0], &full_tma[s], nx, I.m0, qg * p.bqk, pp);
                         tma_load_4d(b_dst, &p.bmap[T.map], &full_tma[s], nx, I.col0, qg * p.bqk + T.dw, pp + T.dh);
+                        if (++nc == p.NC) {
+                            nc = 0;
+                            if (++qg == p.QG) {
+                                qg = 0;
+                                ++pp;
+                            }
+                        }
                     }
                 }
             }
@@ -259,21 +281,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            uint32_t it = 0, tcount = 0;
+            uint32_t tcount = 0;
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = true;
             const uint32_t swz = swizzle_of(p.wkb);
-            const uint32_t row_bytes = 32u * p.wkb;
+            // descriptors of stage 0, sub-tile 0; other positions add (byte offset >> 4)
+            const uint64_t adesc0 = make_smem_desc(smem_u32(sA), 16, 8 * row_bytes, swz);
+            const uint64_t bdesc0 = make_smem_desc(smem_u32(sB), 16, 8 * row_bytes, swz);
+            const uint64_t sfa_desc0 = make_smem_desc(smem_u32(sSFA), 0, 128, kSwizzleNone);
+            const uint64_t sfb_desc0 = make_smem_desc(smem_u32(sSFB), 0, 128, kSwizzleNone);
+            const uint32_t a_sub = (128 * row_bytes) >> 4, b_sub = (p.BN * row_bytes) >> 4;
             for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
                 const UnitInfo I = decode_unit<KIND>(p, u);
                 if (I.nk == 0) continue;
-                const uint32_t acc = tcount % p.nacc;
-                const uint32_t aph = (tcount / p.nacc) & 1u;
+                const uint32_t acc = tcount & 1u & static_cast<uint32_t>(p.nacc - 1);
+                const uint32_t aph = (p.nacc == 2 ? (tcount >> 1) : tcount) & 1u;
                 if (!mbar_wait(&acc_empty[acc], aph ^ 1u, lim, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + acc * p.BN;
-                for (int ki = 0; ki < I.nk; ++ki, ++it) {
-                    const int s = static_cast<int>(it % S);
-                    const uint32_t ph = (it / S) & 1u;
+                for (int ki = 0; ki < I.nk; ++ki, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
                     if (!mbar_wait(&full_tma[s], ph, lim, abort_flag) || !mbar_wait(&full_sf[s], ph, lim, abort_flag)) {
                         ok = false;
                         break;
@@ -281,23 +308,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     tc_fence_after();
                     const uint32_t sfa_t = tmem + kSfTmemBase + s * sf_cols;
                     const uint32_t sfb_t = sfa_t + 4;
-                    tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(smem_u32(sSFA + s * 512), 0, 128, kSwizzleNone));
+                    tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + static_cast<uint64_t>((s * 512) >> 4));
                     for (int a = 0; a < p.nb_atoms; ++a)
-                        tc_cp_32x128b_warpx4(sfb_t + 4 * a, make_smem_desc(smem_u32(sSFB + s * sfb_stage + a * 512),
-                                                                           0, 128, kSwizzleNone));
+                        tc_cp_32x128b_warpx4(sfb_t + 4 * a,
+                                             sfb_desc0 + static_cast<uint64_t>((s * sfb_stage + a * 512) >> 4));
                     const int nkb = KIND == kConv ? min(4, p.total_kb - 4 * ki) : 4;
-                    const uint32_t a_base = smem_u32(sA + s * a_stage);
-                    const uint32_t b_base = smem_u32(sB + s * b_stage);
+                    const uint64_t a_s = adesc0 + static_cast<uint64_t>((s * a_stage) >> 4);
+                    const uint64_t b_s = bdesc0 + static_cast<uint64_t>((s * b_stage) >> 4);
                     for (int kb = 0; kb < nkb; ++kb) {
-                        const int j = kb / p.wkb, within = kb % p.wkb;
-                        const uint64_t adesc =
-                            make_smem_desc(a_base + j * 128 * row_bytes + within * 32, 16, 8 * row_bytes, swz);
-                        const uint64_t bdesc =
-                            make_smem_desc(b_base + j * p.BN * row_bytes + within * 32, 16, 8 * row_bytes, swz);
-                        const uint32_t idesc = p.idesc | (static_cast<uint32_t>(kb) << 29) |
-                                               (static_cast<uint32_t>(kb) << 4);
-                        tc_mma_mxf8f6f4(d_tmem, adesc, bdesc, idesc, sfa_t | (static_cast<uint32_t>(kb) << 30),
-                                        sfb_t | (static_cast<uint32_t>(kb) << 30), (ki > 0 || kb > 0) ? 1u : 0u);
+                        const uint32_t j = static_cast<uint32_t>(kb >> lg_wkb);
+                        const uint32_t within = static_cast<uint32_t>(kb & (p.wkb - 1));
+                        const uint64_t adesc = a_s + j * a_sub + within * 2;
+                        const uint64_t bdesc = b_s + j * b_sub + within * 2;
+                        const uint32_t kbu = static_cast<uint32_t>(kb);
+                        tc_mma_mxf8f6f4(d_tmem, adesc, bdesc, p.idesc | (kbu << 29) | (kbu << 4), sfa_t | (kbu << 30),
+                                        sfb_t | (kbu << 30), (ki > 0 || kb > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                 }
@@ -308,11 +333,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         }
     } else if (warp < 6) {
         // ------------------------------------------------------------ scale-factor gather
+        // warp 2+w handles the stages whose global index is w modulo 4
         const int sfw = warp - 2;
-        uint32_t it = 0;
+        uint32_t it = 0;             // global index of the first stage of the unit
+        uint32_t g = static_cast<uint32_t>(sfw);   // global index of this warp's next stage
+        int s = sfw % S;
+        uint32_t ph = static_cast<uint32_t>(sfw / S) & 1u;
         bool ok = true;
         for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
+            const uint32_t it_unit = it;
+            it += static_cast<uint32_t>(I.nk);
+            if (g >= it) continue;
+            const int first = static_cast<int>(g - it_unit);
             // A rows of this lane: m = lane + 32 j
             int ra_h[4], ra_w[4], ra_off[4];
             bool ra_ok[4];
@@ -335,46 +368,61 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     ra_off[j] = (k / p.sfa.row_div) * p.sfa.row_pitch;
                 }
             }
-            for (int ki = 0; ki < I.nk; ++ki, ++it) {
-                if (static_cast<int>(it & 3u) != sfw) continue;
-                const int s = static_cast<int>(it % S);
-                const uint32_t ph = (it / S) & 1u;
+            // B rows of this lane: col0 + 128 at + 32 j + lane
+            int rb_off[2][4];
+            bool rb_ok[2][4];
+#pragma unroll
+            for (int at = 0; at < 2; ++at)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int rl = 128 * at + 32 * j + lane;
+                    const int r = I.col0 + rl;
+                    rb_ok[at][j] = at < p.nb_atoms && rl < p.BN && r < p.sfb.rows;
+                    rb_off[at][j] = (r / p.sfb.row_div) * p.sfb.row_pitch;
+                }
+            KbWalker kw{0, 0};
+            if (KIND == kConv) kw.advance(4 * first, p.CB);
+            int kg = I.kbase + first;
+            int nc = 0, qg = 0, pp = 0;
+            if (KIND == kWgrad) {
+                nc = kg % p.NC;
+                qg = (kg / p.NC) % p.QG;
+                pp = kg / (p.NC * p.QG);
+            }
+            for (int ki = first; ki < I.nk; ki += 4) {
                 uint32_t wa[4] = {0u, 0u, 0u, 0u};      // A atom bytes: row lane+32j, byte kb
                 uint32_t wb[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
                 if (KIND == kConv) {
                     const int nkb = min(4, p.total_kb - 4 * ki);
+                    KbWalker k2 = kw;
                     for (int kb = 0; kb < nkb; ++kb) {
-                        const int g = 4 * ki + kb;
-                        const int tap = g / p.CB, cb = g % p.CB;
-                        const ConvTap T = p.taps[tap];
+                        const ConvTap T = p.taps[k2.tap];
+                        const int cb = k2.cb;
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
                             if (ra_ok[j] && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W) {
-                                const uint8_t *src = p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
+                                const uint8_t *src = p.sfa.base +
+                                                     (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
                                                      ra_off[j] + cb * p.sfa.kb_pitch;
                                 wa[j] |= static_cast<uint32_t>(__ldg(src)) << (8 * kb);
                             }
                         }
-                        const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
-                        for (int at = 0; at < p.nb_atoms; ++at)
+                        const uint8_t *bsrc =
+                            p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const int r = I.col0 + 128 * at + 32 * j + lane;
-                                if (128 * at + 32 * j + lane < p.BN && r < p.sfb.rows)
-                                    wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + (r / p.sfb.row_div) * p.sfb.row_pitch))
-                                                 << (8 * kb);
-                            }
+                        for (int at = 0; at < 2; ++at)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                if (rb_ok[at][j]) wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                        k2.advance(1, p.CB);
                     }
+                    kw.advance(16, p.CB);
                 } else {
-                    const int kg = I.kbase + ki;
-                    const int nc = kg % p.NC;
-                    const int qg = (kg / p.NC) % p.QG;
-                    const int pp = kg / (p.NC * p.QG);
                     const ConvTap T = p.taps[I.tap];
                     for (int kb = 0; kb < 4; ++kb) {
-                        const int q = qg * p.bqk + kb / p.wkb;
-                        const int nb = nc * p.wkb + kb % p.wkb;
+                        const int q = qg * p.bqk + (kb >> lg_wkb);
+                        const int nb = nc * p.wkb + (kb & (p.wkb - 1));
                         if (q >= p.Q) continue;
                         const uint8_t *asrc = p.sfa.base + (static_cast<int64_t>(pp) * p.Q + q) * p.sfa.pix_pitch +
                                               nb * p.sfa.kb_pitch;
@@ -385,27 +433,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         if (hh < 0 || hh >= p.sfb.H || ww < 0 || ww >= p.sfb.W) continue;
                         const uint8_t *bsrc = p.sfb.base + (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
                                               nb * p.sfb.kb_pitch;
-                        for (int at = 0; at < p.nb_atoms; ++at)
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const int r = I.col0 + 128 * at + 32 * j + lane;
-                                if (128 * at + 32 * j + lane < p.BN && r < p.sfb.rows)
-                                    wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + (r / p.sfb.row_div) * p.sfb.row_pitch))
-                                                 << (8 * kb);
-                            }
+                        for (int at = 0; at < 2; ++at)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                if (rb_ok[at][j]) wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
                     }
+                    // advance the (pixel row, q-group, n-chunk) walker by 4 K iterations
+                    for (int step = 0; step < 4; ++step)
+                        if (++nc == p.NC) {
+                            nc = 0;
+                            if (++qg == p.QG) {
+                                qg = 0;
+                                ++pp;
+                            }
+                        }
                 }
                 if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) {
                     ok = false;
                     break;
                 }
                 *reinterpret_cast<uint4 *>(sSFA + s * 512 + lane * 16) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-                for (int at = 0; at < p.nb_atoms; ++at)
-                    *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + at * 512 + lane * 16) =
-                        make_uint4(wb[at][0], wb[at][1], wb[at][2], wb[at][3]);
+                *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + lane * 16) = make_uint4(wb[0][0], wb[0][1], wb[0][2], wb[0][3]);
+                if (p.nb_atoms > 1)
+                    *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + 512 + lane * 16) =
+                        make_uint4(wb[1][0], wb[1][1], wb[1][2], wb[1][3]);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_sf[s]);
+                g += 4;
+                s += 4;
+                while (s >= S) {
+                    s -= S;
+                    ph ^= 1u;
+                }
             }
         }
     } else {
@@ -433,21 +494,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     for (int c = I.col0; c < min(I.col0 + p.BN, p.Ncols); ++c) p.out[row_off + c * p.os_c] = 0.0f;
                 continue;
             }
-            const uint32_t acc = tcount % p.nacc;
-            const uint32_t aph = (tcount / p.nacc) & 1u;
+            const uint32_t acc = tcount & 1u & static_cast<uint32_t>(p.nacc - 1);
+            const uint32_t aph = (p.nacc == 2 ? (tcount >> 1) : tcount) & 1u;
             if (!mbar_wait(&acc_full[acc], aph, lim, abort_flag)) break;
             tc_fence_after();
             const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16) + acc * p.BN;
+            float *orow = p.out + row_off;
             for (int c16 = 0; c16 < p.BN / 16; ++c16) {
                 uint32_t r[16];
                 tc_ld_32x32b_x16(t_row + c16 * 16, r);
                 tc_wait_ld();
                 if (row_ok) {
+                    const int c0 = I.col0 + c16 * 16;
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int c = I.col0 + c16 * 16 + jj;
-                        if (c < p.Ncols) p.out[row_off + c * p.os_c] = __uint_as_float(r[jj]);
-                    }
+                    for (int jj = 0; jj < 16; ++jj)
+                        if (c0 + jj < p.Ncols) orow[(c0 + jj) * p.os_c] = __uint_as_float(r[jj]);
                 }
             }
             tc_fence_before();

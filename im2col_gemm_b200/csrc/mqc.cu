@@ -201,11 +201,11 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     const int fixed = 1024 + 64 * 8 + 64;
     int S = std::min(8, (d.max_smem - fixed) / per_stage);
     S = std::min(S, (kTmemCols - kSfTmemBase) / sf_cols);
-    if (S < 2) return fail(MQC_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+    if (S < 4) return fail(MQC_ERR_UNSUPPORTED, "tile does not fit in shared memory");
     P.stages = S;
     P.nacc = (P.BN <= 128) ? 2 : 1;
     P.timeout_ns = kDefaultTimeoutNs;
-    const int smem = fixed + S * per_stage;
+    const int smem = fixed + P.stages * per_stage;
     if (!d.gemm_attr[KIND]) {
         cudaError_t e = cudaFuncSetAttribute(conv_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              d.max_smem);
@@ -313,28 +313,33 @@ mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, 
     p.Ap1 = static_cast<int32_t>(Ap);
     p.Bp1 = static_cast<int32_t>(Bp);
     const bool map_a = mx->order == MQC_ORDER_BA;
+    const bool fp4 = mx->fmt == MQC_E2M1;
     const int64_t r = row_elems(mx->fmt);
     p.I = map_a ? p.A : p.B;
     p.O = map_a ? p.B : p.A;
     p.I1 = static_cast<int32_t>(map_a ? Ap : Bp);
-    p.O1 = p.O;
     p.codes = static_cast<uint8_t *>(codes);
     p.codes_alt = static_cast<uint8_t *>(codes_alt);
     p.O2 = static_cast<int32_t>(round_up(p.O, r));
     p.scales = scales;
-    p.block = mx->block;
     p.fmt = mx->fmt;
     p.emax = emax_elem(mx->fmt);
-    p.nIT = static_cast<int32_t>(ceil_div(p.I1, 32));
-    p.nOT = static_cast<int32_t>(ceil_div(codes_alt ? p.O2 : p.O, 32));
-    const int64_t tiles = ceil_div(p.npix, 32) * p.nOT * p.nIT;
+    // tile: IT = 16 when the innermost axis holds at most 16 FP8 codes, OT = 16
+    // when the other axis (and its padded copy) has at most 16 elements
+    const int it = (!fp4 && p.I1 <= 16) ? 16 : 32;
+    p.OT = (!fp4 && p.O <= 16 && (codes_alt == nullptr || p.O2 <= 16)) ? 16 : 32;
+    const int gsize = p.OT == 16 ? 2 : 1;
+    p.nPT = static_cast<int32_t>(ceil_div(p.npix, 32 * gsize));
+    p.nIT = static_cast<int32_t>(ceil_div(p.I1, it));
+    p.nOT = static_cast<int32_t>(ceil_div(codes_alt ? std::max(p.O, p.O2) : p.O, p.OT));
+    const int64_t tiles = int64_t(p.nPT) * p.nOT * p.nIT;
     if (tiles > (int64_t(1) << 31) - 1) return fail(MQC_ERR_INVALID, "quantize: tensor too large");
+    const bool along_i = (mx->block == MQC_BLOCK_A32) == map_a && mx->block != MQC_BLOCK_SQ32;
+    const int blk = mx->block == MQC_BLOCK_SQ32 ? kSquare : (along_i ? kAlongI : kAlongO);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool fp4 = mx->fmt == MQC_E2M1;
-    if (map_a && !fp4) mx_quantize_kernel<true, false><<<static_cast<unsigned>(tiles), 256, 0, s>>>(p);
-    else if (map_a && fp4) mx_quantize_kernel<true, true><<<static_cast<unsigned>(tiles), 256, 0, s>>>(p);
-    else if (!fp4) mx_quantize_kernel<false, false><<<static_cast<unsigned>(tiles), 256, 0, s>>>(p);
-    else mx_quantize_kernel<false, true><<<static_cast<unsigned>(tiles), 256, 0, s>>>(p);
+    const bool dual = codes_alt != nullptr;
+    if (map_a) launch_quantize_blk<true>(p, blk, dual, it, static_cast<unsigned>(tiles), s);
+    else launch_quantize_blk<false>(p, blk, dual, it, static_cast<unsigned>(tiles), s);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "mx_quantize_kernel launch");
     return MQC_OK;

@@ -53,6 +53,11 @@ def parse_args(argv=None):
                          "dgrad, wgrad) --reps times and exit")
     ap.add_argument("--layer", type=int, default=0)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--workload", default="3",
+                    help="workload of --profile / --sweep: 3 (YOLO training step), 4, or 5:fp8:N / 5:fp4:N")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every call of every layer of --workload (the other configurations: parity-test "
+                         "cases, reported separately from the bench line)")
     return ap.parse_args(argv)
 
 
@@ -306,6 +311,51 @@ def reference_arm(args):
     return 0
 
 
+def workload_by_name(name: str) -> synth.Workload:
+    if ":" in name:
+        cfg, fmt, n = name.split(":")
+        return synth.WORKLOADS[(int(cfg), fmt, int(n))]
+    return synth.WORKLOADS[int(name)]
+
+
+def sweep(mqc, torch, wl, args):
+    """Per-call times of every layer of a workload, with roofline fractions."""
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    out = []
+    for i, L in enumerate(wl.layers):
+        lb = LayerBuffers(mqc, torch, L, wl, i, False)
+        workspace = torch.empty(max(lb.ws_bytes, 16), dtype=torch.uint8, device="cuda")
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        for _ in range(2):
+            run_layer(mqc, lb, workspace, stream)
+        events = []
+        for _ in range(args.reps):
+            run_layer(mqc, lb, workspace, stream, events)
+        torch.cuda.synchronize()
+        mqc.check(mqc.get_device_status())
+        per = {}
+        for name, e0, e1 in events:
+            per.setdefault(name, []).append(e0.elapsed_time(e1))
+        for name, v in per.items():
+            ms = statistics.median(v)
+            if name.startswith("quantize"):
+                byt, fl = lb.quant_bytes(name[-1]), 0
+            else:
+                byt, fl = lb.gemm_bytes(name), lb.gemm_flops()
+            t_roof = max(byt / (pk["hbm_gbs"] * 1e9), fl / (fp8_peak * 1e12))
+            out.append({"workload": wl.name, "layer": i, "call": name, "ms": round(ms, 5),
+                        "tflops": round(fl / (ms * 1e-3) / 1e12, 1) if fl else None,
+                        "gbs": round(byt / (ms * 1e-3) / 1e9, 1),
+                        "frac_of_roofline": round(1e3 * t_roof / ms, 4),
+                        "frac_of_mxfp8_peak": round(fl / (ms * 1e-3) / 1e12 / fp8_peak, 4) if fl else None})
+        del lb, workspace
+        torch.cuda.empty_cache()
+    for o in out:
+        print(json.dumps(o), flush=True)
+    return 0
+
+
 # --------------------------------------------------------------------------- profiling driver
 def profile_call(mqc, torch, wl, args):
     """Runs one layer's calls once (so every operand exists), then the chosen
@@ -336,7 +386,10 @@ def main(argv=None):
     import im2col_gemm_b200 as mqc
 
     wl = synth.WORKLOADS[WORKLOAD_CFG]
-    if args.profile:
+    if args.profile or args.sweep:
+        wl = workload_by_name(args.workload)
+        if args.sweep:
+            return sweep(mqc, torch, wl, args)
         return profile_call(mqc, torch, wl, args)
     pk = peaks()
     want_host = not args.skip_e2e

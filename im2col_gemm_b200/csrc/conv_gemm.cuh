@@ -35,7 +35,15 @@
 namespace mqc {
 
 constexpr int kMaxTaps = 64;
-constexpr int kGemmThreads = 320;
+constexpr int kGemmThreads = 384;
+// Warp roles (a warp's SM sub-partition is its index modulo 4):
+//   0 TMA producer, 1 MMA issuer (alone on its sub-partition apart from one
+//   epilogue warp), 4-7 epilogue (one per TMEM lane quadrant), and the
+//   scale-factor gather warps below; warp 9 only joins the final barrier.
+constexpr int kNumSfWarps = 5;
+__device__ __forceinline__ int sf_warp_index(int warp) {
+    return warp == 2 ? 0 : warp == 3 ? 1 : warp == 8 ? 2 : warp == 10 ? 3 : warp == 11 ? 4 : -1;
+}
 constexpr int kTmemCols = 512;
 constexpr int kSfTmemBase = 256;
 
@@ -174,9 +182,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     uint8_t *sB = sA + S * a_stage;
     uint8_t *sSFA = sB + S * b_stage;
     uint8_t *sSFB = sSFA + S * 512;
-    uint64_t *full_tma = reinterpret_cast<uint64_t *>(sSFB + S * sfb_stage);
-    uint64_t *full_sf = full_tma + S;
-    uint64_t *empty = full_sf + S;
+    // full[s]: completes when the TMA bytes of stage s have landed AND the
+    // scale-gather warp of stage s has arrived (count 2)
+    uint64_t *full = reinterpret_cast<uint64_t *>(sSFB + S * sfb_stage);
+    uint64_t *empty = full + S;
     uint64_t *acc_full = empty + S;
     uint64_t *acc_empty = acc_full + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
@@ -187,8 +196,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full_tma[s], 1);
-            mbar_init(&full_sf[s], 1);
+            mbar_init(&full[s], 2);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -241,26 +249,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     if (KIND == kConv) {
                         const int nkb = min(4, p.total_kb - 4 * ki);
                         const int nbox = nkb >> lg_wkb;
-                        mbar_arrive_expect_tx(&full_tma[s],
+                        mbar_arrive_expect_tx(&full[s],
                                               static_cast<uint32_t>(nbox * (p.a_box_bytes + p.b_box_bytes)));
                         for (int j = 0; j < nbox; ++j) {
                             const ConvTap T = p.taps[kw.tap];
                             const int cx = kw.cb * 32;
                             if (p.rows_nfirst)
-                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full_tma[s], cx, I.n0,
+                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx, I.n0,
                                             I.q0 + T.dw, I.p0 + T.dh);
                             else
-                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full_tma[s], cx,
+                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx,
                                             I.q0 + T.dw, I.p0 + T.dh, I.n0);
-                            tma_load_3d(b_dst + j * p.BN * row_bytes, &p.bmap[0], &full_tma[s], cx, I.col0, T.btap);
+                            tma_load_3d(b_dst + j * p.BN * row_bytes, &p.bmap[0], &full[s], cx, I.col0, T.btap);
                             kw.advance(p.wkb, p.CB);
                         }
                     } else {
                         const ConvTap T = p.taps[I.tap];
-                        mbar_arrive_expect_tx(&full_tma[s], static_cast<uint32_t>(p.a_box_bytes + p.b_box_bytes));
+                        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.a_box_bytes + p.b_box_bytes));
                         const int nx = nc * row_bytes;
-                        tma_load_4d(a_dst, &p.amap[0], &full_tma[s], nx, I.m0, qg * p.bqk, pp);
-                        tma_load_4d(b_dst, &p.bmap[T.map], &full_tma[s], nx, I.col0, qg * p.bqk + T.dw, pp + T.dh);
+                        tma_load_4d(a_dst, &p.amap[0], &full[s], nx, I.m0, qg * p.bqk, pp);
+                        tma_load_4d(b_dst, &p.bmap[T.map], &full[s], nx, I.col0, qg * p.bqk + T.dw, pp + T.dh);
                         if (++nc == p.NC) {
                             nc = 0;
                             if (++qg == p.QG) {
@@ -272,10 +280,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 }
             }
             if (!ok) {
-                // let the copies already in flight land before the CTA exits
+                // let the copies already in flight land before the CTA exits (a
+                // stage whose scale warp gave up never completes; its copy is
+                // long done when the short bounded wait below runs out)
                 const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0u;
                 for (uint32_t c = first; c < it; ++c)
-                    mbar_wait(&full_tma[c % S], (c / S) & 1u, 100000000ull, nullptr);
+                    mbar_wait(&full[c % S], (c / S) & 1u, 20000000ull, nullptr);
             }
         }
     } else if (warp == 1) {
@@ -301,11 +311,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + acc * p.BN;
                 for (int ki = 0; ki < I.nk; ++ki, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
-                    if (!mbar_wait(&full_tma[s], ph, lim, abort_flag) || !mbar_wait(&full_sf[s], ph, lim, abort_flag)) {
+                    if (!mbar_wait(&full[s], ph, lim, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
                     const uint32_t sfa_t = tmem + kSfTmemBase + s * sf_cols;
                     const uint32_t sfb_t = sfa_t + 4;
                     tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + static_cast<uint64_t>((s * 512) >> 4));
@@ -331,10 +340,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 ++tcount;
             }
         }
-    } else if (warp < 6) {
+    } else if (sf_warp_index(warp) >= 0) {
         // ------------------------------------------------------------ scale-factor gather
-        // warp 2+w handles the stages whose global index is w modulo 4
-        const int sfw = warp - 2;
+        // scale warp w handles the stages whose global index is w modulo kNumSfWarps
+        const int sfw = sf_warp_index(warp);
         uint32_t it = 0;             // global index of the first stage of the unit
         uint32_t g = static_cast<uint32_t>(sfw);   // global index of this warp's next stage
         int s = sfw % S;
@@ -389,7 +398,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 qg = (kg / p.NC) % p.QG;
                 pp = kg / (p.NC * p.QG);
             }
-            for (int ki = first; ki < I.nk; ki += 4) {
+            for (int ki = first; ki < I.nk; ki += kNumSfWarps) {
                 uint32_t wa[4] = {0u, 0u, 0u, 0u};      // A atom bytes: row lane+32j, byte kb
                 uint32_t wb[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
                 if (KIND == kConv) {
@@ -417,7 +426,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                                 if (rb_ok[at][j]) wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
                         k2.advance(1, p.CB);
                     }
-                    kw.advance(16, p.CB);
+                    kw.advance(4 * kNumSfWarps, p.CB);
                 } else {
                     const ConvTap T = p.taps[I.tap];
                     for (int kb = 0; kb < 4; ++kb) {
@@ -439,8 +448,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                             for (int j = 0; j < 4; ++j)
                                 if (rb_ok[at][j]) wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
                     }
-                    // advance the (pixel row, q-group, n-chunk) walker by 4 K iterations
-                    for (int step = 0; step < 4; ++step)
+                    // advance the (pixel row, q-group, n-chunk) walker by kNumSfWarps K iterations
+                    for (int step = 0; step < kNumSfWarps; ++step)
                         if (++nc == p.NC) {
                             nc = 0;
                             if (++qg == p.QG) {
@@ -460,16 +469,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         make_uint4(wb[1][0], wb[1][1], wb[1][2], wb[1][3]);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&full_sf[s]);
-                g += 4;
-                s += 4;
+                if (lane == 0) mbar_arrive(&full[s]);
+                g += kNumSfWarps;
+                s += kNumSfWarps;
                 while (s >= S) {
                     s -= S;
                     ph ^= 1u;
                 }
             }
         }
-    } else {
+    } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ epilogue
         const int qd = warp & 3;               // TMEM lane quadrant of this warp
         const int m = qd * 32 + lane;

@@ -83,6 +83,7 @@ struct alignas(64) GemmParams {
     int32_t a_box_bytes, b_box_bytes;
     // CONV kind
     int32_t rows_nfirst;         // A map dims (C, N, W, H) instead of (C, W, H, N)
+    int32_t sf_vec4;             // a stage's 4 K-blocks are 4 aligned consecutive scale bytes (one tap)
     int32_t bq, bp, bn;          // A box extents along q, p, n
     int32_t TQ, TP, TN, NT;      // tile counts
     int32_t Qe, Pe, Ne;          // output extents (row masks)
@@ -225,120 +226,128 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            uint32_t it = 0;
-            int s = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-                const UnitInfo I = decode_unit<KIND>(p, u);
-                KbWalker kw{0, 0};
-                int kg = I.kbase, nc = 0, qg = 0, pp = 0;
-                if (KIND == kWgrad) {
-                    nc = kg % p.NC;
-                    qg = (kg / p.NC) % p.QG;
-                    pp = kg / (p.NC * p.QG);
+        // the whole warp walks the stages; one elected lane issues the copies
+        const bool leader = elect_one();
+        uint32_t it = 0;
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const UnitInfo I = decode_unit<KIND>(p, u);
+            KbWalker kw{0, 0};
+            int kg = I.kbase, nc = 0, qg = 0, pp = 0;
+            if (KIND == kWgrad) {
+                nc = kg % p.NC;
+                qg = (kg / p.NC) % p.QG;
+                pp = kg / (p.NC * p.QG);
+            }
+            for (int ki = 0; ki < I.nk; ++ki, ++it, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag))) {
+                    ok = false;
+                    break;
                 }
-                for (int ki = 0; ki < I.nk; ++ki, ++it, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
-                    if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *a_dst = sA + s * a_stage;
-                    uint8_t *b_dst = sB + s * b_stage;
-                    if (KIND == kConv) {
-                        const int nkb = min(4, p.total_kb - 4 * ki);
-                        const int nbox = nkb >> lg_wkb;
-                        mbar_arrive_expect_tx(&full[s],
-                                              static_cast<uint32_t>(nbox * (p.a_box_bytes + p.b_box_bytes)));
-                        for (int j = 0; j < nbox; ++j) {
-                            const ConvTap T = p.taps[kw.tap];
-                            const int cx = kw.cb * 32;
+                uint8_t *a_dst = sA + s * a_stage;
+                uint8_t *b_dst = sB + s * b_stage;
+                if (KIND == kConv) {
+                    const int nkb = min(4, p.total_kb - 4 * ki);
+                    const int nbox = nkb >> lg_wkb;
+                    if (leader)
+                        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * (p.a_box_bytes + p.b_box_bytes)));
+                    for (int j = 0; j < nbox; ++j) {
+                        const ConvTap T = p.taps[kw.tap];
+                        const int cx = kw.cb * 32;
+                        if (leader) {
                             if (p.rows_nfirst)
                                 tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx, I.n0,
                                             I.q0 + T.dw, I.p0 + T.dh);
                             else
-                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx,
-                                            I.q0 + T.dw, I.p0 + T.dh, I.n0);
+                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx, I.q0 + T.dw,
+                                            I.p0 + T.dh, I.n0);
                             tma_load_3d(b_dst + j * p.BN * row_bytes, &p.bmap[0], &full[s], cx, I.col0, T.btap);
-                            kw.advance(p.wkb, p.CB);
                         }
-                    } else {
-                        const ConvTap T = p.taps[I.tap];
+                        kw.advance(p.wkb, p.CB);
+                    }
+                } else {
+                    const ConvTap T = p.taps[I.tap];
+                    const int nx = nc * row_bytes;
+                    if (leader) {
                         mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.a_box_bytes + p.b_box_bytes));
-                        const int nx = nc * row_bytes;
                         tma_load_4d(a_dst, &p.amap[0], &full[s], nx, I.m0, qg * p.bqk, pp);
                         tma_load_4d(b_dst, &p.bmap[T.map], &full[s], nx, I.col0, qg * p.bqk + T.dw, pp + T.dh);
-                        if (++nc == p.NC) {
-                            nc = 0;
-                            if (++qg == p.QG) {
-                                qg = 0;
-                                ++pp;
-                            }
+                    }
+                    if (++nc == p.NC) {
+                        nc = 0;
+                        if (++qg == p.QG) {
+                            qg = 0;
+                            ++pp;
                         }
                     }
                 }
+                __syncwarp();
             }
-            if (!ok) {
-                // let the copies already in flight land before the CTA exits (a
-                // stage whose scale warp gave up never completes; its copy is
-                // long done when the short bounded wait below runs out)
-                const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0u;
-                for (uint32_t c = first; c < it; ++c)
-                    mbar_wait(&full[c % S], (c / S) & 1u, 20000000ull, nullptr);
-            }
+        }
+        if (!ok && leader) {
+            // let the copies already in flight land before the CTA exits (a
+            // stage whose scale warp gave up never completes; its copy is
+            // long done when the short bounded wait below runs out)
+            const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0u;
+            for (uint32_t c = first; c < it; ++c) mbar_wait(&full[c % S], (c / S) & 1u, 20000000ull, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            uint32_t tcount = 0;
-            int s = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            const uint32_t swz = swizzle_of(p.wkb);
-            // descriptors of stage 0, sub-tile 0; other positions add (byte offset >> 4)
-            const uint64_t adesc0 = make_smem_desc(smem_u32(sA), 16, 8 * row_bytes, swz);
-            const uint64_t bdesc0 = make_smem_desc(smem_u32(sB), 16, 8 * row_bytes, swz);
-            const uint64_t sfa_desc0 = make_smem_desc(smem_u32(sSFA), 0, 128, kSwizzleNone);
-            const uint64_t sfb_desc0 = make_smem_desc(smem_u32(sSFB), 0, 128, kSwizzleNone);
-            const uint32_t a_sub = (128 * row_bytes) >> 4, b_sub = (p.BN * row_bytes) >> 4;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-                const UnitInfo I = decode_unit<KIND>(p, u);
-                if (I.nk == 0) continue;
-                const uint32_t acc = tcount & 1u & static_cast<uint32_t>(p.nacc - 1);
-                const uint32_t aph = (p.nacc == 2 ? (tcount >> 1) : tcount) & 1u;
-                if (!mbar_wait(&acc_empty[acc], aph ^ 1u, lim, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + acc * p.BN;
-                for (int ki = 0; ki < I.nk; ++ki, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
-                    if (!mbar_wait(&full[s], ph, lim, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t sfa_t = tmem + kSfTmemBase + s * sf_cols;
-                    const uint32_t sfb_t = sfa_t + 4;
+        // the whole warp walks the stages (so descriptors and TMEM addresses are
+        // warp-uniform); one elected lane issues tcgen05.cp / mma / commit
+        const bool leader = elect_one();
+        uint32_t tcount = 0;
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        const uint32_t swz = swizzle_of(p.wkb);
+        // descriptors of stage 0, sub-tile 0; other positions add (byte offset >> 4)
+        const uint64_t adesc0 = make_smem_desc(smem_u32(sA), 16, 8 * row_bytes, swz);
+        const uint64_t bdesc0 = make_smem_desc(smem_u32(sB), 16, 8 * row_bytes, swz);
+        const uint64_t sfa_desc0 = make_smem_desc(smem_u32(sSFA), 0, 128, kSwizzleNone);
+        const uint64_t sfb_desc0 = make_smem_desc(smem_u32(sSFB), 0, 128, kSwizzleNone);
+        const uint32_t a_sub = (128 * row_bytes) >> 4, b_sub = (p.BN * row_bytes) >> 4;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const UnitInfo I = decode_unit<KIND>(p, u);
+            if (I.nk == 0) continue;
+            const uint32_t acc = tcount & 1u & static_cast<uint32_t>(p.nacc - 1);
+            const uint32_t aph = (p.nacc == 2 ? (tcount >> 1) : tcount) & 1u;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_empty[acc], aph ^ 1u, lim, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + acc * p.BN;
+            for (int ki = 0; ki < I.nk; ++ki, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], ph, lim, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sfa_t = tmem + kSfTmemBase + s * sf_cols;
+                const uint32_t sfb_t = sfa_t + 4;
+                const int nkb = KIND == kConv ? min(4, p.total_kb - 4 * ki) : 4;
+                const uint64_t a_s = adesc0 + static_cast<uint64_t>((s * a_stage) >> 4);
+                const uint64_t b_s = bdesc0 + static_cast<uint64_t>((s * b_stage) >> 4);
+                if (leader) {
                     tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + static_cast<uint64_t>((s * 512) >> 4));
                     for (int a = 0; a < p.nb_atoms; ++a)
                         tc_cp_32x128b_warpx4(sfb_t + 4 * a,
                                              sfb_desc0 + static_cast<uint64_t>((s * sfb_stage + a * 512) >> 4));
-                    const int nkb = KIND == kConv ? min(4, p.total_kb - 4 * ki) : 4;
-                    const uint64_t a_s = adesc0 + static_cast<uint64_t>((s * a_stage) >> 4);
-                    const uint64_t b_s = bdesc0 + static_cast<uint64_t>((s * b_stage) >> 4);
                     for (int kb = 0; kb < nkb; ++kb) {
                         const uint32_t j = static_cast<uint32_t>(kb >> lg_wkb);
                         const uint32_t within = static_cast<uint32_t>(kb & (p.wkb - 1));
-                        const uint64_t adesc = a_s + j * a_sub + within * 2;
-                        const uint64_t bdesc = b_s + j * b_sub + within * 2;
                         const uint32_t kbu = static_cast<uint32_t>(kb);
-                        tc_mma_mxf8f6f4(d_tmem, adesc, bdesc, p.idesc | (kbu << 29) | (kbu << 4), sfa_t | (kbu << 30),
-                                        sfb_t | (kbu << 30), (ki > 0 || kb > 0) ? 1u : 0u);
+                        tc_mma_mxf8f6f4(d_tmem, a_s + j * a_sub + within * 2, b_s + j * b_sub + within * 2,
+                                        p.idesc | (kbu << 29) | (kbu << 4), sfa_t | (kbu << 30), sfb_t | (kbu << 30),
+                                        (ki > 0 || kb > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                 }
-                if (!ok) break;
-                tc_commit(&acc_full[acc]);
-                ++tcount;
+                __syncwarp();
             }
+            if (!ok) break;
+            if (leader) tc_commit(&acc_full[acc]);
+            __syncwarp();
+            ++tcount;
         }
     } else if (sf_warp_index(warp) >= 0) {
         // ------------------------------------------------------------ scale-factor gather
@@ -401,7 +410,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             for (int ki = first; ki < I.nk; ki += kNumSfWarps) {
                 uint32_t wa[4] = {0u, 0u, 0u, 0u};      // A atom bytes: row lane+32j, byte kb
                 uint32_t wb[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-                if (KIND == kConv) {
+                if (KIND == kConv && p.sf_vec4) {
+                    // one tap, channel blocks cb..cb+3: one 32-bit load per row
+                    const ConvTap T = p.taps[kw.tap];
+                    const int cb = kw.cb;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
+                        if (ra_ok[j] && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W)
+                            wa[j] = __ldg(reinterpret_cast<const uint32_t *>(
+                                p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch + ra_off[j] + cb));
+                    }
+                    const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb;
+#pragma unroll
+                    for (int at = 0; at < 2; ++at)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (rb_ok[at][j]) wb[at][j] = __ldg(reinterpret_cast<const uint32_t *>(bsrc + rb_off[at][j]));
+                    kw.advance(4 * kNumSfWarps, p.CB);
+                } else if (KIND == kConv) {
                     const int nkb = min(4, p.total_kb - 4 * ki);
                     KbWalker k2 = kw;
                     for (int kb = 0; kb < nkb; ++kb) {
@@ -509,20 +536,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             tc_fence_after();
             const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16) + acc * p.BN;
             float *orow = p.out + row_off;
-            for (int c16 = 0; c16 < p.BN / 16; ++c16) {
-                uint32_t r[16];
-                tc_ld_32x32b_x16(t_row + c16 * 16, r);
-                tc_wait_ld();
-                if (row_ok) {
-                    const int c0 = I.col0 + c16 * 16;
+            // up to 128 columns at a time: all their TMEM loads, one wait; the
+            // accumulator is released before the (slow) global stores of the
+            // last part so the MMA issuer can start the next tile on it
+            for (int c0 = 0; c0 < p.BN; c0 += 128) {
+                const int ncol = min(128, p.BN - c0);
+                uint32_t r[128];
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        if (c0 + jj < p.Ncols) orow[(c0 + jj) * p.os_c] = __uint_as_float(r[jj]);
+                for (int q = 0; q < 4; ++q)
+                    if (32 * q < ncol) tc_ld_32x32b_x32(t_row + c0 + 32 * q, r + 32 * q);
+                tc_wait_ld();
+                if (c0 + 128 >= p.BN) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                }
+                if (row_ok) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (32 * q < ncol) {
+                            const int cb = I.col0 + c0 + 32 * q;
+                            float *op = orow + static_cast<int64_t>(cb) * p.os_c;
+                            if (cb + 32 <= p.Ncols) {
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj) op[jj * p.os_c] = __uint_as_float(r[32 * q + jj]);
+                            } else {
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj)
+                                    if (cb + jj < p.Ncols) op[jj * p.os_c] = __uint_as_float(r[32 * q + jj]);
+                            }
+                        }
+                    }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
             ++tcount;
         }
     }

@@ -532,6 +532,9 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     G.sfb.row_pitch = static_cast<int32_t>(nb32(Cp));
     G.sfb.kb_pitch = 1;
     G.sfb.rows = K;
+    G.sf_vec4 = G.CB % 4 == 0 && G.sfa.pix_pitch % 4 == 0 && G.sfa.row_pitch % 4 == 0 &&
+                G.sfb.tap_pitch % 4 == 0 && G.sfb.row_pitch % 4 == 0 &&
+                (reinterpret_cast<uintptr_t>(xs) & 3u) == 0 && (reinterpret_cast<uintptr_t>(ws) & 3u) == 0;
     G.out = y;
     G.out_base = 0;
     G.os_q = 1;
@@ -635,6 +638,7 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
             G.sfb.row_pitch = 1;
             G.sfb.kb_pitch = static_cast<int32_t>(sqw ? nb32(C) : C);
             G.sfb.rows = C;
+            G.sf_vec4 = false;   // the weights' scales run along K with a stride of C per block
             G.out = gx;
             G.out_base = int64_t(ah) * W + aw;
             G.os_q = sw;

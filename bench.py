@@ -43,8 +43,8 @@ METRIC = "MX conv fwd+bwd TFLOPS (quantizer GB/s and % of roofline alongside) at
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="mqc", choices=["mqc", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
@@ -110,7 +110,7 @@ class ClockSampler:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
@@ -412,6 +412,11 @@ def main(argv=None):
             run_layer(mqc, lb, workspace, stream, events)
         allreduce_gw()
 
+    # clocks are sampled from the start of the warm-up to the end of the timed
+    # region (nvidia-smi needs a few hundred ms to produce its first sample)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.5)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -419,8 +424,6 @@ def main(argv=None):
 
     # ---- timed region: inputs resident in HBM
     events = []
-    clocks = ClockSampler(local)
-    clocks.start()
     barrier()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -83,7 +83,10 @@ struct alignas(64) GemmParams {
     int32_t a_box_bytes, b_box_bytes;
     // CONV kind
     int32_t rows_nfirst;         // A map dims (C, N, W, H) instead of (C, W, H, N)
-    int32_t sf_vec4;             // a stage's 4 K-blocks are 4 aligned consecutive scale bytes (one tap)
+    int32_t sf_vec4;             // A: a stage's 4 K-blocks are 4 aligned consecutive scale bytes (one tap)
+    int32_t sfb_vec4;            // B: likewise (the weights' scales along C)
+    int32_t sfb_cached;          // CONV: B scale atoms of every (column tile, stage) built once per CTA
+    int32_t ktiles;              // CONV: stages per tile
     int32_t bq, bp, bn;          // A box extents along q, p, n
     int32_t TQ, TP, TN, NT;      // tile counts
     int32_t Qe, Pe, Ne;          // output extents (row masks)
@@ -183,9 +186,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     uint8_t *sB = sA + S * a_stage;
     uint8_t *sSFA = sB + S * b_stage;
     uint8_t *sSFB = sSFA + S * 512;
+    uint8_t *sSFBc = sSFB + S * sfb_stage;    // cached B atoms: [column tile][stage][atom] x 512 B
+    const int sfbc_bytes = p.sfb_cached ? p.NT * p.ktiles * p.nb_atoms * 512 : 0;
     // full[s]: completes when the TMA bytes of stage s have landed AND the
     // scale-gather warp of stage s has arrived (count 2)
-    uint64_t *full = reinterpret_cast<uint64_t *>(sSFB + S * sfb_stage);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sSFBc + sfbc_bytes);
     uint64_t *empty = full + S;
     uint64_t *acc_full = empty + S;
     uint64_t *acc_empty = acc_full + 2;
@@ -214,6 +219,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     if (warp == 1) {
         tmem_alloc(tmem_holder, kTmemCols);
         tmem_relinquish();
+    }
+    if (KIND == kConv && p.sfb_cached) {
+        // every thread helps build the B scale atoms once: item = (column tile,
+        // stage of the tile, atom); lane l writes rows l, l+32, l+64, l+96
+        const int items = p.NT * p.ktiles * p.nb_atoms;
+        for (int item = warp; item < items; item += kGemmThreads / 32) {
+            const int at = item % p.nb_atoms;
+            const int ks = (item / p.nb_atoms) % p.ktiles;
+            const int nt = item / (p.nb_atoms * p.ktiles);
+            uint32_t wv[4] = {0u, 0u, 0u, 0u};
+            for (int kb = 0; kb < 4; ++kb) {
+                const int g = 4 * ks + kb;
+                if (g >= p.total_kb) break;
+                const ConvTap T = p.taps[g / p.CB];
+                const uint8_t *bsrc =
+                    p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + (g % p.CB) * p.sfb.kb_pitch;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int rl = 128 * at + 32 * j + lane;
+                    const int r = nt * p.BN + rl;
+                    if (rl < p.BN && r < p.sfb.rows)
+                        wv[j] |= static_cast<uint32_t>(__ldg(bsrc + (r / p.sfb.row_div) * p.sfb.row_pitch)) << (8 * kb);
+                }
+            }
+            *reinterpret_cast<uint4 *>(sSFBc + item * 512 + lane * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -308,6 +340,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         const uint64_t bdesc0 = make_smem_desc(smem_u32(sB), 16, 8 * row_bytes, swz);
         const uint64_t sfa_desc0 = make_smem_desc(smem_u32(sSFA), 0, 128, kSwizzleNone);
         const uint64_t sfb_desc0 = make_smem_desc(smem_u32(sSFB), 0, 128, kSwizzleNone);
+        const uint64_t sfbc_desc0 = make_smem_desc(smem_u32(sSFBc), 0, 128, kSwizzleNone);
         const uint32_t a_sub = (128 * row_bytes) >> 4, b_sub = (p.BN * row_bytes) >> 4;
         for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
@@ -317,6 +350,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_empty[acc], aph ^ 1u, lim, abort_flag))) break;
             tc_fence_after();
             const uint32_t d_tmem = tmem + acc * p.BN;
+            const int item_base = (I.col0 / p.BN) * p.ktiles * p.nb_atoms;   // cached B atoms of this column tile
             for (int ki = 0; ki < I.nk; ++ki, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], ph, lim, abort_flag))) {
                     ok = false;
@@ -329,9 +363,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 const uint64_t b_s = bdesc0 + static_cast<uint64_t>((s * b_stage) >> 4);
                 if (leader) {
                     tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + static_cast<uint64_t>((s * 512) >> 4));
-                    for (int a = 0; a < p.nb_atoms; ++a)
-                        tc_cp_32x128b_warpx4(sfb_t + 4 * a,
-                                             sfb_desc0 + static_cast<uint64_t>((s * sfb_stage + a * 512) >> 4));
+                    if (KIND == kConv && p.sfb_cached) {
+                        const int item0 = item_base + ki * p.nb_atoms;
+                        for (int a = 0; a < p.nb_atoms; ++a)
+                            tc_cp_32x128b_warpx4(sfb_t + 4 * a,
+                                                 sfbc_desc0 + static_cast<uint64_t>(((item0 + a) * 512) >> 4));
+                    } else {
+                        for (int a = 0; a < p.nb_atoms; ++a)
+                            tc_cp_32x128b_warpx4(sfb_t + 4 * a,
+                                                 sfb_desc0 + static_cast<uint64_t>((s * sfb_stage + a * 512) >> 4));
+                    }
                     for (int kb = 0; kb < nkb; ++kb) {
                         const uint32_t j = static_cast<uint32_t>(kb >> lg_wkb);
                         const uint32_t within = static_cast<uint32_t>(kb & (p.wkb - 1));
@@ -421,12 +462,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                             wa[j] = __ldg(reinterpret_cast<const uint32_t *>(
                                 p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch + ra_off[j] + cb));
                     }
-                    const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb;
+                    if (!p.sfb_cached) {
+                        const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb;
 #pragma unroll
-                    for (int at = 0; at < 2; ++at)
+                        for (int at = 0; at < 2; ++at)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            if (rb_ok[at][j]) wb[at][j] = __ldg(reinterpret_cast<const uint32_t *>(bsrc + rb_off[at][j]));
+                            for (int j = 0; j < 4; ++j)
+                                if (rb_ok[at][j])
+                                    wb[at][j] = __ldg(reinterpret_cast<const uint32_t *>(bsrc + rb_off[at][j]));
+                    }
                     kw.advance(4 * kNumSfWarps, p.CB);
                 } else if (KIND == kConv) {
                     const int nkb = min(4, p.total_kb - 4 * ki);
@@ -444,13 +488,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                                 wa[j] |= static_cast<uint32_t>(__ldg(src)) << (8 * kb);
                             }
                         }
-                        const uint8_t *bsrc =
-                            p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
+                        if (!p.sfb_cached) {
+                            const uint8_t *bsrc =
+                                p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
 #pragma unroll
-                        for (int at = 0; at < 2; ++at)
+                            for (int at = 0; at < 2; ++at)
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                if (rb_ok[at][j]) wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                                for (int j = 0; j < 4; ++j)
+                                    if (rb_ok[at][j])
+                                        wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                        }
                         k2.advance(1, p.CB);
                     }
                     kw.advance(4 * kNumSfWarps, p.CB);
@@ -490,8 +537,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     break;
                 }
                 *reinterpret_cast<uint4 *>(sSFA + s * 512 + lane * 16) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-                *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + lane * 16) = make_uint4(wb[0][0], wb[0][1], wb[0][2], wb[0][3]);
-                if (p.nb_atoms > 1)
+                if (!(KIND == kConv && p.sfb_cached))
+                    *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + lane * 16) =
+                        make_uint4(wb[0][0], wb[0][1], wb[0][2], wb[0][3]);
+                if (!(KIND == kConv && p.sfb_cached) && p.nb_atoms > 1)
                     *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + 512 + lane * 16) =
                         make_uint4(wb[1][0], wb[1][1], wb[1][2], wb[1][3]);
                 fence_proxy_async_smem();

@@ -198,7 +198,14 @@ template <int KIND>
 mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     const int per_stage = 128 * 128 + P.BN * 128 + 512 + 512 * P.nb_atoms;
     const int sf_cols = 4 + 4 * P.nb_atoms;
-    const int fixed = 1024 + 64 * 8 + 64;
+    // CONV: the weights' scale atoms are the same for every output tile of a
+    // column tile; build them once per CTA when they fit in 16 KB
+    P.ktiles = (P.total_kb + 3) / 4;
+    const int cache = KIND == kConv ? P.NT * P.ktiles * P.nb_atoms * 512 : 0;
+    P.sfb_cached = KIND == kConv && cache <= 16384 && !P.sfb_vec4;
+    // the 32-bit scale path reads B four bytes at a time unless B is cached
+    if (!P.sfb_cached && !P.sfb_vec4) P.sf_vec4 = 0;
+    const int fixed = 1024 + 64 * 8 + 64 + (P.sfb_cached ? cache : 0);
     int S = std::min(8, (d.max_smem - fixed) / per_stage);
     S = std::min(S, (kTmemCols - kSfTmemBase) / sf_cols);
     if (S < 4) return fail(MQC_ERR_UNSUPPORTED, "tile does not fit in shared memory");
@@ -533,8 +540,9 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     G.sfb.kb_pitch = 1;
     G.sfb.rows = K;
     G.sf_vec4 = G.CB % 4 == 0 && G.sfa.pix_pitch % 4 == 0 && G.sfa.row_pitch % 4 == 0 &&
-                G.sfb.tap_pitch % 4 == 0 && G.sfb.row_pitch % 4 == 0 &&
-                (reinterpret_cast<uintptr_t>(xs) & 3u) == 0 && (reinterpret_cast<uintptr_t>(ws) & 3u) == 0;
+                (reinterpret_cast<uintptr_t>(xs) & 3u) == 0;
+    G.sfb_vec4 = G.CB % 4 == 0 && G.sfb.tap_pitch % 4 == 0 && G.sfb.row_pitch % 4 == 0 &&
+                 (reinterpret_cast<uintptr_t>(ws) & 3u) == 0;
     G.out = y;
     G.out_base = 0;
     G.os_q = 1;
@@ -638,7 +646,9 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
             G.sfb.row_pitch = 1;
             G.sfb.kb_pitch = static_cast<int32_t>(sqw ? nb32(C) : C);
             G.sfb.rows = C;
-            G.sf_vec4 = false;   // the weights' scales run along K with a stride of C per block
+            G.sf_vec4 = G.CB % 4 == 0 && G.sfa.pix_pitch % 4 == 0 && G.sfa.row_pitch % 4 == 0 &&
+                        (reinterpret_cast<uintptr_t>(gs) & 3u) == 0;
+            G.sfb_vec4 = false;   // the weights' scales run along K with a stride of C per block
             G.out = gx;
             G.out_base = int64_t(ah) * W + aw;
             G.os_q = sw;

@@ -48,8 +48,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="mqc", choices=["mqc", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
-    ap.add_argument("--profile", default=None, metavar="CALL",
-                    help="profiling mode: build one layer, then run CALL (quantize_x, quantize_w, quantize_g, fwd, "
+    ap.add_argument("--profile", default=None, metavar="CALL[,CALL...]",
+                    help="profiling mode: build one layer, then run the listed calls (quantize_x, quantize_w, quantize_g, fwd, "
                          "dgrad, wgrad) --reps times and exit")
     ap.add_argument("--layer", type=int, default=0)
     ap.add_argument("--reps", type=int, default=3)
@@ -220,12 +220,12 @@ class LayerBuffers:
 def run_layer(mqc, lb: LayerBuffers, workspace, stream, events=None, only=None):
     """All calls of one layer through the C ABI; `events` (optional) collects
     (name, start, end) CUDA events around every call on `stream`; `only`
-    restricts the run to one named call (profiling)."""
+    (a tuple of call names) restricts the run to those calls (profiling)."""
     c_void = ctypes.c_void_p
     P = lambda t: c_void(t.data_ptr())
 
     def timed(name, fn):
-        if only is not None and name != only:
+        if only is not None and name not in only:
             return
         if events is not None:
             import torch
@@ -366,7 +366,7 @@ def profile_call(mqc, torch, wl, args):
     run_layer(mqc, lb, workspace, stream)
     events = []
     for _ in range(args.reps):
-        run_layer(mqc, lb, workspace, stream, events, only=args.profile)
+        run_layer(mqc, lb, workspace, stream, events, only=tuple(args.profile.split(",")))
     torch.cuda.synchronize()
     mqc.check(mqc.get_device_status())
     ms = [e0.elapsed_time(e1) for _, e0, e1 in events]

@@ -19,13 +19,15 @@
 //   WGRAD (weight gradient): rows = C_out, columns = C_in of one tap,
 //         reduction = (output pixel, batch) with N contiguous; split over K.
 //
-// CTA layout (persistent, one CTA per SM, 10 warps):
+// CTA layout (persistent, one CTA per SM, 12 warps):
 //   warp 0      TMA producer (codes of A and B, one elected thread)
-//   warp 1      TMEM allocator + MMA issuer (one thread): scale factors
-//               smem -> TMEM with tcgen05.cp, then tcgen05.mma block_scale
-//   warps 2-5   scale-factor gather: E8M0 bytes of every operand row and
-//               K-block into the 128x4 shared-memory atom the MMA expects
-//   warps 6-9   epilogue: TMEM -> registers -> fp32 global stores
+//   warp 1      TMEM allocator + MMA issuer (one elected thread): scale
+//               factors smem -> TMEM with tcgen05.cp, then tcgen05.mma
+//               block_scale, 4 or 8 K-blocks (of 32) per pipeline stage
+//   warps 2, 3, 8, 10, 11   scale-factor gather: E8M0 bytes of every operand
+//               row and K-block into the 128x4 shared-memory atoms the MMA
+//               expects (one stage per warp in turn)
+//   warps 4-7   epilogue: TMEM -> registers -> fp32 global stores
 // Every wait is bounded in time; a wait that runs out records a device error
 // and the CTA winds down without hanging.
 #pragma once
@@ -35,6 +37,7 @@
 namespace mqc {
 
 constexpr int kMaxTaps = 64;
+constexpr int kMaxPhases = 4;   // CONV: output stride phases sharing one launch
 constexpr int kGemmThreads = 384;
 // Warp roles (a warp's SM sub-partition is its index modulo 4):
 //   0 TMA producer, 1 MMA issuer (alone on its sub-partition apart from one
@@ -77,23 +80,34 @@ struct alignas(64) GemmParams {
     int32_t ntaps;
     int32_t n_amaps, n_bmaps;    // tensor maps in use
     int32_t BN, nb_atoms, wkb, stages, nacc;
+    int32_t kbs;                 // K-blocks (of 32) per pipeline stage: 4 or 8
     uint32_t idesc;
     uint64_t timeout_ns;
     int32_t num_units;
     int32_t a_box_bytes, b_box_bytes;
     // CONV kind
     int32_t rows_nfirst;         // A map dims (C, N, W, H) instead of (C, W, H, N)
-    int32_t sf_vec4;             // A: a stage's 4 K-blocks are 4 aligned consecutive scale bytes (one tap)
+    int32_t sf_vec4;             // A: each group of 4 K-blocks is 4 aligned consecutive scale bytes (one tap)
     int32_t sfb_vec4;            // B: likewise (the weights' scales along C)
-    int32_t sfb_cached;          // CONV: B scale atoms of every (column tile, stage) built once per CTA
-    int32_t ktiles;              // CONV: stages per tile
+    int32_t sfb_cached;          // CONV: B scale atoms of every (column tile, group) built once per CTA
+    int32_t groups;              // CONV: groups of 4 K-blocks per tile
     int32_t bq, bp, bn;          // A box extents along q, p, n
     int32_t TQ, TP, TN, NT;      // tile counts
-    int32_t Qe, Pe, Ne;          // output extents (row masks)
-    int32_t CB, total_kb;        // K-blocks per tap, K-blocks per tile
+    int32_t Ne;                  // output extent along n (row mask)
+    int32_t CB, total_kb;        // K-blocks per tap, most K-blocks of a tile over the phases
+    // CONV output phases (the input gradient of a strided convolution splits
+    // its output into stride phases with different tap sets; the forward has
+    // one phase).  Units run phase-fastest within a tile so the phases that
+    // interleave in memory are written at about the same time.
+    int32_t nph;
+    int32_t ph_tap0[kMaxPhases];  // first tap of the phase in taps[]
+    int32_t ph_tkb[kMaxPhases];   // K-blocks of a tile of the phase
+    int32_t ph_gofs[kMaxPhases];  // first group of 4 K-blocks of the phase (scale cache index)
+    int32_t ph_Qe[kMaxPhases], ph_Pe[kMaxPhases];   // output extents of the phase (row masks)
+    int64_t ph_out_base[kMaxPhases];
     int32_t a_st_h, a_st_w;      // output coordinate -> scale pixel multiplier
     int32_t Ncols;               // GEMM columns (output channels)
-    // WGRAD kind
+    // WGRAD kind: K is walked in "kits" of 4 K-blocks (one TMA box per operand)
     int32_t MT, Mrows, splits, kiters_total, QG, NC, bqk, P, Q;
     int32_t x_st_h, x_st_w;      // stride of X pixels per output pixel
     // output
@@ -102,8 +116,9 @@ struct alignas(64) GemmParams {
 };
 
 struct UnitInfo {
-    int nk;                 // K iterations (stages) of this unit
-    int kbase;              // WGRAD: first global K iteration
+    int nk;                 // pipeline stages of this unit
+    int ph, tap0, tkb;      // CONV: output phase, its first tap and K-blocks
+    int kbase, nkit;        // WGRAD: first kit and number of kits
     int q0, p0, n0;         // CONV: tile origin
     int m0;                 // WGRAD: first output channel row
     int col0;               // first GEMM column
@@ -116,7 +131,9 @@ __device__ __forceinline__ UnitInfo decode_unit(const GemmParams &p, int u) {
     UnitInfo I{};
     if (KIND == kConv) {
         const int nt = u % p.NT;
-        const int mt = u / p.NT;
+        const int r = u / p.NT;
+        const int ph = r % p.nph;
+        const int mt = r / p.nph;
         const int tq = mt % p.TQ;
         const int tp = (mt / p.TQ) % p.TP;
         const int tn = mt / (p.TQ * p.TP);
@@ -124,7 +141,10 @@ __device__ __forceinline__ UnitInfo decode_unit(const GemmParams &p, int u) {
         I.p0 = tp * p.bp;
         I.n0 = tn * p.bn;
         I.col0 = nt * p.BN;
-        I.nk = (p.total_kb + 3) / 4;
+        I.ph = ph;
+        I.tap0 = p.ph_tap0[ph];
+        I.tkb = p.ph_tkb[ph];
+        I.nk = (I.tkb + p.kbs - 1) / p.kbs;
     } else {
         int r = u;
         const int mt = r % p.MT;
@@ -138,7 +158,9 @@ __device__ __forceinline__ UnitInfo decode_unit(const GemmParams &p, int u) {
         const int64_t k0 = static_cast<int64_t>(I.split) * p.kiters_total / p.splits;
         const int64_t k1 = static_cast<int64_t>(I.split + 1) * p.kiters_total / p.splits;
         I.kbase = static_cast<int>(k0);
-        I.nk = static_cast<int>(k1 - k0);
+        I.nkit = static_cast<int>(k1 - k0);
+        const int ga = p.kbs / 4;
+        I.nk = (I.nkit + ga - 1) / ga;
     }
     return I;
 }
@@ -173,21 +195,45 @@ struct KbWalker {
     }
 };
 
+// Walks the kits of a WGRAD unit as (output row pp, q-group qg, n-chunk nc).
+struct KitWalker {
+    int nc, qg, pp;
+    __device__ __forceinline__ void init(const GemmParams &p, int kit) {
+        nc = kit % p.NC;
+        qg = (kit / p.NC) % p.QG;
+        pp = kit / (p.NC * p.QG);
+    }
+    __device__ __forceinline__ void next(const GemmParams &p) {
+        if (++nc == p.NC) {
+            nc = 0;
+            if (++qg == p.QG) {
+                qg = 0;
+                ++pp;
+            }
+        }
+    }
+};
+
 template <int KIND>
 __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int S = p.stages;                 // at least 4
-    const int a_stage = 128 * 128;
-    const int b_stage = p.BN * 128;
-    const int sfb_stage = 512 * p.nb_atoms;
+    const int S = p.stages;                   // at least 2
+    const int KS = p.kbs;                     // K-blocks per stage
+    const int GA = KS / 4;                    // groups of 4 K-blocks (one scale atom) per stage
+    const int row_bytes = 32 * p.wkb;         // bytes of one operand row of a TMA box
+    const int lg_wkb = p.wkb == 4 ? 2 : (p.wkb == 2 ? 1 : 0);
+    const int a_stage = 128 * 32 * KS;
+    const int b_stage = p.BN * 32 * KS;
+    const int sfa_stage = 512 * GA;
+    const int sfb_stage = 512 * GA * p.nb_atoms;
     uint8_t *sA = smem;
     uint8_t *sB = sA + S * a_stage;
     uint8_t *sSFA = sB + S * b_stage;
-    uint8_t *sSFB = sSFA + S * 512;
-    uint8_t *sSFBc = sSFB + S * sfb_stage;    // cached B atoms: [column tile][stage][atom] x 512 B
-    const int sfbc_bytes = p.sfb_cached ? p.NT * p.ktiles * p.nb_atoms * 512 : 0;
+    uint8_t *sSFB = sSFA + S * sfa_stage;
+    uint8_t *sSFBc = sSFB + S * sfb_stage;    // cached B atoms: [column tile][group][atom] x 512 B
+    const int sfbc_bytes = p.sfb_cached ? p.NT * p.groups * p.nb_atoms * 512 : 0;
     // full[s]: completes when the TMA bytes of stage s have landed AND the
     // scale-gather warp of stage s has arrived (count 2)
     uint64_t *full = reinterpret_cast<uint64_t *>(sSFBc + sfbc_bytes);
@@ -222,17 +268,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     }
     if (KIND == kConv && p.sfb_cached) {
         // every thread helps build the B scale atoms once: item = (column tile,
-        // stage of the tile, atom); lane l writes rows l, l+32, l+64, l+96
-        const int items = p.NT * p.ktiles * p.nb_atoms;
+        // group of 4 K-blocks, atom); lane l writes rows l, l+32, l+64, l+96
+        const int items = p.NT * p.groups * p.nb_atoms;
         for (int item = warp; item < items; item += kGemmThreads / 32) {
             const int at = item % p.nb_atoms;
-            const int ks = (item / p.nb_atoms) % p.ktiles;
-            const int nt = item / (p.nb_atoms * p.ktiles);
+            const int gq = (item / p.nb_atoms) % p.groups;
+            const int nt = item / (p.nb_atoms * p.groups);
+            int ph = 0;
+            while (ph + 1 < p.nph && p.ph_gofs[ph + 1] <= gq) ++ph;
             uint32_t wv[4] = {0u, 0u, 0u, 0u};
             for (int kb = 0; kb < 4; ++kb) {
-                const int g = 4 * ks + kb;
-                if (g >= p.total_kb) break;
-                const ConvTap T = p.taps[g / p.CB];
+                const int g = 4 * (gq - p.ph_gofs[ph]) + kb;
+                if (g >= p.ph_tkb[ph]) break;
+                const ConvTap T = p.taps[p.ph_tap0[ph] + g / p.CB];
                 const uint8_t *bsrc =
                     p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + (g % p.CB) * p.sfb.kb_pitch;
 #pragma unroll
@@ -252,9 +300,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const uint64_t lim = p.timeout_ns;
-    const int sf_cols = 4 + 4 * p.nb_atoms;
-    const int row_bytes = 32 * p.wkb;          // bytes of one operand row of a TMA box
-    const int lg_wkb = p.wkb == 4 ? 2 : (p.wkb == 2 ? 1 : 0);
+    const int sf_cols = GA * (4 + 4 * p.nb_atoms);   // TMEM scale columns per stage
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -266,13 +312,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         bool ok = true;
         for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
-            KbWalker kw{0, 0};
-            int kg = I.kbase, nc = 0, qg = 0, pp = 0;
-            if (KIND == kWgrad) {
-                nc = kg % p.NC;
-                qg = (kg / p.NC) % p.QG;
-                pp = kg / (p.NC * p.QG);
-            }
+            KbWalker kw{I.tap0, 0};
+            KitWalker kt{0, 0, 0};
+            if (KIND == kWgrad) kt.init(p, I.kbase);
             for (int ki = 0; ki < I.nk; ++ki, ++it, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag))) {
                     ok = false;
@@ -281,7 +323,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 uint8_t *a_dst = sA + s * a_stage;
                 uint8_t *b_dst = sB + s * b_stage;
                 if (KIND == kConv) {
-                    const int nkb = min(4, p.total_kb - 4 * ki);
+                    const int nkb = min(KS, I.tkb - KS * ki);
                     const int nbox = nkb >> lg_wkb;
                     if (leader)
                         mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * (p.a_box_bytes + p.b_box_bytes)));
@@ -301,18 +343,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     }
                 } else {
                     const ConvTap T = p.taps[I.tap];
-                    const int nx = nc * row_bytes;
-                    if (leader) {
-                        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.a_box_bytes + p.b_box_bytes));
-                        tma_load_4d(a_dst, &p.amap[0], &full[s], nx, I.m0, qg * p.bqk, pp);
-                        tma_load_4d(b_dst, &p.bmap[T.map], &full[s], nx, I.col0, qg * p.bqk + T.dw, pp + T.dh);
-                    }
-                    if (++nc == p.NC) {
-                        nc = 0;
-                        if (++qg == p.QG) {
-                            qg = 0;
-                            ++pp;
+                    const int nkit = min(GA, I.nkit - GA * ki);
+                    if (leader)
+                        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nkit * (p.a_box_bytes + p.b_box_bytes)));
+                    for (int g = 0; g < nkit; ++g) {
+                        const int nx = kt.nc * row_bytes;
+                        if (leader) {
+                            tma_load_4d(a_dst + g * 128 * 128, &p.amap[0], &full[s], nx, I.m0, kt.qg * p.bqk, kt.pp);
+                            tma_load_4d(b_dst + g * p.BN * 128, &p.bmap[T.map], &full[s], nx, I.col0,
+                                        kt.qg * p.bqk + T.dw, kt.pp + T.dh);
                         }
+                        kt.next(p);
                     }
                 }
                 __syncwarp();
@@ -350,36 +391,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_empty[acc], aph ^ 1u, lim, abort_flag))) break;
             tc_fence_after();
             const uint32_t d_tmem = tmem + acc * p.BN;
-            const int item_base = (I.col0 / p.BN) * p.ktiles * p.nb_atoms;   // cached B atoms of this column tile
+            // cached B atoms of this column tile
+            const int item_base = KIND == kConv ? ((I.col0 / p.BN) * p.groups + p.ph_gofs[I.ph]) * p.nb_atoms : 0;
             for (int ki = 0; ki < I.nk; ++ki, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], ph, lim, abort_flag))) {
                     ok = false;
                     break;
                 }
-                const uint32_t sfa_t = tmem + kSfTmemBase + s * sf_cols;
-                const uint32_t sfb_t = sfa_t + 4;
-                const int nkb = KIND == kConv ? min(4, p.total_kb - 4 * ki) : 4;
+                const uint32_t sf_t = tmem + kSfTmemBase + s * sf_cols;     // SFA groups, then SFB groups
+                const uint32_t sfb_t = sf_t + 4 * GA;
+                const int nkb = KIND == kConv ? min(KS, I.tkb - KS * ki) : 4 * min(GA, I.nkit - GA * ki);
+                const int ngr = (nkb + 3) >> 2;
                 const uint64_t a_s = adesc0 + static_cast<uint64_t>((s * a_stage) >> 4);
                 const uint64_t b_s = bdesc0 + static_cast<uint64_t>((s * b_stage) >> 4);
                 if (leader) {
-                    tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + static_cast<uint64_t>((s * 512) >> 4));
-                    if (KIND == kConv && p.sfb_cached) {
-                        const int item0 = item_base + ki * p.nb_atoms;
-                        for (int a = 0; a < p.nb_atoms; ++a)
-                            tc_cp_32x128b_warpx4(sfb_t + 4 * a,
-                                                 sfbc_desc0 + static_cast<uint64_t>(((item0 + a) * 512) >> 4));
-                    } else {
-                        for (int a = 0; a < p.nb_atoms; ++a)
-                            tc_cp_32x128b_warpx4(sfb_t + 4 * a,
-                                                 sfb_desc0 + static_cast<uint64_t>((s * sfb_stage + a * 512) >> 4));
+                    for (int g = 0; g < ngr; ++g) {
+                        tc_cp_32x128b_warpx4(sf_t + 4 * g, sfa_desc0 + static_cast<uint64_t>((s * sfa_stage + g * 512) >> 4));
+                        for (int a = 0; a < p.nb_atoms; ++a) {
+                            const uint64_t src =
+                                (KIND == kConv && p.sfb_cached)
+                                    ? sfbc_desc0 + static_cast<uint64_t>(((item_base + (ki * GA + g) * p.nb_atoms + a) * 512) >> 4)
+                                    : sfb_desc0 + static_cast<uint64_t>((s * sfb_stage + (g * p.nb_atoms + a) * 512) >> 4);
+                            tc_cp_32x128b_warpx4(sfb_t + 4 * (g * p.nb_atoms + a), src);
+                        }
                     }
                     for (int kb = 0; kb < nkb; ++kb) {
                         const uint32_t j = static_cast<uint32_t>(kb >> lg_wkb);
                         const uint32_t within = static_cast<uint32_t>(kb & (p.wkb - 1));
-                        const uint32_t kbu = static_cast<uint32_t>(kb);
+                        const uint32_t g = static_cast<uint32_t>(kb >> 2), k4 = static_cast<uint32_t>(kb & 3);
                         tc_mma_mxf8f6f4(d_tmem, a_s + j * a_sub + within * 2, b_s + j * b_sub + within * 2,
-                                        p.idesc | (kbu << 29) | (kbu << 4), sfa_t | (kbu << 30), sfb_t | (kbu << 30),
-                                        (ki > 0 || kb > 0) ? 1u : 0u);
+                                        p.idesc | (k4 << 29) | (k4 << 4), (sf_t + 4 * g) | (k4 << 30),
+                                        (sfb_t + 4 * g * p.nb_atoms) | (k4 << 30), (ki > 0 || kb > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                 }
@@ -390,21 +432,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             __syncwarp();
             ++tcount;
         }
-    } else if (sf_warp_index(warp) >= 0) {
+    } else if (sf_warp_index(warp) >= 0 && sf_warp_index(warp) < min(kNumSfWarps, S)) {
         // ------------------------------------------------------------ scale-factor gather
-        // scale warp w handles the stages whose global index is w modulo kNumSfWarps
+        // scale warp w handles the stages whose global index is w modulo nsf.
+        // nsf <= S: a warp's consecutive stages are at most S apart, so when
+        // it waits for slot s it is never two phases ahead of the consumer
+        // (a parity wait cannot tell phase r from phase r - 2)
+        const int nsf = min(kNumSfWarps, S);
         const int sfw = sf_warp_index(warp);
         uint32_t it = 0;             // global index of the first stage of the unit
-        uint32_t g = static_cast<uint32_t>(sfw);   // global index of this warp's next stage
+        uint32_t gnext = static_cast<uint32_t>(sfw);   // global index of this warp's next stage
         int s = sfw % S;
         uint32_t ph = static_cast<uint32_t>(sfw / S) & 1u;
         bool ok = true;
+        const bool skip_b = KIND == kConv && p.sfb_cached;
         for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
             const uint32_t it_unit = it;
             it += static_cast<uint32_t>(I.nk);
-            if (g >= it) continue;
-            const int first = static_cast<int>(g - it_unit);
+            if (gnext >= it) continue;
+            const int first = static_cast<int>(gnext - it_unit);
             // A rows of this lane: m = lane + 32 j
             int ra_h[4], ra_w[4], ra_off[4];
             bool ra_ok[4];
@@ -415,7 +462,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     int iq, ip, in;
                     conv_row(p, m, iq, ip, in);
                     const int q = I.q0 + iq, pr = I.p0 + ip, n = I.n0 + in;
-                    ra_ok[j] = m < p.bq * p.bp * p.bn && q < p.Qe && pr < p.Pe && n < p.Ne;
+                    ra_ok[j] = m < p.bq * p.bp * p.bn && q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
                     ra_h[j] = p.a_st_h * pr;
                     ra_w[j] = p.a_st_w * q;
                     ra_off[j] = (n / p.sfa.row_div) * p.sfa.row_pitch;
@@ -439,115 +486,125 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     rb_ok[at][j] = at < p.nb_atoms && rl < p.BN && r < p.sfb.rows;
                     rb_off[at][j] = (r / p.sfb.row_div) * p.sfb.row_pitch;
                 }
-            KbWalker kw{0, 0};
-            if (KIND == kConv) kw.advance(4 * first, p.CB);
-            int kg = I.kbase + first;
-            int nc = 0, qg = 0, pp = 0;
-            if (KIND == kWgrad) {
-                nc = kg % p.NC;
-                qg = (kg / p.NC) % p.QG;
-                pp = kg / (p.NC * p.QG);
-            }
-            for (int ki = first; ki < I.nk; ki += kNumSfWarps) {
-                uint32_t wa[4] = {0u, 0u, 0u, 0u};      // A atom bytes: row lane+32j, byte kb
-                uint32_t wb[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-                if (KIND == kConv && p.sf_vec4) {
-                    // one tap, channel blocks cb..cb+3: one 32-bit load per row
-                    const ConvTap T = p.taps[kw.tap];
-                    const int cb = kw.cb;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
-                        if (ra_ok[j] && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W)
-                            wa[j] = __ldg(reinterpret_cast<const uint32_t *>(
-                                p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch + ra_off[j] + cb));
-                    }
-                    if (!p.sfb_cached) {
-                        const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb;
-#pragma unroll
-                        for (int at = 0; at < 2; ++at)
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                if (rb_ok[at][j])
-                                    wb[at][j] = __ldg(reinterpret_cast<const uint32_t *>(bsrc + rb_off[at][j]));
-                    }
-                    kw.advance(4 * kNumSfWarps, p.CB);
-                } else if (KIND == kConv) {
-                    const int nkb = min(4, p.total_kb - 4 * ki);
+            KbWalker kw{I.tap0, 0};
+            KitWalker kt{0, 0, 0};
+            if (KIND == kConv) kw.advance(KS * first, p.CB);
+            else kt.init(p, I.kbase + GA * first);
+            for (int ki = first; ki < I.nk; ki += nsf) {
+                uint32_t wa[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};          // [group][row j]
+                uint32_t wb[2][2][4] = {};                                          // [group][atom][row j]
+                if (KIND == kConv) {
+                    const int nkb = min(KS, I.tkb - KS * ki);
                     KbWalker k2 = kw;
-                    for (int kb = 0; kb < nkb; ++kb) {
-                        const ConvTap T = p.taps[k2.tap];
-                        const int cb = k2.cb;
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
-                            if (ra_ok[j] && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W) {
-                                const uint8_t *src = p.sfa.base +
-                                                     (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
-                                                     ra_off[j] + cb * p.sfa.kb_pitch;
-                                wa[j] |= static_cast<uint32_t>(__ldg(src)) << (8 * kb);
+                    for (int g = 0; g < 2; ++g) {
+                        if (4 * g >= nkb) break;
+                        if (p.sf_vec4) {
+                            // one tap, channel blocks cb..cb+3: one 32-bit load per row
+                            const ConvTap T = p.taps[k2.tap];
+                            const int cb = k2.cb;
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
+                                if (ra_ok[j] && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W)
+                                    wa[g][j] = __ldg(reinterpret_cast<const uint32_t *>(
+                                        p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
+                                        ra_off[j] + cb));
+                            }
+                            if (!skip_b) {
+                                const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb;
+#pragma unroll
+                                for (int at = 0; at < 2; ++at)
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j)
+                                        if (rb_ok[at][j])
+                                            wb[g][at][j] = __ldg(reinterpret_cast<const uint32_t *>(bsrc + rb_off[at][j]));
+                            }
+                            k2.advance(4, p.CB);
+                        } else {
+                            for (int kb = 0; kb < 4 && 4 * g + kb < nkb; ++kb) {
+                                const ConvTap T = p.taps[k2.tap];
+                                const int cb = k2.cb;
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
+                                    if (ra_ok[j] && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W) {
+                                        const uint8_t *src = p.sfa.base +
+                                                             (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
+                                                             ra_off[j] + cb * p.sfa.kb_pitch;
+                                        wa[g][j] |= static_cast<uint32_t>(__ldg(src)) << (8 * kb);
+                                    }
+                                }
+                                if (!skip_b) {
+                                    const uint8_t *bsrc =
+                                        p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
+#pragma unroll
+                                    for (int at = 0; at < 2; ++at)
+#pragma unroll
+                                        for (int j = 0; j < 4; ++j)
+                                            if (rb_ok[at][j])
+                                                wb[g][at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                                }
+                                k2.advance(1, p.CB);
                             }
                         }
-                        if (!p.sfb_cached) {
-                            const uint8_t *bsrc =
-                                p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
+                    }
+                    kw.advance(KS * nsf, p.CB);
+                } else {
+                    const ConvTap T = p.taps[I.tap];
+                    const int nkit = min(GA, I.nkit - GA * ki);
+                    KitWalker k2 = kt;
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        if (g >= nkit) break;
+                        for (int kb = 0; kb < 4; ++kb) {
+                            const int q = k2.qg * p.bqk + (kb >> lg_wkb);
+                            const int nb = k2.nc * p.wkb + (kb & (p.wkb - 1));
+                            if (q >= p.Q) continue;
+                            const uint8_t *asrc = p.sfa.base +
+                                                  (static_cast<int64_t>(k2.pp) * p.Q + q) * p.sfa.pix_pitch +
+                                                  nb * p.sfa.kb_pitch;
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                if (ra_ok[j]) wa[g][j] |= static_cast<uint32_t>(__ldg(asrc + ra_off[j])) << (8 * kb);
+                            const int hh = p.x_st_h * k2.pp + T.sf_dh, ww = p.x_st_w * q + T.sf_dw;
+                            if (hh < 0 || hh >= p.sfb.H || ww < 0 || ww >= p.sfb.W) continue;
+                            const uint8_t *bsrc = p.sfb.base +
+                                                  (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
+                                                  nb * p.sfb.kb_pitch;
 #pragma unroll
                             for (int at = 0; at < 2; ++at)
 #pragma unroll
                                 for (int j = 0; j < 4; ++j)
                                     if (rb_ok[at][j])
-                                        wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                                        wb[g][at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
                         }
-                        k2.advance(1, p.CB);
+                        k2.next(p);
                     }
-                    kw.advance(4 * kNumSfWarps, p.CB);
-                } else {
-                    const ConvTap T = p.taps[I.tap];
-                    for (int kb = 0; kb < 4; ++kb) {
-                        const int q = qg * p.bqk + (kb >> lg_wkb);
-                        const int nb = nc * p.wkb + (kb & (p.wkb - 1));
-                        if (q >= p.Q) continue;
-                        const uint8_t *asrc = p.sfa.base + (static_cast<int64_t>(pp) * p.Q + q) * p.sfa.pix_pitch +
-                                              nb * p.sfa.kb_pitch;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            if (ra_ok[j]) wa[j] |= static_cast<uint32_t>(__ldg(asrc + ra_off[j])) << (8 * kb);
-                        const int hh = p.x_st_h * pp + T.sf_dh, ww = p.x_st_w * q + T.sf_dw;
-                        if (hh < 0 || hh >= p.sfb.H || ww < 0 || ww >= p.sfb.W) continue;
-                        const uint8_t *bsrc = p.sfb.base + (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
-                                              nb * p.sfb.kb_pitch;
-#pragma unroll
-                        for (int at = 0; at < 2; ++at)
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                if (rb_ok[at][j]) wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
-                    }
-                    // advance the (pixel row, q-group, n-chunk) walker by kNumSfWarps K iterations
-                    for (int step = 0; step < kNumSfWarps; ++step)
-                        if (++nc == p.NC) {
-                            nc = 0;
-                            if (++qg == p.QG) {
-                                qg = 0;
-                                ++pp;
-                            }
-                        }
+                    for (int step = 0; step < GA * nsf; ++step) kt.next(p);
                 }
                 if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) {
                     ok = false;
                     break;
                 }
-                *reinterpret_cast<uint4 *>(sSFA + s * 512 + lane * 16) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-                if (!(KIND == kConv && p.sfb_cached))
-                    *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + lane * 16) =
-                        make_uint4(wb[0][0], wb[0][1], wb[0][2], wb[0][3]);
-                if (!(KIND == kConv && p.sfb_cached) && p.nb_atoms > 1)
-                    *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + 512 + lane * 16) =
-                        make_uint4(wb[1][0], wb[1][1], wb[1][2], wb[1][3]);
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    if (g >= GA) break;
+                    *reinterpret_cast<uint4 *>(sSFA + s * sfa_stage + g * 512 + lane * 16) =
+                        make_uint4(wa[g][0], wa[g][1], wa[g][2], wa[g][3]);
+                    if (!skip_b) {
+                        *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + (g * p.nb_atoms) * 512 + lane * 16) =
+                            make_uint4(wb[g][0][0], wb[g][0][1], wb[g][0][2], wb[g][0][3]);
+                        if (p.nb_atoms > 1)
+                            *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + (g * p.nb_atoms + 1) * 512 + lane * 16) =
+                                make_uint4(wb[g][1][0], wb[g][1][1], wb[g][1][2], wb[g][1][3]);
+                    }
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[s]);
-                g += kNumSfWarps;
-                s += kNumSfWarps;
+                gnext += nsf;
+                s += nsf;
                 while (s >= S) {
                     s -= S;
                     ph ^= 1u;
@@ -567,8 +624,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 int iq, ip, in;
                 conv_row(p, m, iq, ip, in);
                 const int q = I.q0 + iq, pr = I.p0 + ip, n = I.n0 + in;
-                row_ok = m < p.bq * p.bp * p.bn && q < p.Qe && pr < p.Pe && n < p.Ne;
-                row_off = p.out_base + n * p.os_n + pr * p.os_p + q * p.os_q;
+                row_ok = m < p.bq * p.bp * p.bn && q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
+                row_off = p.ph_out_base[I.ph] + n * p.os_n + pr * p.os_p + q * p.os_q;
             } else {
                 const int k = I.m0 + m;
                 row_ok = k < p.Mrows;

@@ -196,23 +196,48 @@ const uint64_t kDefaultTimeoutNs = 4000000000ull;
 
 template <int KIND>
 mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
-    const int per_stage = 128 * 128 + P.BN * 128 + 512 + 512 * P.nb_atoms;
-    const int sf_cols = 4 + 4 * P.nb_atoms;
     // CONV: the weights' scale atoms are the same for every output tile of a
-    // column tile; build them once per CTA when they fit in 16 KB
-    P.ktiles = (P.total_kb + 3) / 4;
-    const int cache = KIND == kConv ? P.NT * P.ktiles * P.nb_atoms * 512 : 0;
+    // column tile; build them once per CTA when they fit in 16 KB and cannot
+    // be read four bytes at a time
+    // groups of 4 K-blocks: per phase for CONV (their sum indexes the scale
+    // cache), per unit otherwise
+    if (KIND == kConv) {
+        P.groups = 0;
+        P.total_kb = 0;
+        for (int ph = 0; ph < P.nph; ++ph) {
+            P.ph_gofs[ph] = P.groups;
+            P.groups += (P.ph_tkb[ph] + 3) / 4;
+            P.total_kb = std::max(P.total_kb, P.ph_tkb[ph]);
+        }
+    } else {
+        P.groups = (P.total_kb + 3) / 4;
+    }
+    const int cache = KIND == kConv ? P.NT * P.groups * P.nb_atoms * 512 : 0;
     P.sfb_cached = KIND == kConv && cache <= 16384 && !P.sfb_vec4;
     // the 32-bit scale path reads B four bytes at a time unless B is cached
     if (!P.sfb_cached && !P.sfb_vec4) P.sf_vec4 = 0;
     const int fixed = 1024 + 64 * 8 + 64 + (P.sfb_cached ? cache : 0);
-    int S = std::min(8, (d.max_smem - fixed) / per_stage);
-    S = std::min(S, (kTmemCols - kSfTmemBase) / sf_cols);
-    if (S < 4) return fail(MQC_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+    auto stages_for = [&](int kbs, int &S) {
+        const int ga = kbs / 4;
+        const int per_stage = 128 * 32 * kbs + P.BN * 32 * kbs + 512 * ga + 512 * ga * P.nb_atoms;
+        const int sf_cols = ga * (4 + 4 * P.nb_atoms);
+        S = std::min(8, (d.max_smem - fixed) / per_stage);
+        S = std::min(S, (kTmemCols - kSfTmemBase) / sf_cols);
+        return per_stage;
+    };
+    // 8 K-blocks per stage (twice the MMAs per barrier round trip) when at
+    // least 3 such stages fit and the tile has more than 4 K-blocks
+    int S8 = 0, S4 = 0;
+    const int ps8 = stages_for(8, S8), ps4 = stages_for(4, S4);
+    const bool long_k = KIND == kConv ? P.total_kb > 4 : P.kiters_total > 1;
+    P.kbs = (long_k && S8 >= 3) ? 8 : 4;
+    const int S = P.kbs == 8 ? S8 : S4;
+    const int per_stage = P.kbs == 8 ? ps8 : ps4;
+    if (S < 3) return fail(MQC_ERR_UNSUPPORTED, "tile does not fit in shared memory");
     P.stages = S;
     P.nacc = (P.BN <= 128) ? 2 : 1;
     P.timeout_ns = kDefaultTimeoutNs;
-    const int smem = fixed + P.stages * per_stage;
+    const int smem = fixed + S * per_stage;
     if (!d.gemm_attr[KIND]) {
         cudaError_t e = cudaFuncSetAttribute(conv_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              d.max_smem);
@@ -453,8 +478,6 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     choose_rows(Q, P, N, G.bq, G.bp, G.bn);
     G.BN = choose_bn(K);
     G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
-    G.Qe = Q;
-    G.Pe = P;
     G.Ne = N;
     G.TQ = static_cast<int32_t>(ceil_div(Q, G.bq));
     G.TP = static_cast<int32_t>(ceil_div(P, G.bp));
@@ -517,7 +540,12 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
                 T.sf_dh = T.sf_dw = -30000;
             }
         }
-    G.total_kb = G.ntaps * G.CB;
+    G.nph = 1;
+    G.ph_tap0[0] = 0;
+    G.ph_tkb[0] = G.ntaps * G.CB;
+    G.ph_Qe[0] = Q;
+    G.ph_Pe[0] = P;
+    G.ph_out_base[0] = 0;
     for (int i = 0; i < sh * sw; ++i)          // unused phases get a valid copy (never read)
         if (!phase_ok[i]) G.amap[i] = G.amap[0];
     G.n_amaps = sh * sw;
@@ -544,7 +572,6 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     G.sfb_vec4 = G.CB % 4 == 0 && G.sfb.tap_pitch % 4 == 0 && G.sfb.row_pitch % 4 == 0 &&
                  (reinterpret_cast<uintptr_t>(ws) & 3u) == 0;
     G.out = y;
-    G.out_base = 0;
     G.os_q = 1;
     G.os_p = Q;
     G.os_n = int64_t(K) * P * Q;
@@ -569,51 +596,65 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
     const int64_t Kp = round_up(K, 16);
     const bool sqg = gf->block == MQC_BLOCK_SQ32, sqw = wf->block == MQC_BLOCK_SQ32;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    // output stride phases (ah, aw) with at least one row; the first one has
+    // the largest extents and sets the tiling shared by a launch
+    if (sh * sw > 64) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_data: stride product above 64");
+    int phases[64][2];
+    int nphase = 0;
     for (int ah = 0; ah < sh; ++ah)
-        for (int aw = 0; aw < sw; ++aw) {
-            const int Pe = static_cast<int>(ceil_div(H - ah, sh)), Qe = static_cast<int>(ceil_div(W - aw, sw));
-            if (Pe <= 0 || Qe <= 0) continue;
-            GemmParams G;
-            memset(&G, 0, sizeof G);
-            G.CB = static_cast<int32_t>(nb32(Kp));
-            G.wkb = largest_wkb(G.CB);
-            choose_rows(Qe, Pe, N, G.bq, G.bp, G.bn);
-            G.BN = choose_bn(C);
-            G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
-            G.Qe = Qe;
-            G.Pe = Pe;
-            G.Ne = N;
-            G.TQ = static_cast<int32_t>(ceil_div(Qe, G.bq));
-            G.TP = static_cast<int32_t>(ceil_div(Pe, G.bp));
-            G.TN = static_cast<int32_t>(ceil_div(N, G.bn));
-            G.NT = static_cast<int32_t>(ceil_div(C, G.BN));
-            G.Ncols = C;
-            G.a_st_h = 1;
-            G.a_st_w = 1;
-            G.idesc = make_idesc_mx(mma_fmt(gf->fmt), mma_fmt(wf->fmt), 128, G.BN);
-            st = MQC_ERR_CUDA;
-            for (int attempt = 0; attempt < 2 && st != MQC_OK; ++attempt) {
-                G.rows_nfirst = attempt;
-                if (!G.rows_nfirst) {
-                    const uint64_t dims[4] = {uint64_t(Kp), uint64_t(Q), uint64_t(P), uint64_t(N)};
-                    const uint64_t strd[3] = {uint64_t(N) * Kp, uint64_t(Q) * N * Kp, uint64_t(Kp)};
-                    const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bq), uint32_t(G.bp), uint32_t(G.bn)};
-                    st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
-                } else {
-                    const uint64_t dims[4] = {uint64_t(Kp), uint64_t(N), uint64_t(Q), uint64_t(P)};
-                    const uint64_t strd[3] = {uint64_t(Kp), uint64_t(N) * Kp, uint64_t(Q) * N * Kp};
-                    const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bn), uint32_t(G.bq), uint32_t(G.bp)};
-                    st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
-                }
+        for (int aw = 0; aw < sw; ++aw)
+            if (H - ah > 0 && W - aw > 0) {
+                phases[nphase][0] = ah;
+                phases[nphase][1] = aw;
+                ++nphase;
             }
-            if (st != MQC_OK) return st;
-            {
-                const uint64_t dims[3] = {uint64_t(Kp), uint64_t(C), uint64_t(R) * S};
-                const uint64_t strd[2] = {uint64_t(Kp), uint64_t(C) * Kp};
-                const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(G.BN), 1u};
-                if ((st = encode_codes_map(&G.bmap[0], wq, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
+    const int Pe0 = static_cast<int>(ceil_div(H, sh)), Qe0 = static_cast<int>(ceil_div(W, sw));
+    for (int first = 0; first < nphase; first += kMaxPhases) {
+        const int nph = std::min(kMaxPhases, nphase - first);
+        GemmParams G;
+        memset(&G, 0, sizeof G);
+        G.CB = static_cast<int32_t>(nb32(Kp));
+        G.wkb = largest_wkb(G.CB);
+        choose_rows(Qe0, Pe0, N, G.bq, G.bp, G.bn);
+        G.BN = choose_bn(C);
+        G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
+        G.Ne = N;
+        G.TQ = static_cast<int32_t>(ceil_div(Qe0, G.bq));
+        G.TP = static_cast<int32_t>(ceil_div(Pe0, G.bp));
+        G.TN = static_cast<int32_t>(ceil_div(N, G.bn));
+        G.NT = static_cast<int32_t>(ceil_div(C, G.BN));
+        G.Ncols = C;
+        G.a_st_h = 1;
+        G.a_st_w = 1;
+        G.idesc = make_idesc_mx(mma_fmt(gf->fmt), mma_fmt(wf->fmt), 128, G.BN);
+        st = MQC_ERR_CUDA;
+        for (int attempt = 0; attempt < 2 && st != MQC_OK; ++attempt) {
+            G.rows_nfirst = attempt;
+            if (!G.rows_nfirst) {
+                const uint64_t dims[4] = {uint64_t(Kp), uint64_t(Q), uint64_t(P), uint64_t(N)};
+                const uint64_t strd[3] = {uint64_t(N) * Kp, uint64_t(Q) * N * Kp, uint64_t(Kp)};
+                const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bq), uint32_t(G.bp), uint32_t(G.bn)};
+                st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
+            } else {
+                const uint64_t dims[4] = {uint64_t(Kp), uint64_t(N), uint64_t(Q), uint64_t(P)};
+                const uint64_t strd[3] = {uint64_t(Kp), uint64_t(N) * Kp, uint64_t(Q) * N * Kp};
+                const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bn), uint32_t(G.bq), uint32_t(G.bp)};
+                st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
             }
-            G.ntaps = 0;
+        }
+        if (st != MQC_OK) return st;
+        {
+            const uint64_t dims[3] = {uint64_t(Kp), uint64_t(C), uint64_t(R) * S};
+            const uint64_t strd[2] = {uint64_t(Kp), uint64_t(C) * Kp};
+            const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(G.BN), 1u};
+            if ((st = encode_codes_map(&G.bmap[0], wq, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
+        }
+        // taps of each phase: kernel offsets r with (ah + pad - r) divisible by the stride
+        G.ntaps = 0;
+        G.nph = nph;
+        for (int k = 0; k < nph; ++k) {
+            const int ah = phases[first + k][0], aw = phases[first + k][1];
+            G.ph_tap0[k] = G.ntaps;
             for (int r = 0; r < R; ++r) {
                 if (((ah + c->pad_h - r) % sh + sh) % sh != 0) continue;
                 const int dr = (ah + c->pad_h - r) / sh;
@@ -627,37 +668,40 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
                     T.btap = static_cast<int16_t>(r * S + s);
                 }
             }
-            G.total_kb = G.ntaps * G.CB;
-            G.n_amaps = 1;
-            G.n_bmaps = 1;
-            G.a_box_bytes = 32 * G.wkb * G.bq * G.bp * G.bn;
-            G.b_box_bytes = 32 * G.wkb * G.BN;
-            G.sfa.base = gs;
-            G.sfa.pix_pitch = (sqg ? nb32(N) : N) * nb32(Kp);
-            G.sfa.row_div = sqg ? 32 : 1;
-            G.sfa.row_pitch = static_cast<int32_t>(nb32(Kp));
-            G.sfa.kb_pitch = 1;
-            G.sfa.rows = N;
-            G.sfa.H = P;
-            G.sfa.W = Q;
-            G.sfb.base = ws;
-            G.sfb.tap_pitch = nb32(Kp) * (sqw ? nb32(C) : C);
-            G.sfb.row_div = sqw ? 32 : 1;
-            G.sfb.row_pitch = 1;
-            G.sfb.kb_pitch = static_cast<int32_t>(sqw ? nb32(C) : C);
-            G.sfb.rows = C;
-            G.sf_vec4 = G.CB % 4 == 0 && G.sfa.pix_pitch % 4 == 0 && G.sfa.row_pitch % 4 == 0 &&
-                        (reinterpret_cast<uintptr_t>(gs) & 3u) == 0;
-            G.sfb_vec4 = false;   // the weights' scales run along K with a stride of C per block
-            G.out = gx;
-            G.out_base = int64_t(ah) * W + aw;
-            G.os_q = sw;
-            G.os_p = int64_t(sh) * W;
-            G.os_n = int64_t(C) * H * W;
-            G.os_c = int64_t(H) * W;
-            G.num_units = G.TQ * G.TP * G.TN * G.NT;
-            if ((st = launch_gemm<kConv>(G, *dv, strm)) != MQC_OK) return st;
+            G.ph_tkb[k] = (G.ntaps - G.ph_tap0[k]) * G.CB;
+            G.ph_Pe[k] = static_cast<int32_t>(ceil_div(H - ah, sh));
+            G.ph_Qe[k] = static_cast<int32_t>(ceil_div(W - aw, sw));
+            G.ph_out_base[k] = int64_t(ah) * W + aw;
         }
+        G.n_amaps = 1;
+        G.n_bmaps = 1;
+        G.a_box_bytes = 32 * G.wkb * G.bq * G.bp * G.bn;
+        G.b_box_bytes = 32 * G.wkb * G.BN;
+        G.sfa.base = gs;
+        G.sfa.pix_pitch = (sqg ? nb32(N) : N) * nb32(Kp);
+        G.sfa.row_div = sqg ? 32 : 1;
+        G.sfa.row_pitch = static_cast<int32_t>(nb32(Kp));
+        G.sfa.kb_pitch = 1;
+        G.sfa.rows = N;
+        G.sfa.H = P;
+        G.sfa.W = Q;
+        G.sfb.base = ws;
+        G.sfb.tap_pitch = nb32(Kp) * (sqw ? nb32(C) : C);
+        G.sfb.row_div = sqw ? 32 : 1;
+        G.sfb.row_pitch = 1;
+        G.sfb.kb_pitch = static_cast<int32_t>(sqw ? nb32(C) : C);
+        G.sfb.rows = C;
+        G.sf_vec4 = G.CB % 4 == 0 && G.sfa.pix_pitch % 4 == 0 && G.sfa.row_pitch % 4 == 0 &&
+                    (reinterpret_cast<uintptr_t>(gs) & 3u) == 0;
+        G.sfb_vec4 = false;   // the weights' scales run along K with a stride of C per block
+        G.out = gx;
+        G.os_q = sw;
+        G.os_p = int64_t(sh) * W;
+        G.os_n = int64_t(C) * H * W;
+        G.os_c = int64_t(H) * W;
+        G.num_units = G.TQ * G.TP * G.TN * G.nph * G.NT;
+        if ((st = launch_gemm<kConv>(G, *dv, strm)) != MQC_OK) return st;
+    }
     return MQC_OK;
 }
 

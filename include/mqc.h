@@ -159,8 +159,10 @@ MQC_API mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_m
 
 /* Input gradient, Eq. 2: G_X = W^T * G_Y as the GEMM
  * G_X'{Cin,N} = W_f^T . G_Yf{Cout,N} of section IV-B, computed directly as a
- * transposed convolution (one implicit GEMM per stride phase); no G_X' is
- * materialized.
+ * transposed convolution: one implicit GEMM per output stride phase, up to
+ * four phases per kernel launch, their tiles interleaved so that the
+ * phases' outputs (which interleave in memory) are written together; no
+ * G_X' is materialized.  stride_h * stride_w must be at most 64.
  *   wq, ws  W quantized with blocks along K: block B32 or SQ32, order AB.
  *   gq, gs  G_Y quantized with blocks along K: block A32 or SQ32, order BA.
  *   gx      fp32 output [N][C][H][W] (overwritten).

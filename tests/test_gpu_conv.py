@@ -84,7 +84,18 @@ BWD_CASES = [
 ]
 
 
-@pytest.mark.parametrize("case", BWD_CASES)
+# input-gradient cases beyond the shared ones: output stride phases without
+# taps (1x1 stride 2), nine phases over three launches (stride 3), a 5x5
+# kernel with uneven tap counts per phase, unequal phase extents (odd H, W)
+DGRAD_CASES = BWD_CASES + [
+    (4, 32, 10, 9, 32, 1, 1, 2, 0),
+    (2, 32, 11, 10, 48, 3, 3, 3, 1),
+    (3, 16, 13, 12, 32, 5, 5, 2, 2),
+    (2, 64, 7, 9, 160, 3, 3, 2, 1),
+]
+
+
+@pytest.mark.parametrize("case", DGRAD_CASES)
 @pytest.mark.parametrize("sq", [False, True])
 def test_conv_bwd_data_parity(mqc, orc, case, sq):
     N, C, H, W, K, R, S, st, pad = case

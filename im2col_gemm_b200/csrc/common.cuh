@@ -19,6 +19,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Unsigned division by a divisor d >= 1 fixed at launch, for dividends below
+// 2^31: multiply by a rounded-up reciprocal and shift (Granlund and
+// Montgomery, "Division by invariant integers using multiplication", PLDI
+// 1994).  With l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
+// floor(n / d) = (hi32(n * m) + n) >> l; the host builds (d, m, l).
+struct FastDiv {
+    uint32_t d, m, l;
+#ifdef __CUDACC__
+    __device__ __forceinline__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> l; }
+    __device__ __forceinline__ uint32_t mod(uint32_t n) const { return n - div(n) * d; }
+#endif
+};
+
 __device__ __forceinline__ void record_device_error(int code) {
     atomicCAS(&g_mqc_device_error, 0, code);
 }
@@ -118,6 +131,15 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
         "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
         "%5, %6}], [%2];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
+                                            int c2, int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+        "%5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
         : "memory");
 }
 

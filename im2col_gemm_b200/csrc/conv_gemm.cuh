@@ -53,12 +53,12 @@ constexpr int kSfTmemBase = 256;
 enum GemmKind : int { kConv = 0, kWgrad = 1 };
 
 // Where the E8M0 scale of (row, K-block) of an operand lives:
-//   base + pixel*pix_pitch + (row/row_div)*row_pitch + kblock*kb_pitch (+ tap*tap_pitch)
+//   base + pixel*pix_pitch + (row >> row_shift)*row_pitch + kblock*kb_pitch (+ tap*tap_pitch)
 struct ScaleSrc {
     const uint8_t *base;
     int64_t pix_pitch;
     int64_t tap_pitch;
-    int32_t row_div;
+    int32_t row_shift;     // 5 when 32 rows share a scale (square blocks), else 0
     int32_t row_pitch;
     int32_t kb_pitch;
     int32_t rows;
@@ -70,6 +70,7 @@ struct ConvTap {
     int16_t sf_dh, sf_dw;  // offsets of the pixel whose scales apply
     int16_t map;           // tensor map (stride phase) of the shifted operand
     int16_t btap;          // CONV: tap index of W; WGRAD: output offset r*S + s
+    int16_t aw;            // CONV with interleaved rows: the interleave slot this tap feeds
 };
 
 struct alignas(64) GemmParams {
@@ -87,6 +88,12 @@ struct alignas(64) GemmParams {
     int32_t a_box_bytes, b_box_bytes;
     // CONV kind
     int32_t rows_nfirst;         // A map dims (C, N, W, H) instead of (C, W, H, N)
+    // rows interleaved along the output width: tile row m = aw + sub * (q +
+    // bq * (p + bp * n)) lands on output column sub * q + aw.  The input
+    // gradient of a stride-s convolution uses sub = s: a tap feeds only the
+    // rows of its slot aw, the other rows of its A box are zero (the box
+    // reads them out of range).  sub = 1 otherwise.
+    int32_t sub;
     int32_t sf_vec4;             // A: each group of 4 K-blocks is 4 aligned consecutive scale bytes (one tap)
     int32_t sfb_vec4;            // B: likewise (the weights' scales along C)
     int32_t sfb_cached;          // CONV: B scale atoms of every (column tile, group) built once per CTA
@@ -109,6 +116,8 @@ struct alignas(64) GemmParams {
     int32_t Ncols;               // GEMM columns (output channels)
     // WGRAD kind: K is walked in "kits" of 4 K-blocks (one TMA box per operand)
     int32_t MT, Mrows, splits, kiters_total, QG, NC, bqk, P, Q;
+    // the divisions of the unit and row decoding, by launch constants
+    FastDiv fd_NT, fd_nph, fd_TQ, fd_TP, fd_sub, fd_bq, fd_bp, fd_bn, fd_MT, fd_ntaps, fd_splits;
     int32_t x_st_h, x_st_w;      // stride of X pixels per output pixel
     // output
     float *out;
@@ -117,6 +126,7 @@ struct alignas(64) GemmParams {
 
 struct UnitInfo {
     int nk;                 // pipeline stages of this unit
+    int nt;                 // column tile
     int ph, tap0, tkb;      // CONV: output phase, its first tap and K-blocks
     int kbase, nkit;        // WGRAD: first kit and number of kits
     int q0, p0, n0;         // CONV: tile origin
@@ -130,51 +140,63 @@ template <int KIND>
 __device__ __forceinline__ UnitInfo decode_unit(const GemmParams &p, int u) {
     UnitInfo I{};
     if (KIND == kConv) {
-        const int nt = u % p.NT;
-        const int r = u / p.NT;
-        const int ph = r % p.nph;
-        const int mt = r / p.nph;
-        const int tq = mt % p.TQ;
-        const int tp = (mt / p.TQ) % p.TP;
-        const int tn = mt / (p.TQ * p.TP);
+        const uint32_t r = p.fd_NT.div(u);
+        const int nt = u - static_cast<int>(r) * p.NT;
+        const uint32_t mt = p.fd_nph.div(r);
+        const int ph = static_cast<int>(r - mt * p.nph);
+        const uint32_t m2 = p.fd_TQ.div(mt);
+        const int tq = static_cast<int>(mt - m2 * p.TQ);
+        const uint32_t tn = p.fd_TP.div(m2);
+        const int tp = static_cast<int>(m2 - tn * p.TP);
+        I.nt = nt;
         I.q0 = tq * p.bq;
         I.p0 = tp * p.bp;
-        I.n0 = tn * p.bn;
+        I.n0 = static_cast<int>(tn) * p.bn;
         I.col0 = nt * p.BN;
         I.ph = ph;
         I.tap0 = p.ph_tap0[ph];
         I.tkb = p.ph_tkb[ph];
         I.nk = (I.tkb + p.kbs - 1) / p.kbs;
     } else {
-        int r = u;
-        const int mt = r % p.MT;
-        r /= p.MT;
-        const int nt = r % p.NT;
-        r /= p.NT;
-        I.tap = r % p.ntaps;
-        I.split = r / p.ntaps;
+        const uint32_t r1 = p.fd_MT.div(u);
+        const int mt = u - static_cast<int>(r1) * p.MT;
+        const uint32_t r2 = p.fd_NT.div(r1);
+        const int nt = static_cast<int>(r1 - r2 * p.NT);
+        const uint32_t sp = p.fd_ntaps.div(r2);
+        I.tap = static_cast<int>(r2 - sp * p.ntaps);
+        I.split = static_cast<int>(sp);
+        I.nt = nt;
         I.m0 = mt * 128;
         I.col0 = nt * p.BN;
-        const int64_t k0 = static_cast<int64_t>(I.split) * p.kiters_total / p.splits;
-        const int64_t k1 = static_cast<int64_t>(I.split + 1) * p.kiters_total / p.splits;
-        I.kbase = static_cast<int>(k0);
-        I.nkit = static_cast<int>(k1 - k0);
+        // split s covers kits [s*K/splits, (s+1)*K/splits); s*K < 2^31 (host check)
+        const int k0 = static_cast<int>(p.fd_splits.div(static_cast<uint32_t>(I.split * p.kiters_total)));
+        const int k1 = static_cast<int>(p.fd_splits.div(static_cast<uint32_t>((I.split + 1) * p.kiters_total)));
+        I.kbase = k0;
+        I.nkit = k1 - k0;
         const int ga = p.kbs / 4;
         I.nk = (I.nkit + ga - 1) / ga;
     }
     return I;
 }
 
-// Row m (0..127) of a CONV tile -> output coordinates within the tile.
-__device__ __forceinline__ void conv_row(const GemmParams &p, int m, int &iq, int &ip, int &in) {
+// Row m (0..127) of a CONV tile -> interleave slot and output coordinates
+// within the tile.
+__device__ __forceinline__ void conv_row(const GemmParams &p, int m, int &aw, int &iq, int &ip, int &in) {
     if (p.rows_nfirst) {
-        in = m % p.bn;
-        iq = (m / p.bn) % p.bq;
-        ip = m / (p.bn * p.bq);
+        const uint32_t t = p.fd_bn.div(m);
+        in = m - static_cast<int>(t) * p.bn;
+        const uint32_t t2 = p.fd_bq.div(t);
+        iq = static_cast<int>(t - t2 * p.bq);
+        ip = static_cast<int>(t2);
+        aw = 0;
     } else {
-        iq = m % p.bq;
-        ip = (m / p.bq) % p.bp;
-        in = m / (p.bq * p.bp);
+        const uint32_t t = p.fd_sub.div(m);
+        aw = m - static_cast<int>(t) * p.sub;
+        const uint32_t t2 = p.fd_bq.div(t);
+        iq = static_cast<int>(t - t2 * p.bq);
+        const uint32_t t3 = p.fd_bp.div(t2);
+        ip = static_cast<int>(t2 - t3 * p.bp);
+        in = static_cast<int>(t3);
     }
 }
 
@@ -214,7 +236,12 @@ struct KitWalker {
     }
 };
 
-template <int KIND>
+// SFV4 (CONV only): the A scales of 4 consecutive K-blocks are 4 aligned
+// bytes of one tap and are read with one 32-bit load per row; otherwise one
+// byte per (row, K-block).  The choice is a template parameter so that each
+// kernel carries only one gather path (the per-stage code of all roles has to
+// share the instruction cache).
+template <int KIND, bool SFV4>
 __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
@@ -288,7 +315,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     const int rl = 128 * at + 32 * j + lane;
                     const int r = nt * p.BN + rl;
                     if (rl < p.BN && r < p.sfb.rows)
-                        wv[j] |= static_cast<uint32_t>(__ldg(bsrc + (r / p.sfb.row_div) * p.sfb.row_pitch)) << (8 * kb);
+                        wv[j] |= static_cast<uint32_t>(__ldg(bsrc + (r >> p.sfb.row_shift) * p.sfb.row_pitch)) << (8 * kb);
                 }
             }
             *reinterpret_cast<uint4 *>(sSFBc + item * 512 + lane * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
@@ -331,7 +358,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         const ConvTap T = p.taps[kw.tap];
                         const int cx = kw.cb * 32;
                         if (leader) {
-                            if (p.rows_nfirst)
+                            if (p.sub > 1)   // slot dimension of extent 1: only slot T.aw is in range
+                                tma_load_5d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx, -T.aw,
+                                            I.q0 + T.dw, I.p0 + T.dh, I.n0);
+                            else if (p.rows_nfirst)
                                 tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx, I.n0,
                                             I.q0 + T.dw, I.p0 + T.dh);
                             else
@@ -392,7 +422,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             tc_fence_after();
             const uint32_t d_tmem = tmem + acc * p.BN;
             // cached B atoms of this column tile
-            const int item_base = KIND == kConv ? ((I.col0 / p.BN) * p.groups + p.ph_gofs[I.ph]) * p.nb_atoms : 0;
+            const int item_base = KIND == kConv ? (I.nt * p.groups + p.ph_gofs[I.ph]) * p.nb_atoms : 0;
             for (int ki = 0; ki < I.nk; ++ki, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], ph, lim, abort_flag))) {
                     ok = false;
@@ -453,25 +483,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             if (gnext >= it) continue;
             const int first = static_cast<int>(gnext - it_unit);
             // A rows of this lane: m = lane + 32 j
-            int ra_h[4], ra_w[4], ra_off[4];
+            int ra_h[4], ra_w[4], ra_off[4], ra_aw[4];
             bool ra_ok[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int m = lane + 32 * j;
                 if (KIND == kConv) {
-                    int iq, ip, in;
-                    conv_row(p, m, iq, ip, in);
+                    int aw, iq, ip, in;
+                    conv_row(p, m, aw, iq, ip, in);
                     const int q = I.q0 + iq, pr = I.p0 + ip, n = I.n0 + in;
-                    ra_ok[j] = m < p.bq * p.bp * p.bn && q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
+                    ra_ok[j] = m < p.sub * p.bq * p.bp * p.bn && p.sub * q + aw < p.ph_Qe[I.ph] &&
+                               pr < p.ph_Pe[I.ph] && n < p.Ne;
                     ra_h[j] = p.a_st_h * pr;
                     ra_w[j] = p.a_st_w * q;
-                    ra_off[j] = (n / p.sfa.row_div) * p.sfa.row_pitch;
+                    ra_aw[j] = aw;
+                    ra_off[j] = (n >> p.sfa.row_shift) * p.sfa.row_pitch;
                 } else {
                     const int k = I.m0 + m;
                     ra_ok[j] = k < p.sfa.rows;
                     ra_h[j] = 0;
                     ra_w[j] = 0;
-                    ra_off[j] = (k / p.sfa.row_div) * p.sfa.row_pitch;
+                    ra_aw[j] = 0;
+                    ra_off[j] = (k >> p.sfa.row_shift) * p.sfa.row_pitch;
                 }
             }
             // B rows of this lane: col0 + 128 at + 32 j + lane
@@ -484,30 +517,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     const int rl = 128 * at + 32 * j + lane;
                     const int r = I.col0 + rl;
                     rb_ok[at][j] = at < p.nb_atoms && rl < p.BN && r < p.sfb.rows;
-                    rb_off[at][j] = (r / p.sfb.row_div) * p.sfb.row_pitch;
+                    rb_off[at][j] = (r >> p.sfb.row_shift) * p.sfb.row_pitch;
                 }
             KbWalker kw{I.tap0, 0};
             KitWalker kt{0, 0, 0};
             if (KIND == kConv) kw.advance(KS * first, p.CB);
             else kt.init(p, I.kbase + GA * first);
             for (int ki = first; ki < I.nk; ki += nsf) {
-                uint32_t wa[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};          // [group][row j]
-                uint32_t wb[2][2][4] = {};                                          // [group][atom][row j]
-                if (KIND == kConv) {
-                    const int nkb = min(KS, I.tkb - KS * ki);
-                    KbWalker k2 = kw;
-#pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        if (4 * g >= nkb) break;
-                        if (p.sf_vec4) {
+                // one group of 4 K-blocks (one scale atom per operand) at a
+                // time: gather into registers, then store; the stage slot is
+                // awaited before the first store (the loads of the first
+                // group are already in flight by then)
+                const int ngr = KIND == kConv ? (min(KS, I.tkb - KS * ki) + 3) >> 2 : min(GA, I.nkit - GA * ki);
+                const int nkb = KIND == kConv ? min(KS, I.tkb - KS * ki) : 4 * ngr;
+                KbWalker k2 = kw;
+                KitWalker k3 = kt;
+                bool slot = false;
+                for (int g = 0; g < GA; ++g) {
+                    uint32_t wa[4] = {0u, 0u, 0u, 0u};      // [row j]
+                    uint32_t wb[2][4] = {};                 // [atom][row j]
+                    if (g < ngr) {
+                        if (KIND == kConv && SFV4) {
                             // one tap, channel blocks cb..cb+3: one 32-bit load per row
                             const ConvTap T = p.taps[k2.tap];
                             const int cb = k2.cb;
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
-                                if (ra_ok[j] && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W)
-                                    wa[g][j] = __ldg(reinterpret_cast<const uint32_t *>(
+                                if (ra_ok[j] && ra_aw[j] == T.aw && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W)
+                                    wa[j] = __ldg(reinterpret_cast<const uint32_t *>(
                                         p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
                                         ra_off[j] + cb));
                             }
@@ -518,22 +556,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
 #pragma unroll
                                     for (int j = 0; j < 4; ++j)
                                         if (rb_ok[at][j])
-                                            wb[g][at][j] = __ldg(reinterpret_cast<const uint32_t *>(bsrc + rb_off[at][j]));
+                                            wb[at][j] = __ldg(reinterpret_cast<const uint32_t *>(bsrc + rb_off[at][j]));
                             }
                             k2.advance(4, p.CB);
-                        } else {
+                        } else if (KIND == kConv) {
                             for (int kb = 0; kb < 4 && 4 * g + kb < nkb; ++kb) {
                                 const ConvTap T = p.taps[k2.tap];
                                 const int cb = k2.cb;
 #pragma unroll
                                 for (int j = 0; j < 4; ++j) {
                                     const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
-                                    if (ra_ok[j] && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W) {
-                                        const uint8_t *src = p.sfa.base +
-                                                             (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
-                                                             ra_off[j] + cb * p.sfa.kb_pitch;
-                                        wa[g][j] |= static_cast<uint32_t>(__ldg(src)) << (8 * kb);
-                                    }
+                                    if (ra_ok[j] && ra_aw[j] == T.aw && hh >= 0 && hh < p.sfa.H && ww >= 0 &&
+                                        ww < p.sfa.W)
+                                        wa[j] |= static_cast<uint32_t>(__ldg(
+                                                     p.sfa.base +
+                                                     (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
+                                                     ra_off[j] + cb * p.sfa.kb_pitch))
+                                                 << (8 * kb);
                                 }
                                 if (!skip_b) {
                                     const uint8_t *bsrc =
@@ -543,63 +582,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
 #pragma unroll
                                         for (int j = 0; j < 4; ++j)
                                             if (rb_ok[at][j])
-                                                wb[g][at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                                                wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
                                 }
                                 k2.advance(1, p.CB);
                             }
-                        }
-                    }
-                    kw.advance(KS * nsf, p.CB);
-                } else {
-                    const ConvTap T = p.taps[I.tap];
-                    const int nkit = min(GA, I.nkit - GA * ki);
-                    KitWalker k2 = kt;
-#pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        if (g >= nkit) break;
-                        for (int kb = 0; kb < 4; ++kb) {
-                            const int q = k2.qg * p.bqk + (kb >> lg_wkb);
-                            const int nb = k2.nc * p.wkb + (kb & (p.wkb - 1));
-                            if (q >= p.Q) continue;
-                            const uint8_t *asrc = p.sfa.base +
-                                                  (static_cast<int64_t>(k2.pp) * p.Q + q) * p.sfa.pix_pitch +
-                                                  nb * p.sfa.kb_pitch;
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                if (ra_ok[j]) wa[g][j] |= static_cast<uint32_t>(__ldg(asrc + ra_off[j])) << (8 * kb);
-                            const int hh = p.x_st_h * k2.pp + T.sf_dh, ww = p.x_st_w * q + T.sf_dw;
-                            if (hh < 0 || hh >= p.sfb.H || ww < 0 || ww >= p.sfb.W) continue;
-                            const uint8_t *bsrc = p.sfb.base +
-                                                  (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
-                                                  nb * p.sfb.kb_pitch;
-#pragma unroll
-                            for (int at = 0; at < 2; ++at)
+                        } else {
+                            const ConvTap T = p.taps[I.tap];
+                            for (int kb = 0; kb < 4; ++kb) {
+                                const int q = k3.qg * p.bqk + (kb >> lg_wkb);
+                                const int nb = k3.nc * p.wkb + (kb & (p.wkb - 1));
+                                if (q >= p.Q) continue;
+                                const uint8_t *asrc = p.sfa.base +
+                                                      (static_cast<int64_t>(k3.pp) * p.Q + q) * p.sfa.pix_pitch +
+                                                      nb * p.sfa.kb_pitch;
 #pragma unroll
                                 for (int j = 0; j < 4; ++j)
-                                    if (rb_ok[at][j])
-                                        wb[g][at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
-                        }
-                        k2.next(p);
-                    }
-                    for (int step = 0; step < GA * nsf; ++step) kt.next(p);
-                }
-                if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) {
-                    ok = false;
-                    break;
-                }
+                                    if (ra_ok[j]) wa[j] |= static_cast<uint32_t>(__ldg(asrc + ra_off[j])) << (8 * kb);
+                                const int hh = p.x_st_h * k3.pp + T.sf_dh, ww = p.x_st_w * q + T.sf_dw;
+                                if (hh < 0 || hh >= p.sfb.H || ww < 0 || ww >= p.sfb.W) continue;
+                                const uint8_t *bsrc = p.sfb.base +
+                                                      (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
+                                                      nb * p.sfb.kb_pitch;
 #pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    if (g >= GA) break;
+                                for (int at = 0; at < 2; ++at)
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j)
+                                        if (rb_ok[at][j])
+                                            wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                            }
+                            k3.next(p);
+                        }
+                    }
+                    if (!slot) {
+                        if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        slot = true;
+                    }
                     *reinterpret_cast<uint4 *>(sSFA + s * sfa_stage + g * 512 + lane * 16) =
-                        make_uint4(wa[g][0], wa[g][1], wa[g][2], wa[g][3]);
+                        make_uint4(wa[0], wa[1], wa[2], wa[3]);
                     if (!skip_b) {
                         *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + (g * p.nb_atoms) * 512 + lane * 16) =
-                            make_uint4(wb[g][0][0], wb[g][0][1], wb[g][0][2], wb[g][0][3]);
+                            make_uint4(wb[0][0], wb[0][1], wb[0][2], wb[0][3]);
                         if (p.nb_atoms > 1)
                             *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + (g * p.nb_atoms + 1) * 512 + lane * 16) =
-                                make_uint4(wb[g][1][0], wb[g][1][1], wb[g][1][2], wb[g][1][3]);
+                                make_uint4(wb[1][0], wb[1][1], wb[1][2], wb[1][3]);
                     }
                 }
+                if (!ok) break;
+                if (KIND == kConv) kw.advance(KS * nsf, p.CB);
+                else
+                    for (int step = 0; step < GA * nsf; ++step) kt.next(p);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[s]);
@@ -621,10 +655,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             bool row_ok;
             int64_t row_off;
             if (KIND == kConv) {
-                int iq, ip, in;
-                conv_row(p, m, iq, ip, in);
-                const int q = I.q0 + iq, pr = I.p0 + ip, n = I.n0 + in;
-                row_ok = m < p.bq * p.bp * p.bn && q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
+                int aw, iq, ip, in;
+                conv_row(p, m, aw, iq, ip, in);
+                const int q = p.sub * (I.q0 + iq) + aw, pr = I.p0 + ip, n = I.n0 + in;
+                row_ok = m < p.sub * p.bq * p.bp * p.bn && q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
                 row_off = p.ph_out_base[I.ph] + n * p.os_n + pr * p.os_p + q * p.os_q;
             } else {
                 const int k = I.m0 + m;
@@ -642,38 +676,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             tc_fence_after();
             const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16) + acc * p.BN;
             float *orow = p.out + row_off;
-            // up to 128 columns at a time: all their TMEM loads, one wait; the
-            // accumulator is released before the (slow) global stores of the
-            // last part so the MMA issuer can start the next tile on it
-            for (int c0 = 0; c0 < p.BN; c0 += 128) {
-                const int ncol = min(128, p.BN - c0);
-                uint32_t r[128];
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (32 * q < ncol) tc_ld_32x32b_x32(t_row + c0 + 32 * q, r + 32 * q);
+            // 32 columns at a time (one TMEM load, one wait); the accumulator
+            // is released after the last load, before its global stores, so
+            // the MMA issuer can start the next tile on it.  The loop body is
+            // kept small: it runs once per 32 columns of every tile, next to
+            // the code of the other roles.
+            for (int c0 = 0; c0 < p.BN; c0 += 32) {
+                uint32_t r[32];
+                tc_ld_32x32b_x32(t_row + c0, r);
                 tc_wait_ld();
-                if (c0 + 128 >= p.BN) {
+                if (c0 + 32 >= p.BN) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acc_empty[acc]);
                 }
-                if (row_ok) {
+                const int cb = I.col0 + c0;
+                const int nv = row_ok ? min(32, p.Ncols - cb) : 0;
+                float *op = orow + static_cast<int64_t>(cb) * p.os_c;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        if (32 * q < ncol) {
-                            const int cb = I.col0 + c0 + 32 * q;
-                            float *op = orow + static_cast<int64_t>(cb) * p.os_c;
-                            if (cb + 32 <= p.Ncols) {
-#pragma unroll
-                                for (int jj = 0; jj < 32; ++jj) op[jj * p.os_c] = __uint_as_float(r[32 * q + jj]);
-                            } else {
-#pragma unroll
-                                for (int jj = 0; jj < 32; ++jj)
-                                    if (cb + jj < p.Ncols) op[jj * p.os_c] = __uint_as_float(r[32 * q + jj]);
-                            }
-                        }
-                    }
-                }
+                for (int jj = 0; jj < 32; ++jj)
+                    if (jj < nv) op[jj * p.os_c] = __uint_as_float(r[jj]);
             }
             ++tcount;
         }

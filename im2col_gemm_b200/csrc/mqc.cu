@@ -86,7 +86,7 @@ int conv_Q(const mqc_conv *c) { return (c->W + 2 * c->pad_w - c->S) / c->stride_
 struct DevInfo {
     int sms = 0;
     int max_smem = 0;
-    bool gemm_attr[2] = {false, false};
+    bool gemm_attr[4] = {false, false, false, false};   // [KIND * 2 + SFV4]
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
@@ -165,12 +165,12 @@ int largest_wkb(int64_t nblocks) { return nblocks % 4 == 0 ? 4 : (nblocks % 2 ==
 // positions (q fastest) with at most 128 rows, chosen to minimise the rows
 // computed over the whole problem, with a preference for long runs along q
 // (contiguous fp32 stores in NCHW).
-void choose_rows(int Qe, int Pe, int Ne, int &bq, int &bp, int &bn) {
+void choose_rows(int Qe, int Pe, int Ne, int &bq, int &bp, int &bn, int rows = 128) {
     double best = 1e300;
     bq = bp = bn = 1;
-    for (int q = 1; q <= std::min(Qe, 128); ++q)
-        for (int n = 1; n <= std::min(Ne, 128 / q); ++n) {
-            const int pr = std::min(Pe, 128 / (q * n));
+    for (int q = 1; q <= std::min(Qe, rows); ++q)
+        for (int n = 1; n <= std::min(Ne, rows / q); ++n) {
+            const int pr = std::min(Pe, rows / (q * n));
             if (pr < 1) continue;
             const double tiles = double(ceil_div(Qe, q)) * ceil_div(Pe, pr) * ceil_div(Ne, n);
             double cost = tiles * 128.0;
@@ -193,6 +193,15 @@ int choose_bn(int ncols) {
 uint32_t mma_fmt(int f) { return f == MQC_E4M3 ? 0u : (f == MQC_E5M2 ? 1u : 5u); }
 
 const uint64_t kDefaultTimeoutNs = 4000000000ull;
+
+FastDiv make_fastdiv(int32_t d) {
+    FastDiv f;
+    f.d = static_cast<uint32_t>(std::max(1, d));
+    f.l = 0;
+    while ((1ull << f.l) < f.d) ++f.l;
+    f.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << f.l) - f.d)) / f.d + 1);
+    return f;
+}
 
 template <int KIND>
 mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
@@ -235,17 +244,33 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     const int per_stage = P.kbs == 8 ? ps8 : ps4;
     if (S < 3) return fail(MQC_ERR_UNSUPPORTED, "tile does not fit in shared memory");
     P.stages = S;
+    if (P.sub < 1) P.sub = 1;
+    P.fd_NT = make_fastdiv(P.NT);
+    P.fd_nph = make_fastdiv(P.nph);
+    P.fd_TQ = make_fastdiv(P.TQ);
+    P.fd_TP = make_fastdiv(P.TP);
+    P.fd_sub = make_fastdiv(P.sub);
+    P.fd_bq = make_fastdiv(P.bq);
+    P.fd_bp = make_fastdiv(P.bp);
+    P.fd_bn = make_fastdiv(P.bn);
+    P.fd_MT = make_fastdiv(P.MT);
+    P.fd_ntaps = make_fastdiv(P.ntaps);
+    P.fd_splits = make_fastdiv(P.splits);
+    if (KIND == kWgrad && int64_t(P.kiters_total) * (P.splits + 1) >= (1ll << 31))
+        return fail(MQC_ERR_UNSUPPORTED, "weight gradient: reduction too long");
     P.nacc = (P.BN <= 128) ? 2 : 1;
     P.timeout_ns = kDefaultTimeoutNs;
     const int smem = fixed + S * per_stage;
-    if (!d.gemm_attr[KIND]) {
-        cudaError_t e = cudaFuncSetAttribute(conv_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             d.max_smem);
+    const bool v4 = KIND == kConv && P.sf_vec4;
+    auto kernel = v4 ? conv_gemm_kernel<KIND, true> : conv_gemm_kernel<KIND, false>;
+    const int ai = KIND * 2 + (v4 ? 1 : 0);
+    if (!d.gemm_attr[ai]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.max_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-        const_cast<DevInfo &>(d).gemm_attr[KIND] = true;
+        const_cast<DevInfo &>(d).gemm_attr[ai] = true;
     }
     const int grid = std::max(1, std::min(P.num_units, d.sms));
-    conv_gemm_kernel<KIND><<<grid, kGemmThreads, smem, stream>>>(P);
+    kernel<<<grid, kGemmThreads, smem, stream>>>(P);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "conv_gemm_kernel launch");
     return MQC_OK;
@@ -555,7 +580,7 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     const bool sqx = xf->block == MQC_BLOCK_SQ32, sqw = wf->block == MQC_BLOCK_SQ32;
     G.sfa.base = xs;
     G.sfa.pix_pitch = (sqx ? nb32(N) : N) * nb32(Cp);
-    G.sfa.row_div = sqx ? 32 : 1;
+    G.sfa.row_shift = sqx ? 5 : 0;
     G.sfa.row_pitch = static_cast<int32_t>(nb32(Cp));
     G.sfa.kb_pitch = 1;
     G.sfa.rows = N;
@@ -563,7 +588,7 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     G.sfa.W = W;
     G.sfb.base = ws;
     G.sfb.tap_pitch = (sqw ? nb32(K) : K) * nb32(Cp);
-    G.sfb.row_div = sqw ? 32 : 1;
+    G.sfb.row_shift = sqw ? 5 : 0;
     G.sfb.row_pitch = static_cast<int32_t>(nb32(Cp));
     G.sfb.kb_pitch = 1;
     G.sfb.rows = K;
@@ -598,28 +623,25 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     // output stride phases (ah, aw) with at least one row; the first one has
     // the largest extents and sets the tiling shared by a launch
-    if (sh * sw > 64) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_data: stride product above 64");
-    int phases[64][2];
-    int nphase = 0;
-    for (int ah = 0; ah < sh; ++ah)
-        for (int aw = 0; aw < sw; ++aw)
-            if (H - ah > 0 && W - aw > 0) {
-                phases[nphase][0] = ah;
-                phases[nphase][1] = aw;
-                ++nphase;
-            }
-    const int Pe0 = static_cast<int>(ceil_div(H, sh)), Qe0 = static_cast<int>(ceil_div(W, sw));
-    for (int first = 0; first < nphase; first += kMaxPhases) {
-        const int nph = std::min(kMaxPhases, nphase - first);
+    if (sh > 64 || sw > 64) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_data: stride above 64");
+    // Output rows h = sh * p' + ah split into sh phases (their tap rows r
+    // differ).  Along the width the sw phases share a tile: its rows
+    // interleave them (sub = sw), so every output row is written whole.
+    const int sub = sw;
+    const int Qw = static_cast<int>(ceil_div(W, sw));     // q' extent (output column w = sw * q' + aw)
+    const int Pe0 = static_cast<int>(ceil_div(H, sh));
+    for (int first = 0; first < sh && first < H; first += kMaxPhases) {
+        const int nph = std::min({kMaxPhases, sh - first, H - first});
         GemmParams G;
         memset(&G, 0, sizeof G);
         G.CB = static_cast<int32_t>(nb32(Kp));
         G.wkb = largest_wkb(G.CB);
-        choose_rows(Qe0, Pe0, N, G.bq, G.bp, G.bn);
+        G.sub = sub;
+        choose_rows(Qw, Pe0, N, G.bq, G.bp, G.bn, 128 / sub);
         G.BN = choose_bn(C);
         G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
         G.Ne = N;
-        G.TQ = static_cast<int32_t>(ceil_div(Qe0, G.bq));
+        G.TQ = static_cast<int32_t>(ceil_div(Qw, G.bq));
         G.TP = static_cast<int32_t>(ceil_div(Pe0, G.bp));
         G.TN = static_cast<int32_t>(ceil_div(N, G.bn));
         G.NT = static_cast<int32_t>(ceil_div(C, G.BN));
@@ -628,18 +650,29 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
         G.a_st_w = 1;
         G.idesc = make_idesc_mx(mma_fmt(gf->fmt), mma_fmt(wf->fmt), 128, G.BN);
         st = MQC_ERR_CUDA;
-        for (int attempt = 0; attempt < 2 && st != MQC_OK; ++attempt) {
-            G.rows_nfirst = attempt;
-            if (!G.rows_nfirst) {
-                const uint64_t dims[4] = {uint64_t(Kp), uint64_t(Q), uint64_t(P), uint64_t(N)};
-                const uint64_t strd[3] = {uint64_t(N) * Kp, uint64_t(Q) * N * Kp, uint64_t(Kp)};
-                const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bq), uint32_t(G.bp), uint32_t(G.bn)};
-                st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
-            } else {
-                const uint64_t dims[4] = {uint64_t(Kp), uint64_t(N), uint64_t(Q), uint64_t(P)};
-                const uint64_t strd[3] = {uint64_t(Kp), uint64_t(N) * Kp, uint64_t(Q) * N * Kp};
-                const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bn), uint32_t(G.bq), uint32_t(G.bp)};
-                st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
+        if (sub > 1) {
+            // (C, slot, q, p, n): the slot dimension has extent 1 and a box of
+            // sub, so a tap's box fills only the rows of its own slot
+            G.rows_nfirst = 0;
+            const uint64_t dims[5] = {uint64_t(Kp), 1u, uint64_t(Q), uint64_t(P), uint64_t(N)};
+            const uint64_t strd[4] = {uint64_t(Kp), uint64_t(N) * Kp, uint64_t(Q) * N * Kp, uint64_t(Kp)};
+            const uint32_t box[5] = {uint32_t(32 * G.wkb), uint32_t(sub), uint32_t(G.bq), uint32_t(G.bp),
+                                     uint32_t(G.bn)};
+            st = encode_codes_map(&G.amap[0], gq, 5, dims, strd, box, G.wkb);
+        } else {
+            for (int attempt = 0; attempt < 2 && st != MQC_OK; ++attempt) {
+                G.rows_nfirst = attempt;
+                if (!G.rows_nfirst) {
+                    const uint64_t dims[4] = {uint64_t(Kp), uint64_t(Q), uint64_t(P), uint64_t(N)};
+                    const uint64_t strd[3] = {uint64_t(N) * Kp, uint64_t(Q) * N * Kp, uint64_t(Kp)};
+                    const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bq), uint32_t(G.bp), uint32_t(G.bn)};
+                    st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
+                } else {
+                    const uint64_t dims[4] = {uint64_t(Kp), uint64_t(N), uint64_t(Q), uint64_t(P)};
+                    const uint64_t strd[3] = {uint64_t(Kp), uint64_t(N) * Kp, uint64_t(Q) * N * Kp};
+                    const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bn), uint32_t(G.bq), uint32_t(G.bp)};
+                    st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
+                }
             }
         }
         if (st != MQC_OK) return st;
@@ -649,37 +682,39 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
             const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(G.BN), 1u};
             if ((st = encode_codes_map(&G.bmap[0], wq, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
         }
-        // taps of each phase: kernel offsets r with (ah + pad - r) divisible by the stride
+        // taps of phase ah: kernel rows r with (ah + pad - r) divisible by sh,
+        // every kernel column s; tap (r, s) feeds slot aw = (s - pad) mod sw
         G.ntaps = 0;
         G.nph = nph;
         for (int k = 0; k < nph; ++k) {
-            const int ah = phases[first + k][0], aw = phases[first + k][1];
+            const int ah = first + k;
             G.ph_tap0[k] = G.ntaps;
             for (int r = 0; r < R; ++r) {
                 if (((ah + c->pad_h - r) % sh + sh) % sh != 0) continue;
                 const int dr = (ah + c->pad_h - r) / sh;
                 for (int s = 0; s < S; ++s) {
-                    if (((aw + c->pad_w - s) % sw + sw) % sw != 0) continue;
+                    const int aw = ((s - c->pad_w) % sw + sw) % sw;
                     const int ds = (aw + c->pad_w - s) / sw;
                     ConvTap &T = G.taps[G.ntaps++];
                     T.dh = T.sf_dh = static_cast<int16_t>(dr);
                     T.dw = T.sf_dw = static_cast<int16_t>(ds);
                     T.map = 0;
+                    T.aw = static_cast<int16_t>(aw);
                     T.btap = static_cast<int16_t>(r * S + s);
                 }
             }
             G.ph_tkb[k] = (G.ntaps - G.ph_tap0[k]) * G.CB;
             G.ph_Pe[k] = static_cast<int32_t>(ceil_div(H - ah, sh));
-            G.ph_Qe[k] = static_cast<int32_t>(ceil_div(W - aw, sw));
-            G.ph_out_base[k] = int64_t(ah) * W + aw;
+            G.ph_Qe[k] = W;                      // limit of the output column sw * q' + aw
+            G.ph_out_base[k] = int64_t(ah) * W;
         }
         G.n_amaps = 1;
         G.n_bmaps = 1;
-        G.a_box_bytes = 32 * G.wkb * G.bq * G.bp * G.bn;
+        G.a_box_bytes = 32 * G.wkb * sub * G.bq * G.bp * G.bn;
         G.b_box_bytes = 32 * G.wkb * G.BN;
         G.sfa.base = gs;
         G.sfa.pix_pitch = (sqg ? nb32(N) : N) * nb32(Kp);
-        G.sfa.row_div = sqg ? 32 : 1;
+        G.sfa.row_shift = sqg ? 5 : 0;
         G.sfa.row_pitch = static_cast<int32_t>(nb32(Kp));
         G.sfa.kb_pitch = 1;
         G.sfa.rows = N;
@@ -687,7 +722,7 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
         G.sfa.W = Q;
         G.sfb.base = ws;
         G.sfb.tap_pitch = nb32(Kp) * (sqw ? nb32(C) : C);
-        G.sfb.row_div = sqw ? 32 : 1;
+        G.sfb.row_shift = sqw ? 5 : 0;
         G.sfb.row_pitch = 1;
         G.sfb.kb_pitch = static_cast<int32_t>(sqw ? nb32(C) : C);
         G.sfb.rows = C;
@@ -695,7 +730,7 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
                     (reinterpret_cast<uintptr_t>(gs) & 3u) == 0;
         G.sfb_vec4 = false;   // the weights' scales run along K with a stride of C per block
         G.out = gx;
-        G.os_q = sw;
+        G.os_q = 1;
         G.os_p = int64_t(sh) * W;
         G.os_n = int64_t(C) * H * W;
         G.os_c = int64_t(H) * W;
@@ -824,7 +859,7 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     G.sfa.base = gs;
     G.sfa.pix_pitch = nb32(Np) * (sqg ? nb32(K) : K);
     G.sfa.kb_pitch = static_cast<int32_t>(sqg ? nb32(K) : K);
-    G.sfa.row_div = sqg ? 32 : 1;
+    G.sfa.row_shift = sqg ? 5 : 0;
     G.sfa.row_pitch = 1;
     G.sfa.rows = K;
     G.sfa.H = P;
@@ -832,7 +867,7 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     G.sfb.base = xs;
     G.sfb.pix_pitch = nb32(Np) * (sqx ? nb32(C) : C);
     G.sfb.kb_pitch = static_cast<int32_t>(sqx ? nb32(C) : C);
-    G.sfb.row_div = sqx ? 32 : 1;
+    G.sfb.row_shift = sqx ? 5 : 0;
     G.sfb.row_pitch = 1;
     G.sfb.rows = C;
     G.sfb.H = H;

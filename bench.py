@@ -318,6 +318,44 @@ def workload_by_name(name: str) -> synth.Workload:
     return synth.WORKLOADS[int(name)]
 
 
+CALLS = ("quantize_x", "quantize_w", "quantize_g", "fwd", "dgrad", "wgrad")
+
+
+def capture_graph(torch, fn):
+    """One CUDA graph of `fn` (C-ABI calls on the capturing stream): replaying
+    it runs the same kernels without the host's per-call argument marshalling
+    and tensor-map encoding between launches."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        fn()
+    return g
+
+
+def graph_call_times(mqc, torch, lb, workspace, reps, names=CALLS):
+    """Device time (ms) of each named call of one layer: the call captured as
+    a CUDA graph and replayed `reps` times, each replay between a pair of
+    events and preceded by an L2 flush (a 256 MiB write)."""
+    cur = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    out = {}
+    for name in names:
+        g = capture_graph(torch, lambda: run_layer(mqc, lb, workspace, cur(), only=(name,)))
+        g.replay()
+        ev = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        out[name] = [a.elapsed_time(b) for a, b in ev]
+        del g
+    mqc.check(mqc.get_device_status())
+    return out
+
+
 def sweep(mqc, torch, wl, args):
     """Per-call times of every layer of a workload, with roofline fractions."""
     pk = peaks()
@@ -329,14 +367,7 @@ def sweep(mqc, torch, wl, args):
         stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
         for _ in range(2):
             run_layer(mqc, lb, workspace, stream)
-        events = []
-        for _ in range(args.reps):
-            run_layer(mqc, lb, workspace, stream, events)
-        torch.cuda.synchronize()
-        mqc.check(mqc.get_device_status())
-        per = {}
-        for name, e0, e1 in events:
-            per.setdefault(name, []).append(e0.elapsed_time(e1))
+        per = graph_call_times(mqc, torch, lb, workspace, max(3, args.reps))
         for name, v in per.items():
             ms = statistics.median(v)
             if name.startswith("quantize"):
@@ -407,10 +438,14 @@ def main(argv=None):
             for t in gws:
                 dist.all_reduce(t)
 
+    def cur_stream():
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
     def step(events=None):
         for lb in layers:
-            run_layer(mqc, lb, workspace, stream, events)
+            run_layer(mqc, lb, workspace, cur_stream(), events)
         allreduce_gw()
+
 
     # clocks are sampled from the start of the warm-up to the end of the timed
     # region (nvidia-smi needs a few hundred ms to produce its first sample)
@@ -421,15 +456,23 @@ def main(argv=None):
         step()
     torch.cuda.synchronize()
     mqc.check(mqc.get_device_status())
+    # the step's kernels as one CUDA graph (the weight-gradient all-reduce of
+    # a multi-GPU run stays outside it)
+    step_graph = capture_graph(torch, lambda: [run_layer(mqc, lb, workspace, cur_stream()) for lb in layers])
+    for _ in range(args.warmup):
+        step_graph.replay()
+        allreduce_gw()
+    torch.cuda.synchronize()
+    mqc.check(mqc.get_device_status())
 
     # ---- timed region: inputs resident in HBM
-    events = []
     barrier()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record()
     for _ in range(args.steps):
-        step(events)
+        step_graph.replay()
+        allreduce_gw()
     t1.record()
     torch.cuda.synchronize()
     barrier()
@@ -439,12 +482,11 @@ def main(argv=None):
     mqc.check(mqc.get_device_status())
     value = world * step_flops / (ms * 1e-3) / 1e12
 
-    # per-call durations (mean over the timed steps)
+    # per-call durations: each call as its own graph (cold L2, no host gaps)
     per = {}
-    nper = len(events) // args.steps
-    for k, (name, e0, e1) in enumerate(events):
-        key = (k % nper) // 6, name
-        per.setdefault(key, []).append(e0.elapsed_time(e1))
+    for li, lb in enumerate(layers):
+        for name, v in graph_call_times(mqc, torch, lb, workspace, max(3, min(args.steps, 10))).items():
+            per[(li, name)] = v
     calls = []
     for (li, name), v in per.items():
         lb = layers[li]
@@ -490,7 +532,8 @@ def main(argv=None):
             for lb in layers:
                 for dst, src in zip((lb.x, lb.w, lb.g), lb.host_in):
                     dst.copy_(src, non_blocking=True)
-            step()
+            step_graph.replay()
+            allreduce_gw()
             for lb in layers:
                 for dst, src in zip(lb.host_out, (lb.y, lb.gx, lb.gw)):
                     dst.copy_(src, non_blocking=True)

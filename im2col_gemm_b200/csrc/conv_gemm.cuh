@@ -86,6 +86,11 @@ struct alignas(64) GemmParams {
     uint64_t timeout_ns;
     int32_t num_units;
     int32_t a_box_bytes, b_box_bytes;
+    // rows between consecutive K sub-tiles (of wkb K-blocks) inside a group
+    // of 4 K-blocks in shared memory: 128 / BN when each sub-tile is its own
+    // box (CONV), the box rows when one box spans the group (WGRAD, whose
+    // boxes hold only the rows that exist)
+    int32_t a_slab, b_slab;
     // CONV kind
     int32_t rows_nfirst;         // A map dims (C, N, W, H) instead of (C, W, H, N)
     // rows interleaved along the output width: tile row m = aw + sub * (q +
@@ -116,8 +121,12 @@ struct alignas(64) GemmParams {
     int32_t Ncols;               // GEMM columns (output channels)
     // WGRAD kind: K is walked in "kits" of 4 K-blocks (one TMA box per operand)
     int32_t MT, Mrows, splits, kiters_total, QG, NC, bqk, P, Q;
+    // WGRAD tap groups: the GEMM columns of a unit are (tap of the group,
+    // input channel), cpad rows per tap (a multiple of 8), so one MMA per
+    // K-block covers ntg taps.  ntg = 1: the columns are channels of one tap.
+    int32_t ntg, ngroups, cpad;
     // the divisions of the unit and row decoding, by launch constants
-    FastDiv fd_NT, fd_nph, fd_TQ, fd_TP, fd_sub, fd_bq, fd_bp, fd_bn, fd_MT, fd_ntaps, fd_splits;
+    FastDiv fd_NT, fd_nph, fd_TQ, fd_TP, fd_sub, fd_bq, fd_bp, fd_bn, fd_MT, fd_ngroups, fd_splits, fd_cpad;
     int32_t x_st_h, x_st_w;      // stride of X pixels per output pixel
     // output
     float *out;
@@ -132,7 +141,7 @@ struct UnitInfo {
     int q0, p0, n0;         // CONV: tile origin
     int m0;                 // WGRAD: first output channel row
     int col0;               // first GEMM column
-    int tap;                // WGRAD: tap of this unit
+    int tap, tig;           // WGRAD: first tap of the unit's group, taps in the group
     int split;              // WGRAD: split index
 };
 
@@ -162,8 +171,9 @@ __device__ __forceinline__ UnitInfo decode_unit(const GemmParams &p, int u) {
         const int mt = u - static_cast<int>(r1) * p.MT;
         const uint32_t r2 = p.fd_NT.div(r1);
         const int nt = static_cast<int>(r1 - r2 * p.NT);
-        const uint32_t sp = p.fd_ntaps.div(r2);
-        I.tap = static_cast<int>(r2 - sp * p.ntaps);
+        const uint32_t sp = p.fd_ngroups.div(r2);
+        I.tap = static_cast<int>(r2 - sp * p.ngroups) * p.ntg;
+        I.tig = min(p.ntg, p.ntaps - I.tap);
         I.split = static_cast<int>(sp);
         I.nt = nt;
         I.m0 = mt * 128;
@@ -372,16 +382,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         kw.advance(p.wkb, p.CB);
                     }
                 } else {
-                    const ConvTap T = p.taps[I.tap];
                     const int nkit = min(GA, I.nkit - GA * ki);
+                    // B: one box over the kit's pixels (one tap), or one box
+                    // per (tap, pixel) of a tap group
+                    const int bmul = p.ntg > 1 ? I.tig * p.bqk : 1;
                     if (leader)
-                        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nkit * (p.a_box_bytes + p.b_box_bytes)));
+                        mbar_arrive_expect_tx(&full[s],
+                                              static_cast<uint32_t>(nkit * (p.a_box_bytes + bmul * p.b_box_bytes)));
                     for (int g = 0; g < nkit; ++g) {
                         const int nx = kt.nc * row_bytes;
                         if (leader) {
                             tma_load_4d(a_dst + g * 128 * 128, &p.amap[0], &full[s], nx, I.m0, kt.qg * p.bqk, kt.pp);
-                            tma_load_4d(b_dst + g * p.BN * 128, &p.bmap[T.map], &full[s], nx, I.col0,
-                                        kt.qg * p.bqk + T.dw, kt.pp + T.dh);
+                            if (p.ntg == 1) {
+                                const ConvTap T = p.taps[I.tap];
+                                tma_load_4d(b_dst + g * p.BN * 128, &p.bmap[T.map], &full[s], nx, I.col0,
+                                            kt.qg * p.bqk + T.dw, kt.pp + T.dh);
+                            } else {
+                                for (int t = 0; t < I.tig; ++t) {
+                                    const ConvTap T = p.taps[I.tap + t];
+                                    for (int jq = 0; jq < p.bqk; ++jq)
+                                        tma_load_4d(b_dst + g * p.BN * 128 + (jq * p.BN + t * p.cpad) * row_bytes,
+                                                    &p.bmap[T.map], &full[s], nx, 0, kt.qg * p.bqk + jq + T.dw,
+                                                    kt.pp + T.dh);
+                                }
+                            }
                         }
                         kt.next(p);
                     }
@@ -412,7 +436,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         const uint64_t sfa_desc0 = make_smem_desc(smem_u32(sSFA), 0, 128, kSwizzleNone);
         const uint64_t sfb_desc0 = make_smem_desc(smem_u32(sSFB), 0, 128, kSwizzleNone);
         const uint64_t sfbc_desc0 = make_smem_desc(smem_u32(sSFBc), 0, 128, kSwizzleNone);
-        const uint32_t a_sub = (128 * row_bytes) >> 4, b_sub = (p.BN * row_bytes) >> 4;
+        const uint32_t a_sub = (p.a_slab * row_bytes) >> 4, b_sub = (p.b_slab * row_bytes) >> 4;
+        const uint32_t a_grp = (128 * 128) >> 4, b_grp = (p.BN * 128) >> 4;   // one group of 4 K-blocks
         for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
             if (I.nk == 0) continue;
@@ -446,10 +471,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         }
                     }
                     for (int kb = 0; kb < nkb; ++kb) {
-                        const uint32_t j = static_cast<uint32_t>(kb >> lg_wkb);
-                        const uint32_t within = static_cast<uint32_t>(kb & (p.wkb - 1));
                         const uint32_t g = static_cast<uint32_t>(kb >> 2), k4 = static_cast<uint32_t>(kb & 3);
-                        tc_mma_mxf8f6f4(d_tmem, a_s + j * a_sub + within * 2, b_s + j * b_sub + within * 2,
+                        const uint32_t j = k4 >> lg_wkb;                       // sub-tile within the group
+                        const uint32_t within = k4 & static_cast<uint32_t>(p.wkb - 1);
+                        tc_mma_mxf8f6f4(d_tmem, a_s + g * a_grp + j * a_sub + within * 2, b_s + g * b_grp + j * b_sub + within * 2,
                                         p.idesc | (k4 << 29) | (k4 << 4), (sf_t + 4 * g) | (k4 << 30),
                                         (sfb_t + 4 * g * p.nb_atoms) | (k4 << 30), (ki > 0 || kb > 0) ? 1u : 0u);
                     }
@@ -508,16 +533,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 }
             }
             // B rows of this lane: col0 + 128 at + 32 j + lane
-            int rb_off[2][4];
+            // (WGRAD: with tap groups a B row is (tap, channel) and carries
+            // its tap's pixel offset; otherwise every row has the unit's tap)
+            int rb_off[2][4], rb_dh[2][4], rb_dw[2][4];
             bool rb_ok[2][4];
 #pragma unroll
             for (int at = 0; at < 2; ++at)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int rl = 128 * at + 32 * j + lane;
-                    const int r = I.col0 + rl;
-                    rb_ok[at][j] = at < p.nb_atoms && rl < p.BN && r < p.sfb.rows;
+                    int r = I.col0 + rl, t = 0;
+                    if (KIND == kWgrad && p.ntg > 1) {
+                        t = static_cast<int>(p.fd_cpad.div(rl));
+                        r = rl - t * p.cpad;
+                    }
+                    rb_ok[at][j] = at < p.nb_atoms && rl < p.BN && r < p.sfb.rows && (KIND == kConv || t < I.tig);
                     rb_off[at][j] = (r >> p.sfb.row_shift) * p.sfb.row_pitch;
+                    if (KIND == kWgrad) {
+                        const ConvTap T = p.taps[I.tap + (rb_ok[at][j] ? t : 0)];
+                        rb_dh[at][j] = T.sf_dh;
+                        rb_dw[at][j] = T.sf_dw;
+                    } else {
+                        rb_dh[at][j] = rb_dw[at][j] = 0;
+                    }
                 }
             KbWalker kw{I.tap0, 0};
             KitWalker kt{0, 0, 0};
@@ -587,7 +625,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                                 k2.advance(1, p.CB);
                             }
                         } else {
-                            const ConvTap T = p.taps[I.tap];
                             for (int kb = 0; kb < 4; ++kb) {
                                 const int q = k3.qg * p.bqk + (kb >> lg_wkb);
                                 const int nb = k3.nc * p.wkb + (kb & (p.wkb - 1));
@@ -598,17 +635,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
 #pragma unroll
                                 for (int j = 0; j < 4; ++j)
                                     if (ra_ok[j]) wa[j] |= static_cast<uint32_t>(__ldg(asrc + ra_off[j])) << (8 * kb);
-                                const int hh = p.x_st_h * k3.pp + T.sf_dh, ww = p.x_st_w * q + T.sf_dw;
-                                if (hh < 0 || hh >= p.sfb.H || ww < 0 || ww >= p.sfb.W) continue;
-                                const uint8_t *bsrc = p.sfb.base +
-                                                      (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
-                                                      nb * p.sfb.kb_pitch;
+                                const int h0 = p.x_st_h * k3.pp, w0 = p.x_st_w * q;
+                                if (p.ntg == 1) {
+                                    // every row has the unit's tap: one pixel per K-block
+                                    const int hh = h0 + rb_dh[0][0], ww = w0 + rb_dw[0][0];
+                                    if (hh < 0 || hh >= p.sfb.H || ww < 0 || ww >= p.sfb.W) continue;
+                                    const uint8_t *bsrc = p.sfb.base +
+                                                          (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
+                                                          nb * p.sfb.kb_pitch;
+#pragma unroll
+                                    for (int at = 0; at < 2; ++at)
+#pragma unroll
+                                        for (int j = 0; j < 4; ++j)
+                                            if (rb_ok[at][j])
+                                                wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                                    continue;
+                                }
 #pragma unroll
                                 for (int at = 0; at < 2; ++at)
 #pragma unroll
-                                    for (int j = 0; j < 4; ++j)
-                                        if (rb_ok[at][j])
-                                            wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                                    for (int j = 0; j < 4; ++j) {
+                                        const int hh = h0 + rb_dh[at][j], ww = w0 + rb_dw[at][j];
+                                        if (rb_ok[at][j] && hh >= 0 && hh < p.sfb.H && ww >= 0 && ww < p.sfb.W)
+                                            wb[at][j] |= static_cast<uint32_t>(__ldg(
+                                                             p.sfb.base +
+                                                             (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
+                                                             nb * p.sfb.kb_pitch + rb_off[at][j]))
+                                                         << (8 * kb);
+                                    }
                             }
                             k3.next(p);
                         }
@@ -663,11 +717,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             } else {
                 const int k = I.m0 + m;
                 row_ok = k < p.Mrows;
-                row_off = p.out_base + I.split * p.split_pitch + k * p.os_m + p.taps[I.tap].btap;
+                row_off = p.out_base + I.split * p.split_pitch + k * p.os_m + (p.ntg == 1 ? p.taps[I.tap].btap : 0);
             }
+            const bool tap_cols = KIND == kWgrad && p.ntg > 1;   // columns are (tap, channel)
             if (I.nk == 0) {
                 if (row_ok)
-                    for (int c = I.col0; c < min(I.col0 + p.BN, p.Ncols); ++c) p.out[row_off + c * p.os_c] = 0.0f;
+                    for (int n = 0; n < p.BN; ++n) {
+                        if (tap_cols) {
+                            const int t = static_cast<int>(p.fd_cpad.div(n)), c = n - t * p.cpad;
+                            if (t < I.tig && c < p.Ncols) p.out[row_off + c * p.os_c + p.taps[I.tap + t].btap] = 0.0f;
+                        } else if (I.col0 + n < p.Ncols) {
+                            p.out[row_off + (I.col0 + n) * p.os_c] = 0.0f;
+                        }
+                    }
                 continue;
             }
             const uint32_t acc = tcount & 1u & static_cast<uint32_t>(p.nacc - 1);
@@ -689,6 +751,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                }
+                if (tap_cols) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int n = c0 + jj;
+                        const int t = static_cast<int>(p.fd_cpad.div(n)), c = n - t * p.cpad;
+                        if (row_ok && n < p.BN && t < I.tig && c < p.Ncols)
+                            orow[c * p.os_c + p.taps[I.tap + t].btap] = __uint_as_float(r[jj]);
+                    }
+                    continue;
                 }
                 const int cb = I.col0 + c0;
                 const int nv = row_ok ? min(32, p.Ncols - cb) : 0;

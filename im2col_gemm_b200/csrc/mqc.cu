@@ -87,6 +87,7 @@ struct DevInfo {
     int sms = 0;
     int max_smem = 0;
     bool gemm_attr[4] = {false, false, false, false};   // [KIND * 2 + SFV4]
+    bool quant_attr[2] = {false, false};                  // staged quantizer, [fmt]
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
@@ -186,9 +187,14 @@ void choose_rows(int Qe, int Pe, int Ne, int &bq, int &bp, int &bn, int rows = 1
 }
 
 int choose_bn(int ncols) {
-    if (ncols <= 128) return static_cast<int>(round_up(ncols, 32));
+    if (ncols <= 128) return static_cast<int>(round_up(ncols, 16));
     return 128;
 }
+
+// Rows of a box that holds a whole operand tile dimension of `rows` (when it
+// fits one tile): rows beyond the operand are not copied (the MMA reads stale
+// shared memory there; those accumulator rows or columns are never stored).
+int box_rows(int rows, int tile) { return rows < tile ? static_cast<int>(round_up(rows, 8)) : tile; }
 
 uint32_t mma_fmt(int f) { return f == MQC_E4M3 ? 0u : (f == MQC_E5M2 ? 1u : 5u); }
 
@@ -254,7 +260,8 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     P.fd_bp = make_fastdiv(P.bp);
     P.fd_bn = make_fastdiv(P.bn);
     P.fd_MT = make_fastdiv(P.MT);
-    P.fd_ntaps = make_fastdiv(P.ntaps);
+    P.fd_ngroups = make_fastdiv(P.ngroups);
+    P.fd_cpad = make_fastdiv(P.cpad);
     P.fd_splits = make_fastdiv(P.splits);
     if (KIND == kWgrad && int64_t(P.kiters_total) * (P.splits + 1) >= (1ll << 31))
         return fail(MQC_ERR_UNSUPPORTED, "weight gradient: reduction too long");
@@ -395,6 +402,34 @@ mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, 
     const int blk = mx->block == MQC_BLOCK_SQ32 ? kSquare : (along_i ? kAlongI : kAlongO);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool dual = codes_alt != nullptr;
+    // staged kernel: FP8, positions contiguous (element stride 1 along W,
+    // W along H), every plane 16-byte aligned
+    if (!fp4 && d->s3 == 1 && d->s2 == d->d3 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && d->s0 % 4 == 0 &&
+        d->s1 % 4 == 0) {
+        StagedParams sp{};
+        sp.q = p;
+        sp.IT = p.I1 <= 16 ? 16 : 32;
+        sp.OT = (dual ? std::max(p.O, p.O2) : p.O) <= 16 ? 16 : 32;
+        sp.PT = kStagedTileBytes / (4 * sp.OT * sp.IT);
+        sp.nPT = static_cast<int32_t>(ceil_div(p.npix, sp.PT));
+        sp.nOT = static_cast<int32_t>(ceil_div(dual ? std::max(p.O, p.O2) : p.O, sp.OT));
+        sp.nIT = static_cast<int32_t>(ceil_div(p.I1, sp.IT));
+        sp.blk = blk;
+        sp.map_a = map_a ? 1 : 0;
+        const int64_t ntiles = int64_t(sp.nPT) * sp.nOT * sp.nIT;
+        if (ntiles > (int64_t(1) << 31) - 1) return fail(MQC_ERR_INVALID, "quantize: tensor too large");
+        const int smem = kStagedTileBytes + 32 * 64 * 4 + 64 * 4;
+        auto kernel = p.fmt == MQC_E4M3 ? mx_quantize_staged_kernel<0> : mx_quantize_staged_kernel<1>;
+        if (!dv->quant_attr[p.fmt]) {
+            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+            dv->quant_attr[p.fmt] = true;
+        }
+        kernel<<<static_cast<unsigned>(ntiles), 256, smem, s>>>(sp);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "mx_quantize_staged_kernel launch");
+        return MQC_OK;
+    }
     if (map_a) launch_quantize_blk<true>(p, blk, dual, it, static_cast<unsigned>(tiles), s);
     else launch_quantize_blk<false>(p, blk, dual, it, static_cast<unsigned>(tiles), s);
     cudaError_t e = cudaGetLastError();
@@ -542,7 +577,7 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     {
         const uint64_t dims[3] = {uint64_t(Cp), uint64_t(K), uint64_t(R) * S};
         const uint64_t strd[2] = {uint64_t(Cp), uint64_t(K) * Cp};
-        const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(G.BN), 1u};
+        const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(box_rows(K, G.BN)), 1u};
         if ((st = encode_codes_map(&G.bmap[0], wq, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
     }
     G.ntaps = 0;
@@ -576,7 +611,9 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     G.n_amaps = sh * sw;
     G.n_bmaps = 1;
     G.a_box_bytes = 32 * G.wkb * G.bq * G.bp * G.bn;
-    G.b_box_bytes = 32 * G.wkb * G.BN;
+    G.b_box_bytes = 32 * G.wkb * box_rows(K, G.BN);
+    G.a_slab = 128;
+    G.b_slab = G.BN;
     const bool sqx = xf->block == MQC_BLOCK_SQ32, sqw = wf->block == MQC_BLOCK_SQ32;
     G.sfa.base = xs;
     G.sfa.pix_pitch = (sqx ? nb32(N) : N) * nb32(Cp);
@@ -679,7 +716,7 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
         {
             const uint64_t dims[3] = {uint64_t(Kp), uint64_t(C), uint64_t(R) * S};
             const uint64_t strd[2] = {uint64_t(Kp), uint64_t(C) * Kp};
-            const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(G.BN), 1u};
+            const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(box_rows(C, G.BN)), 1u};
             if ((st = encode_codes_map(&G.bmap[0], wq, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
         }
         // taps of phase ah: kernel rows r with (ah + pad - r) divisible by sh,
@@ -711,7 +748,9 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
         G.n_amaps = 1;
         G.n_bmaps = 1;
         G.a_box_bytes = 32 * G.wkb * sub * G.bq * G.bp * G.bn;
-        G.b_box_bytes = 32 * G.wkb * G.BN;
+        G.b_box_bytes = 32 * G.wkb * box_rows(C, G.BN);
+        G.a_slab = 128;
+        G.b_slab = G.BN;
         G.sfa.base = gs;
         G.sfa.pix_pitch = (sqg ? nb32(N) : N) * nb32(Kp);
         G.sfa.row_shift = sqg ? 5 : 0;
@@ -741,18 +780,40 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
 }
 
 // ------------------------------------------------------------------ weight gradient
-static void wgrad_plan(const mqc_conv *c, const DevInfo &d, int &BN, int &splits, int64_t &kiters) {
+// Weight-gradient tiling.  With at most 128 input channels the kernel taps
+// join the GEMM columns: a unit covers ntg taps x cpad channel rows (cpad =
+// C rounded up to 8, at most 256 columns), so one MMA per K-block serves all
+// of them instead of one narrow MMA per tap.
+struct WgradPlan {
+    int BN, splits, ntg, ngroups, cpad;
+    int64_t kiters;
+};
+
+static WgradPlan wgrad_plan(const mqc_conv *c, const DevInfo &d) {
+    WgradPlan w{};
     const int P = conv_P(c), Q = conv_Q(c);
     const int64_t Np = round_up(c->N, 16);
     const int64_t NB = nb32(Np);
     const int wkb = largest_wkb(NB);
     const int bqk = 4 / wkb;
-    kiters = int64_t(P) * ceil_div(Q, bqk) * (NB / wkb);
-    BN = choose_bn(c->C);
-    const int64_t base = ceil_div(c->K, 128) * ceil_div(c->C, BN) * int64_t(c->R) * c->S;
+    const int ntaps = c->R * c->S;
+    w.kiters = int64_t(P) * ceil_div(Q, bqk) * (NB / wkb);
+    w.cpad = static_cast<int>(round_up(c->C, 8));
+    if (ntaps > 1 && c->C <= 128) {
+        const int most = std::max(1, 256 / w.cpad);
+        w.ngroups = static_cast<int>(ceil_div(ntaps, most));
+        w.ntg = static_cast<int>(ceil_div(ntaps, w.ngroups));
+        w.BN = static_cast<int>(round_up(w.ntg * w.cpad, 16));
+    } else {
+        w.ntg = 1;
+        w.ngroups = ntaps;
+        w.BN = choose_bn(c->C);
+    }
+    const int64_t base = ceil_div(c->K, 128) * ceil_div(c->C, w.ntg > 1 ? c->C : w.BN) * int64_t(w.ngroups);
     int64_t sp = base >= d.sms ? 1 : d.sms / base;
-    sp = std::min<int64_t>(sp, std::max<int64_t>(1, kiters / 8));
-    splits = static_cast<int>(std::max<int64_t>(1, sp));
+    sp = std::min<int64_t>(sp, std::max<int64_t>(1, w.kiters / 8));
+    w.splits = static_cast<int>(std::max<int64_t>(1, sp));
+    return w;
 }
 
 size_t mqc_conv2d_bwd_weight_workspace_bytes(const mqc_conv *c, const mqc_mx *gf, const mqc_mx *xf) {
@@ -761,11 +822,9 @@ size_t mqc_conv2d_bwd_weight_workspace_bytes(const mqc_conv *c, const mqc_mx *gf
     if (!conv_ok(c)) return 0;
     DevInfo *dv;
     if (dev_info(dv) != MQC_OK) return 0;
-    int BN, splits;
-    int64_t kiters;
-    wgrad_plan(c, *dv, BN, splits, kiters);
-    if (splits <= 1) return 0;
-    return size_t(splits) * size_t(c->K) * c->C * c->R * c->S * sizeof(float);
+    const WgradPlan w = wgrad_plan(c, *dv);
+    if (w.splits <= 1) return 0;
+    return size_t(w.splits) * size_t(c->K) * c->C * c->R * c->S * sizeof(float);
 }
 
 mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx *gf, const void *xq,
@@ -784,9 +843,14 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     const int64_t Np = round_up(N, 16);
     GemmParams G;
     memset(&G, 0, sizeof G);
-    int64_t kiters;
     if (sh * sw > 4) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_weight: stride product above 4");
-    wgrad_plan(c, *dv, G.BN, G.splits, kiters);
+    const WgradPlan plan = wgrad_plan(c, *dv);
+    const int64_t kiters = plan.kiters;
+    G.BN = plan.BN;
+    G.splits = plan.splits;
+    G.ntg = plan.ntg;
+    G.ngroups = plan.ngroups;
+    G.cpad = plan.cpad;
     const size_t need = G.splits > 1 ? size_t(G.splits) * K * C * R * S * sizeof(float) : 0;
     if (need > 0 && (workspace == nullptr || workspace_bytes < need))
         return fail(MQC_ERR_WORKSPACE, "conv2d_bwd_weight: needs %zu workspace bytes", need);
@@ -801,7 +865,7 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     G.Q = Q;
     G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
     G.MT = static_cast<int32_t>(ceil_div(K, 128));
-    G.NT = static_cast<int32_t>(ceil_div(C, G.BN));
+    G.NT = G.ntg > 1 ? 1 : static_cast<int32_t>(ceil_div(C, G.BN));
     G.Mrows = K;
     G.Ncols = C;
     G.x_st_h = sh;
@@ -810,7 +874,7 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     {
         const uint64_t dims[4] = {uint64_t(Np), uint64_t(K), uint64_t(Q), uint64_t(P)};
         const uint64_t strd[3] = {uint64_t(Np), uint64_t(K) * Np, uint64_t(Q) * K * Np};
-        const uint32_t box[4] = {uint32_t(32 * G.wkb), 128u, uint32_t(G.bqk), 1u};
+        const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(box_rows(K, 128)), uint32_t(G.bqk), 1u};
         if ((st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb)) != MQC_OK) return st;
     }
     bool phase_ok[16] = {};
@@ -822,7 +886,11 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
             const uint8_t *base = static_cast<const uint8_t *>(xq) + (int64_t(a) * W + b) * C * Np;
             const uint64_t dims[4] = {uint64_t(Np), uint64_t(C), uint64_t(Ww), uint64_t(Hh)};
             const uint64_t strd[3] = {uint64_t(Np), uint64_t(sw) * C * Np, uint64_t(sh) * W * C * Np};
-            const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.BN), uint32_t(G.bqk), 1u};
+            // one tap: a box over the kit's bqk pixels; tap groups: one pixel
+            // of one tap per box (cpad rows), placed at that tap's rows
+            const uint32_t box[4] = {uint32_t(32 * G.wkb),
+                                     uint32_t(G.ntg > 1 ? G.cpad : box_rows(C, G.BN)),
+                                     uint32_t(G.ntg > 1 ? 1 : G.bqk), 1u};
             if ((st = encode_codes_map(&G.bmap[a * sw + b], base, 4, dims, strd, box, G.wkb)) != MQC_OK) return st;
         }
     G.ntaps = 0;
@@ -853,8 +921,10 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
                 if (phase_ok[j]) { G.bmap[i] = G.bmap[j]; break; }
     G.n_amaps = 1;
     G.n_bmaps = sh * sw;
-    G.a_box_bytes = 32 * G.wkb * 128 * G.bqk;
-    G.b_box_bytes = 32 * G.wkb * G.BN * G.bqk;
+    G.a_slab = box_rows(K, 128);
+    G.b_slab = G.ntg > 1 ? G.BN : box_rows(C, G.BN);
+    G.a_box_bytes = 32 * G.wkb * G.a_slab * G.bqk;
+    G.b_box_bytes = G.ntg > 1 ? 32 * G.wkb * G.cpad : 32 * G.wkb * G.b_slab * G.bqk;
     const bool sqg = gf->block == MQC_BLOCK_SQ32, sqx = xf->block == MQC_BLOCK_SQ32;
     G.sfa.base = gs;
     G.sfa.pix_pitch = nb32(Np) * (sqg ? nb32(K) : K);
@@ -877,7 +947,7 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     G.os_m = int64_t(C) * R * S;
     G.os_c = int64_t(R) * S;
     G.split_pitch = int64_t(K) * C * R * S;
-    G.num_units = G.MT * G.NT * G.ntaps * G.splits;
+    G.num_units = G.MT * G.NT * G.ngroups * G.splits;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     if ((st = launch_gemm<kWgrad>(G, *dv, strm)) != MQC_OK) return st;
     if (G.splits > 1) {

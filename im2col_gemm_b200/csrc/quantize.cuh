@@ -322,3 +322,176 @@ inline void launch_quantize_blk(const QuantParams &p, int blk, bool dual, int it
 }
 
 }  // namespace mqc
+
+namespace mqc {
+
+// ---------------------------------------------------------------------------
+// Staged variant for the common case: FP8 codes, the spatial positions of the
+// source contiguous (NCHW-like, H*W flattened) and every plane 16-byte
+// aligned.  A CTA copies its whole fp32 tile (PT positions x OT rows of the
+// primary order's outer axis x IT of its inner axis, 64 KB) into shared
+// memory with 16-byte cp.async, all copies in flight at once, then works from
+// shared memory only: block maxima (pass 0), the primary rows (pass 1) and
+// the second code order (pass 2).  Three CTAs per SM keep about 200 KB of
+// loads in flight per SM.  Same arithmetic as mx_quantize_kernel: value times
+// the exact power of two 2^-e, then cvt.rn.satfinite.
+constexpr int kStagedTileBytes = 65536;
+
+struct StagedParams {
+    QuantParams q;
+    int32_t PT, OT, IT;          // tile extents (PT * OT * IT * 4 = 64 KB)
+    int32_t nPT, nOT, nIT;       // tile counts
+    int32_t blk;                 // kAlongI, kAlongO or kSquare
+    int32_t map_a;               // the inner axis i is A (order BA)
+};
+
+__device__ __forceinline__ void cp_async_16(void *smem, const void *gmem, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid_constant__ StagedParams sp) {
+    extern __shared__ __align__(16) uint8_t smem_q[];
+    float *tile = reinterpret_cast<float *>(smem_q);                        // [o][i][pos]
+    float *s_inv = reinterpret_cast<float *>(smem_q + kStagedTileBytes);    // [block][pos], up to 32 x 64
+    int *s_amax = reinterpret_cast<int *>(s_inv + 32 * 64);                 // [pos] (square blocks)
+    const QuantParams &p = sp.q;
+    const int PT = sp.PT, OT = sp.OT, IT = sp.IT;
+    const int NS = 256 / PT;                 // threads per position
+    const int tid = threadIdx.x;
+    const int pos = tid % PT, sub = tid / PT;
+
+    int t = blockIdx.x;
+    const int pT = t % sp.nPT;
+    t /= sp.nPT;
+    const int oT = t % sp.nOT;
+    const int iT = t / sp.nOT;
+    const int p0 = pT * PT, o0 = oT * OT, i0 = iT * IT;
+    const int64_t so = sp.map_a ? p.sb : p.sa, si = sp.map_a ? p.sa : p.sb;
+
+    // ---- stage the tile: chunk = 4 positions of one (o, i) row
+    {
+        const int cpr = PT / 4;              // chunks per row
+        for (int c = tid; c < OT * IT * cpr; c += 256) {
+            const int row = c / cpr, pc = c - row * cpr;
+            const int o = row / IT, i = row - o * IT;
+            const int pix = p0 + 4 * pc;
+            int bytes = 0;
+            const float *g = p.src;
+            if (o0 + o < p.O && i0 + i < p.I && pix < p.npix) {
+                bytes = 4 * min(4, p.npix - pix);
+                g = p.src + (o0 + o) * so + (i0 + i) * si + pix;
+            }
+            cp_async_16(tile + row * PT + 4 * pc, g, bytes);
+        }
+        if (sp.blk == kSquare && tid < PT) s_amax[tid] = 0;
+        cp_async_wait_all();
+        __syncthreads();
+    }
+    const int pix = p0 + pos;
+    const bool pix_ok = pix < p.npix;
+    const int nbA = (p.Ap1 + 31) / 32, nbB = (p.Bp1 + 31) / 32;
+
+    // ---- pass 0: block maxima and scales
+    if (sp.blk == kSquare) {
+        float m = 0.0f;
+        for (int o = sub; o < OT; o += NS)
+            for (int i = 0; i < IT; ++i) m = fmaxf(m, fabsf(tile[(o * IT + i) * PT + pos]));
+        atomicMax(s_amax + pos, __float_as_int(m));
+        __syncthreads();
+        if (sub == 0) {
+            const uint32_t c = e8m0_code(__int_as_float(s_amax[pos]), p.emax);
+            s_inv[pos] = e8m0_inv(c);
+            if (pix_ok) {
+                const int bT = sp.map_a ? oT : iT, aT = sp.map_a ? iT : oT;
+                p.scales[(static_cast<int64_t>(pix) * nbB + bT) * nbA + aT] = static_cast<uint8_t>(c);
+            }
+        }
+    } else if (sp.blk == kAlongI) {          // one block per (pos, o) row
+        for (int o = sub; o < OT; o += NS) {
+            float m = 0.0f;
+            for (int i = 0; i < IT; ++i) m = fmaxf(m, fabsf(tile[(o * IT + i) * PT + pos]));
+            const uint32_t c = e8m0_code(m, p.emax);
+            s_inv[o * PT + pos] = e8m0_inv(c);
+            const int og = o0 + o;
+            if (pix_ok) {
+                if (sp.map_a) {              // A32: row b = o, block iT along a
+                    if (og < p.Bp1) p.scales[(static_cast<int64_t>(pix) * p.Bp1 + og) * nbA + iT] = static_cast<uint8_t>(c);
+                } else {                     // B32: column a = o, block iT along b
+                    if (og < p.Ap1) p.scales[(static_cast<int64_t>(pix) * nbB + iT) * p.Ap1 + og] = static_cast<uint8_t>(c);
+                }
+            }
+        }
+    } else {                                 // one block per (pos, i) column
+        for (int i = sub; i < IT; i += NS) {
+            float m = 0.0f;
+            for (int o = 0; o < OT; ++o) m = fmaxf(m, fabsf(tile[(o * IT + i) * PT + pos]));
+            const uint32_t c = e8m0_code(m, p.emax);
+            s_inv[i * PT + pos] = e8m0_inv(c);
+            const int ig = i0 + i;
+            if (pix_ok) {
+                if (sp.map_a) {              // B32: block oT along b, column a = i
+                    if (ig < p.Ap1) p.scales[(static_cast<int64_t>(pix) * nbB + oT) * p.Ap1 + ig] = static_cast<uint8_t>(c);
+                } else {                     // A32: row b = i, block oT along a
+                    if (ig < p.Bp1) p.scales[(static_cast<int64_t>(pix) * p.Bp1 + ig) * nbA + oT] = static_cast<uint8_t>(c);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (!pix_ok) return;
+    auto inv_of = [&](int o, int i) -> float {
+        return sp.blk == kSquare ? s_inv[pos] : (sp.blk == kAlongI ? s_inv[o * PT + pos] : s_inv[i * PT + pos]);
+    };
+
+    // ---- pass 1: primary rows [pix][o][i0 .. i0 + IT) (clipped to the padded I1)
+    const int prow = min(IT, p.I1 - i0);     // 16 or 32 bytes
+    for (int o = sub; o < OT; o += NS) {
+        if (o0 + o >= p.O) break;
+        uint32_t words[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            uint32_t v = 0u;
+            if (4 * w < IT) {
+                const float *tp = tile + (o * IT + 4 * w) * PT + pos;
+                const uint32_t lo = cvt_pair<FMT>(tp[0] * inv_of(o, 4 * w), tp[PT] * inv_of(o, 4 * w + 1));
+                const uint32_t hi = cvt_pair<FMT>(tp[2 * PT] * inv_of(o, 4 * w + 2), tp[3 * PT] * inv_of(o, 4 * w + 3));
+                v = lo | (hi << 16);
+            }
+            words[w] = v;
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(p.codes + (static_cast<int64_t>(pix) * p.O + o0 + o) * p.I1 + i0);
+        dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+        if (prow == 32) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+    }
+    if (p.codes_alt == nullptr) return;
+
+    // ---- pass 2: second order rows [pix][i][o0 .. o0 + OT) (clipped to the padded O2)
+    const int arow = min(OT, p.O2 - o0);
+    if (arow <= 0) return;
+    for (int i = sub; i < IT; i += NS) {
+        if (i0 + i >= p.I) break;
+        uint32_t words[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            uint32_t v = 0u;
+            if (4 * w < OT) {
+                const float *tp = tile + (4 * w * IT + i) * PT + pos;
+                const int st = IT * PT;
+                const uint32_t lo = cvt_pair<FMT>(tp[0] * inv_of(4 * w, i), tp[st] * inv_of(4 * w + 1, i));
+                const uint32_t hi = cvt_pair<FMT>(tp[2 * st] * inv_of(4 * w + 2, i), tp[3 * st] * inv_of(4 * w + 3, i));
+                v = lo | (hi << 16);
+            }
+            words[w] = v;
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(p.codes_alt + (static_cast<int64_t>(pix) * p.I + i0 + i) * p.O2 + o0);
+        dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+        if (arow == 32) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+    }
+}
+
+}  // namespace mqc

@@ -66,7 +66,8 @@ def test_element_encoding_every_fp32_in_range(mqc, orc, fmt):
     assert np.array_equal(_host(q.codes), orc.quantize(x, fmt, 0, 0)[0])
 
 
-SHAPES = [(2, 32, 8, 8), (37, 45, 3, 5), (16, 16, 33, 17), (64, 96, 4, 6), (5, 3, 2, 40), (40, 70, 1, 1)]
+SHAPES = [(2, 32, 8, 8), (37, 45, 3, 5), (16, 16, 33, 17), (64, 96, 4, 6), (5, 3, 2, 40), (40, 70, 1, 1),
+          (24, 40, 4, 8)]
 
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])

@@ -87,7 +87,7 @@ struct DevInfo {
     int sms = 0;
     int max_smem = 0;
     bool gemm_attr[4] = {false, false, false, false};   // [KIND * 2 + SFV4]
-    bool quant_attr[2] = {false, false};                  // staged quantizer, [fmt]
+    bool quant_attr[24] = {};                             // staged quantizer, [(fmt*3 + blk)*4 + tile]
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
@@ -419,13 +419,13 @@ mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, 
         const int64_t ntiles = int64_t(sp.nPT) * sp.nOT * sp.nIT;
         if (ntiles > (int64_t(1) << 31) - 1) return fail(MQC_ERR_INVALID, "quantize: tensor too large");
         const int smem = kStagedTileBytes + 32 * 64 * 4 + 64 * 4;
-        auto kernel = p.fmt == MQC_E4M3 ? mx_quantize_staged_kernel<0> : mx_quantize_staged_kernel<1>;
-        if (!dv->quant_attr[p.fmt]) {
-            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-            dv->quant_attr[p.fmt] = true;
-        }
-        kernel<<<static_cast<unsigned>(ntiles), 256, smem, s>>>(sp);
+        // the shared-memory limit is raised once per (format, block, tile) kernel
+        const int ai = (p.fmt * 3 + blk) * 4 + (sp.OT == 32 ? 2 : 0) + (sp.IT == 32 ? 1 : 0);
+        cudaError_t ae = cudaSuccess;
+        if (p.fmt == MQC_E4M3) launch_staged<0>(sp, static_cast<unsigned>(ntiles), smem, s, ae, !dv->quant_attr[ai]);
+        else launch_staged<1>(sp, static_cast<unsigned>(ntiles), smem, s, ae, !dv->quant_attr[ai]);
+        if (ae != cudaSuccess) return cuda_fail(ae, "cudaFuncSetAttribute");
+        dv->quant_attr[ai] = true;
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "mx_quantize_staged_kernel launch");
         return MQC_OK;

@@ -353,15 +353,19 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-template <int FMT>
+// OT, IT: tile extents (16 or 32); PT = positions per tile; NS = threads per
+// position.  A thread owns o-rows {sub, sub + NS, ...} in the primary pass and
+// i-columns {sub, sub + NS, ...} in the second-order pass (64 values each).
+template <int FMT, int BLK, int OT, int IT>
 __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid_constant__ StagedParams sp) {
+    constexpr int PT = kStagedTileBytes / (4 * OT * IT);
+    constexpr int NS = 256 / PT;
+    constexpr int RO = OT / NS, RI = IT / NS;       // owned rows / columns per thread
     extern __shared__ __align__(16) uint8_t smem_q[];
     float *tile = reinterpret_cast<float *>(smem_q);                        // [o][i][pos]
-    float *s_inv = reinterpret_cast<float *>(smem_q + kStagedTileBytes);    // [block][pos], up to 32 x 64
+    float *s_inv = reinterpret_cast<float *>(smem_q + kStagedTileBytes);    // [block][pos]
     int *s_amax = reinterpret_cast<int *>(s_inv + 32 * 64);                 // [pos] (square blocks)
     const QuantParams &p = sp.q;
-    const int PT = sp.PT, OT = sp.OT, IT = sp.IT;
-    const int NS = 256 / PT;                 // threads per position
     const int tid = threadIdx.x;
     const int pos = tid % PT, sub = tid / PT;
 
@@ -375,10 +379,11 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
 
     // ---- stage the tile: chunk = 4 positions of one (o, i) row
     {
-        const int cpr = PT / 4;              // chunks per row
-        for (int c = tid; c < OT * IT * cpr; c += 256) {
-            const int row = c / cpr, pc = c - row * cpr;
-            const int o = row / IT, i = row - o * IT;
+        constexpr int CPR = PT / 4;          // chunks per row
+#pragma unroll 4
+        for (int c = tid; c < OT * IT * CPR; c += 256) {
+            const int row = c / CPR, pc = c % CPR;
+            const int o = row / IT, i = row % IT;
             const int pix = p0 + 4 * pc;
             int bytes = 0;
             const float *g = p.src;
@@ -388,19 +393,22 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
             }
             cp_async_16(tile + row * PT + 4 * pc, g, bytes);
         }
-        if (sp.blk == kSquare && tid < PT) s_amax[tid] = 0;
+        if (BLK == kSquare && tid < PT) s_amax[tid] = 0;
         cp_async_wait_all();
         __syncthreads();
     }
     const int pix = p0 + pos;
     const bool pix_ok = pix < p.npix;
     const int nbA = (p.Ap1 + 31) / 32, nbB = (p.Bp1 + 31) / 32;
+    const float *tp = tile + pos;
 
     // ---- pass 0: block maxima and scales
-    if (sp.blk == kSquare) {
+    if (BLK == kSquare) {
         float m = 0.0f;
-        for (int o = sub; o < OT; o += NS)
-            for (int i = 0; i < IT; ++i) m = fmaxf(m, fabsf(tile[(o * IT + i) * PT + pos]));
+#pragma unroll
+        for (int r = 0; r < RO; ++r)
+#pragma unroll
+            for (int i = 0; i < IT; ++i) m = fmaxf(m, fabsf(tp[((sub + NS * r) * IT + i) * PT]));
         atomicMax(s_amax + pos, __float_as_int(m));
         __syncthreads();
         if (sub == 0) {
@@ -411,10 +419,13 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
                 p.scales[(static_cast<int64_t>(pix) * nbB + bT) * nbA + aT] = static_cast<uint8_t>(c);
             }
         }
-    } else if (sp.blk == kAlongI) {          // one block per (pos, o) row
-        for (int o = sub; o < OT; o += NS) {
+    } else if (BLK == kAlongI) {             // one block per (pos, o) row
+#pragma unroll
+        for (int r = 0; r < RO; ++r) {
+            const int o = sub + NS * r;
             float m = 0.0f;
-            for (int i = 0; i < IT; ++i) m = fmaxf(m, fabsf(tile[(o * IT + i) * PT + pos]));
+#pragma unroll
+            for (int i = 0; i < IT; ++i) m = fmaxf(m, fabsf(tp[(o * IT + i) * PT]));
             const uint32_t c = e8m0_code(m, p.emax);
             s_inv[o * PT + pos] = e8m0_inv(c);
             const int og = o0 + o;
@@ -427,9 +438,12 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
             }
         }
     } else {                                 // one block per (pos, i) column
-        for (int i = sub; i < IT; i += NS) {
+#pragma unroll
+        for (int r = 0; r < RI; ++r) {
+            const int i = sub + NS * r;
             float m = 0.0f;
-            for (int o = 0; o < OT; ++o) m = fmaxf(m, fabsf(tile[(o * IT + i) * PT + pos]));
+#pragma unroll
+            for (int o = 0; o < OT; ++o) m = fmaxf(m, fabsf(tp[(o * IT + i) * PT]));
             const uint32_t c = e8m0_code(m, p.emax);
             s_inv[i * PT + pos] = e8m0_inv(c);
             const int ig = i0 + i;
@@ -444,54 +458,89 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
     }
     __syncthreads();
     if (!pix_ok) return;
-    auto inv_of = [&](int o, int i) -> float {
-        return sp.blk == kSquare ? s_inv[pos] : (sp.blk == kAlongI ? s_inv[o * PT + pos] : s_inv[i * PT + pos]);
-    };
 
     // ---- pass 1: primary rows [pix][o][i0 .. i0 + IT) (clipped to the padded I1)
-    const int prow = min(IT, p.I1 - i0);     // 16 or 32 bytes
-    for (int o = sub; o < OT; o += NS) {
-        if (o0 + o >= p.O) break;
-        uint32_t words[8];
+    {
+        const bool full_row = IT == 16 || p.I1 - i0 >= 32;
+        float inv_i[BLK == kAlongO ? IT : 1];
+        if (BLK == kAlongO) {
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            uint32_t v = 0u;
-            if (4 * w < IT) {
-                const float *tp = tile + (o * IT + 4 * w) * PT + pos;
-                const uint32_t lo = cvt_pair<FMT>(tp[0] * inv_of(o, 4 * w), tp[PT] * inv_of(o, 4 * w + 1));
-                const uint32_t hi = cvt_pair<FMT>(tp[2 * PT] * inv_of(o, 4 * w + 2), tp[3 * PT] * inv_of(o, 4 * w + 3));
-                v = lo | (hi << 16);
-            }
-            words[w] = v;
+            for (int i = 0; i < (BLK == kAlongO ? IT : 1); ++i) inv_i[i] = s_inv[i * PT + pos];
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(p.codes + (static_cast<int64_t>(pix) * p.O + o0 + o) * p.I1 + i0);
-        dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-        if (prow == 32) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+        const float inv_sq = BLK == kSquare ? s_inv[pos] : 1.0f;
+#pragma unroll
+        for (int r = 0; r < RO; ++r) {
+            const int o = sub + NS * r;
+            if (o0 + o >= p.O) break;
+            const float inv_row = BLK == kAlongI ? s_inv[o * PT + pos] : inv_sq;
+            uint32_t w[IT / 4];
+#pragma unroll
+            for (int q = 0; q < IT / 4; ++q) {
+                float v[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    v[k] = tp[(o * IT + 4 * q + k) * PT] * (BLK == kAlongO ? inv_i[(4 * q + k) % (BLK == kAlongO ? IT : 1)] : inv_row);
+                w[q] = cvt_pair<FMT>(v[0], v[1]) | (cvt_pair<FMT>(v[2], v[3]) << 16);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(p.codes + (static_cast<int64_t>(pix) * p.O + o0 + o) * p.I1 + i0);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            if (IT == 32 && full_row) dst[1] = make_uint4(w[4 % (IT / 4)], w[5 % (IT / 4)], w[6 % (IT / 4)], w[7 % (IT / 4)]);
+        }
     }
     if (p.codes_alt == nullptr) return;
 
     // ---- pass 2: second order rows [pix][i][o0 .. o0 + OT) (clipped to the padded O2)
-    const int arow = min(OT, p.O2 - o0);
-    if (arow <= 0) return;
-    for (int i = sub; i < IT; i += NS) {
-        if (i0 + i >= p.I) break;
-        uint32_t words[8];
+    {
+        const bool full_row = OT == 16 || p.O2 - o0 >= 32;
+        float inv_o[BLK == kAlongI ? OT : 1];
+        if (BLK == kAlongI) {
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            uint32_t v = 0u;
-            if (4 * w < OT) {
-                const float *tp = tile + (4 * w * IT + i) * PT + pos;
-                const int st = IT * PT;
-                const uint32_t lo = cvt_pair<FMT>(tp[0] * inv_of(4 * w, i), tp[st] * inv_of(4 * w + 1, i));
-                const uint32_t hi = cvt_pair<FMT>(tp[2 * st] * inv_of(4 * w + 2, i), tp[3 * st] * inv_of(4 * w + 3, i));
-                v = lo | (hi << 16);
-            }
-            words[w] = v;
+            for (int o = 0; o < (BLK == kAlongI ? OT : 1); ++o) inv_o[o] = s_inv[o * PT + pos];
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(p.codes_alt + (static_cast<int64_t>(pix) * p.I + i0 + i) * p.O2 + o0);
-        dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-        if (arow == 32) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+        const float inv_sq = BLK == kSquare ? s_inv[pos] : 1.0f;
+#pragma unroll
+        for (int r = 0; r < RI; ++r) {
+            const int i = sub + NS * r;
+            if (i0 + i >= p.I) break;
+            const float inv_col = BLK == kAlongO ? s_inv[i * PT + pos] : inv_sq;
+            uint32_t w[OT / 4];
+#pragma unroll
+            for (int q = 0; q < OT / 4; ++q) {
+                float v[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    v[k] = tp[((4 * q + k) * IT + i) * PT] * (BLK == kAlongI ? inv_o[(4 * q + k) % (BLK == kAlongI ? OT : 1)] : inv_col);
+                w[q] = cvt_pair<FMT>(v[0], v[1]) | (cvt_pair<FMT>(v[2], v[3]) << 16);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(p.codes_alt + (static_cast<int64_t>(pix) * p.I + i0 + i) * p.O2 + o0);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            if (OT == 32 && full_row) dst[1] = make_uint4(w[4 % (OT / 4)], w[5 % (OT / 4)], w[6 % (OT / 4)], w[7 % (OT / 4)]);
+        }
     }
+}
+
+template <int FMT, int BLK>
+inline void launch_staged_tiles(const StagedParams &sp, unsigned grid, int smem, cudaStream_t s, cudaError_t &attr_err,
+                                bool set_attr) {
+    auto pick = [&](auto kernel) {
+        if (set_attr) {
+            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) attr_err = e;
+        }
+        kernel<<<grid, 256, smem, s>>>(sp);
+    };
+    if (sp.OT == 16 && sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 16>);
+    else if (sp.OT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 32>);
+    else if (sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 32, 16>);
+    else pick(mx_quantize_staged_kernel<FMT, BLK, 32, 32>);
+}
+
+template <int FMT>
+inline void launch_staged(const StagedParams &sp, unsigned grid, int smem, cudaStream_t s, cudaError_t &attr_err,
+                          bool set_attr) {
+    if (sp.blk == kAlongI) launch_staged_tiles<FMT, kAlongI>(sp, grid, smem, s, attr_err, set_attr);
+    else if (sp.blk == kAlongO) launch_staged_tiles<FMT, kAlongO>(sp, grid, smem, s, attr_err, set_attr);
+    else launch_staged_tiles<FMT, kSquare>(sp, grid, smem, s, attr_err, set_attr);
 }
 
 }  // namespace mqc

@@ -21,6 +21,8 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import glob
+import hashlib
 import json
 import os
 import statistics
@@ -146,6 +148,32 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- peaks
+def kernel_sources_sha256() -> str:
+    """Hash of the CUDA sources and the C header: DRAM counters taken by ncu
+    on one version of the kernels are reported only for that version."""
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "im2col_gemm_b200", "csrc", "*.cu*")))
+    for f in files + [os.path.join(ROOT, "include", "mqc.h")]:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel: str):
+    """dram__bytes_read.sum + dram__bytes_write.sum of one launch of `kernel`
+    (e.g. "dgrad layer 0") from the ncu record under profiles/, or None when
+    no record exists for the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("sources_sha256") != kernel_sources_sha256():
+        return None
+    k = rec.get("calls", {}).get(kernel)
+    return None if k is None else k["dram_bytes_read"] + k["dram_bytes_write"]
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -213,8 +241,12 @@ class LayerBuffers:
         return qg.codes.numel() + qg.scales.numel() + qx.codes.numel() + qx.scales.numel() + 4 * self.gw.numel()
 
     def launches(self, mqc):
+        """Kernels one pass of this layer launches: 3 quantizations, the
+        forward GEMM, the input gradient (its stride phases share launches of
+        up to 4 height phases), the weight-gradient GEMM and, with split-K
+        partials, their reduction."""
         L = self.L
-        return 3 + 1 + L.stride * L.stride + (2 if self.ws_bytes > 0 else 1)
+        return 3 + 1 + -(-L.stride // 4) + (2 if self.ws_bytes > 0 else 1)
 
 
 def run_layer(mqc, lb: LayerBuffers, workspace, stream, events=None, only=None):
@@ -513,7 +545,8 @@ def main(argv=None):
         achieved = top["flops"] / (top["ms"] * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp8_peak}
-    roof.update({"traffic": None, "kernel": f"{top['call']} layer {top['layer']}",
+    top_name = f"{top['call']} layer {top['layer']}"
+    roof.update({"traffic": measured_traffic(top_name), "kernel": top_name,
                  "share": top["ms"] / total_call_ms, "peak_source": pk["source"] + " (MXFP8 = 2 x bf16)"
                  if roof["bound"] == "tensor" else pk["source"]})
     qcalls = [c for c in calls if c["call"].startswith("quantize")]

@@ -48,6 +48,7 @@ __device__ __forceinline__ int sf_warp_index(int warp) {
     return warp == 2 ? 0 : warp == 3 ? 1 : warp == 8 ? 2 : warp == 10 ? 3 : warp == 11 ? 4 : -1;
 }
 constexpr int kTmemCols = 512;
+constexpr int kMaxAcc = 4;       // accumulator ring: tiles between the MMA issuer and the epilogue
 constexpr int kSfTmemBase = 256;
 
 enum GemmKind : int { kConv = 0, kWgrad = 1 };
@@ -80,7 +81,7 @@ struct alignas(64) GemmParams {
     ConvTap taps[kMaxTaps];
     int32_t ntaps;
     int32_t n_amaps, n_bmaps;    // tensor maps in use
-    int32_t BN, nb_atoms, wkb, stages, nacc;
+    int32_t BN, nb_atoms, wkb, stages, nacc, lg_nacc;   // nacc accumulators in TMEM (1, 2 or 4)
     int32_t kbs;                 // K-blocks (of 32) per pipeline stage: 4 or 8
     uint32_t idesc;
     uint64_t timeout_ns;
@@ -103,6 +104,10 @@ struct alignas(64) GemmParams {
     int32_t sfb_vec4;            // B: likewise (the weights' scales along C)
     int32_t sfb_cached;          // CONV: B scale atoms of every (column tile, group) built once per CTA
     int32_t groups;              // CONV: groups of 4 K-blocks per tile
+    // CONV: a unit is um consecutive 128-row tiles (sub-tiles) sharing the
+    // B operand, the pipeline stages and the per-unit bookkeeping; each
+    // sub-tile has its own accumulator (um x BN TMEM columns per unit)
+    int32_t um, MTILES;
     int32_t bq, bp, bn;          // A box extents along q, p, n
     int32_t TQ, TP, TN, NT;      // tile counts
     int32_t Ne;                  // output extent along n (row mask)
@@ -136,6 +141,7 @@ struct alignas(64) GemmParams {
 struct UnitInfo {
     int nk;                 // pipeline stages of this unit
     int nt;                 // column tile
+    int mt0;                // CONV: first 128-row tile of the unit
     int ph, tap0, tkb;      // CONV: output phase, its first tap and K-blocks
     int kbase, nkit;        // WGRAD: first kit and number of kits
     int q0, p0, n0;         // CONV: tile origin
@@ -151,8 +157,10 @@ __device__ __forceinline__ UnitInfo decode_unit(const GemmParams &p, int u) {
     if (KIND == kConv) {
         const uint32_t r = p.fd_NT.div(u);
         const int nt = u - static_cast<int>(r) * p.NT;
-        const uint32_t mt = p.fd_nph.div(r);
-        const int ph = static_cast<int>(r - mt * p.nph);
+        const uint32_t mg = p.fd_nph.div(r);
+        const int ph = static_cast<int>(r - mg * p.nph);
+        const uint32_t mt = mg * p.um;
+        I.mt0 = static_cast<int>(mt);
         const uint32_t m2 = p.fd_TQ.div(mt);
         const int tq = static_cast<int>(mt - m2 * p.TQ);
         const uint32_t tn = p.fd_TP.div(m2);
@@ -210,6 +218,17 @@ __device__ __forceinline__ void conv_row(const GemmParams &p, int m, int &aw, in
     }
 }
 
+// Origin (q, p, n) of the 128-row tile mt of a CONV launch (tiles run q
+// fastest, then p, then n; mt past the last tile gives n >= N: all rows out
+// of range, its boxes read zeros).
+__device__ __forceinline__ void tile_origin(const GemmParams &p, int mt, int &q0, int &p0, int &n0) {
+    const uint32_t m2 = p.fd_TQ.div(mt);
+    const uint32_t tn = p.fd_TP.div(m2);
+    q0 = (mt - static_cast<int>(m2) * p.TQ) * p.bq;
+    p0 = (static_cast<int>(m2) - static_cast<int>(tn) * p.TP) * p.bp;
+    n0 = static_cast<int>(tn) * p.bn;
+}
+
 __device__ __forceinline__ uint32_t swizzle_of(int wkb) {
     return wkb == 4 ? kSwizzle128B : (wkb == 2 ? kSwizzle64B : kSwizzle32B);
 }
@@ -251,7 +270,11 @@ struct KitWalker {
 // byte per (row, K-block).  The choice is a template parameter so that each
 // kernel carries only one gather path (the per-stage code of all roles has to
 // share the instruction cache).
-template <int KIND, bool SFV4>
+//
+// UMT (CONV only): 128-row sub-tiles per unit (1, 2 or 4; p.um equals it).
+// A template parameter as well, so that the one-tile kernel carries no
+// sub-tile loops.
+template <int KIND, bool SFV4, int UMT>
 __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
@@ -261,9 +284,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     const int GA = KS / 4;                    // groups of 4 K-blocks (one scale atom) per stage
     const int row_bytes = 32 * p.wkb;         // bytes of one operand row of a TMA box
     const int lg_wkb = p.wkb == 4 ? 2 : (p.wkb == 2 ? 1 : 0);
-    const int a_stage = 128 * 32 * KS;
+    constexpr int UM = KIND == kConv ? UMT : 1;   // 128-row sub-tiles per unit
+    const int a_sub_stage = 128 * 32 * KS;     // one sub-tile's A rows of a stage
+    const int a_stage = UM * a_sub_stage;
     const int b_stage = p.BN * 32 * KS;
-    const int sfa_stage = 512 * GA;
+    const int sfa_stage = 512 * GA * UM;       // A atoms [group][sub-tile]
     const int sfb_stage = 512 * GA * p.nb_atoms;
     uint8_t *sA = smem;
     uint8_t *sB = sA + S * a_stage;
@@ -276,8 +301,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     uint64_t *full = reinterpret_cast<uint64_t *>(sSFBc + sfbc_bytes);
     uint64_t *empty = full + S;
     uint64_t *acc_full = empty + S;
-    uint64_t *acc_empty = acc_full + 2;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *acc_empty = acc_full + kMaxAcc;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + kMaxAcc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -288,7 +313,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             mbar_init(&full[s], 2);
             mbar_init(&empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < kMaxAcc; ++a) {
             mbar_init(&acc_full[a], 1);
             mbar_init(&acc_empty[a], 4);
         }
@@ -337,7 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const uint64_t lim = p.timeout_ns;
-    const int sf_cols = GA * (4 + 4 * p.nb_atoms);   // TMEM scale columns per stage
+    const int sf_cols = GA * (4 * UM + 4 * p.nb_atoms);   // TMEM scale columns per stage
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -352,6 +377,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             KbWalker kw{I.tap0, 0};
             KitWalker kt{0, 0, 0};
             if (KIND == kWgrad) kt.init(p, I.kbase);
+            int oq[4], op[4], on[4];             // sub-tile origins
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                oq[i] = I.q0;
+                op[i] = I.p0;
+                on[i] = I.n0;
+                if (KIND == kConv && i > 0 && i < UM) tile_origin(p, I.mt0 + i, oq[i], op[i], on[i]);
+            }
             for (int ki = 0; ki < I.nk; ++ki, ++it, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag))) {
                     ok = false;
@@ -363,20 +396,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     const int nkb = min(KS, I.tkb - KS * ki);
                     const int nbox = nkb >> lg_wkb;
                     if (leader)
-                        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * (p.a_box_bytes + p.b_box_bytes)));
+                        mbar_arrive_expect_tx(&full[s],
+                                              static_cast<uint32_t>(nbox * (UM * p.a_box_bytes + p.b_box_bytes)));
                     for (int j = 0; j < nbox; ++j) {
                         const ConvTap T = p.taps[kw.tap];
                         const int cx = kw.cb * 32;
                         if (leader) {
-                            if (p.sub > 1)   // slot dimension of extent 1: only slot T.aw is in range
-                                tma_load_5d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx, -T.aw,
-                                            I.q0 + T.dw, I.p0 + T.dh, I.n0);
-                            else if (p.rows_nfirst)
-                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx, I.n0,
-                                            I.q0 + T.dw, I.p0 + T.dh);
-                            else
-                                tma_load_4d(a_dst + j * 128 * row_bytes, &p.amap[T.map], &full[s], cx, I.q0 + T.dw,
-                                            I.p0 + T.dh, I.n0);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                if (i >= UM) break;
+                                uint8_t *dst = a_dst + i * a_sub_stage + j * 128 * row_bytes;
+                                if (p.sub > 1)   // slot dimension of extent 1: only slot T.aw is in range
+                                    tma_load_5d(dst, &p.amap[T.map], &full[s], cx, -T.aw, oq[i] + T.dw, op[i] + T.dh,
+                                                on[i]);
+                                else if (p.rows_nfirst)
+                                    tma_load_4d(dst, &p.amap[T.map], &full[s], cx, on[i], oq[i] + T.dw, op[i] + T.dh);
+                                else
+                                    tma_load_4d(dst, &p.amap[T.map], &full[s], cx, oq[i] + T.dw, op[i] + T.dh, on[i]);
+                            }
                             tma_load_3d(b_dst + j * p.BN * row_bytes, &p.bmap[0], &full[s], cx, I.col0, T.btap);
                         }
                         kw.advance(p.wkb, p.CB);
@@ -441,11 +478,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
             if (I.nk == 0) continue;
-            const uint32_t acc = tcount & 1u & static_cast<uint32_t>(p.nacc - 1);
-            const uint32_t aph = (p.nacc == 2 ? (tcount >> 1) : tcount) & 1u;
+            const uint32_t acc = tcount & static_cast<uint32_t>(p.nacc - 1);
+            const uint32_t aph = (tcount >> p.lg_nacc) & 1u;
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_empty[acc], aph ^ 1u, lim, abort_flag))) break;
             tc_fence_after();
-            const uint32_t d_tmem = tmem + acc * p.BN;
+            const uint32_t d_tmem = tmem + acc * UM * p.BN;   // sub-tile i at + i * BN
             // cached B atoms of this column tile
             const int item_base = KIND == kConv ? (I.nt * p.groups + p.ph_gofs[I.ph]) * p.nb_atoms : 0;
             for (int ki = 0; ki < I.nk; ++ki, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
@@ -453,15 +490,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     ok = false;
                     break;
                 }
-                const uint32_t sf_t = tmem + kSfTmemBase + s * sf_cols;     // SFA groups, then SFB groups
-                const uint32_t sfb_t = sf_t + 4 * GA;
+                const uint32_t sf_t = tmem + kSfTmemBase + s * sf_cols;     // SFA [group][sub-tile], then SFB
+                const uint32_t sfb_t = sf_t + 4 * GA * UM;
                 const int nkb = KIND == kConv ? min(KS, I.tkb - KS * ki) : 4 * min(GA, I.nkit - GA * ki);
                 const int ngr = (nkb + 3) >> 2;
                 const uint64_t a_s = adesc0 + static_cast<uint64_t>((s * a_stage) >> 4);
                 const uint64_t b_s = bdesc0 + static_cast<uint64_t>((s * b_stage) >> 4);
                 if (leader) {
                     for (int g = 0; g < ngr; ++g) {
-                        tc_cp_32x128b_warpx4(sf_t + 4 * g, sfa_desc0 + static_cast<uint64_t>((s * sfa_stage + g * 512) >> 4));
+                        for (int i = 0; i < UM; ++i)
+                            tc_cp_32x128b_warpx4(sf_t + 4 * (g * UM + i),
+                                                 sfa_desc0 + static_cast<uint64_t>((s * sfa_stage + (g * UM + i) * 512) >> 4));
                         for (int a = 0; a < p.nb_atoms; ++a) {
                             const uint64_t src =
                                 (KIND == kConv && p.sfb_cached)
@@ -474,9 +513,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         const uint32_t g = static_cast<uint32_t>(kb >> 2), k4 = static_cast<uint32_t>(kb & 3);
                         const uint32_t j = k4 >> lg_wkb;                       // sub-tile within the group
                         const uint32_t within = k4 & static_cast<uint32_t>(p.wkb - 1);
-                        tc_mma_mxf8f6f4(d_tmem, a_s + g * a_grp + j * a_sub + within * 2, b_s + g * b_grp + j * b_sub + within * 2,
-                                        p.idesc | (k4 << 29) | (k4 << 4), (sf_t + 4 * g) | (k4 << 30),
-                                        (sfb_t + 4 * g * p.nb_atoms) | (k4 << 30), (ki > 0 || kb > 0) ? 1u : 0u);
+                        for (int i = 0; i < UM; ++i)
+                            tc_mma_mxf8f6f4(d_tmem + i * p.BN,
+                                            a_s + static_cast<uint64_t>((i * a_sub_stage) >> 4) + g * a_grp + j * a_sub + within * 2,
+                                            b_s + g * b_grp + j * b_sub + within * 2, p.idesc | (k4 << 29) | (k4 << 4),
+                                            (sf_t + 4 * (g * UM + i)) | (k4 << 30), (sfb_t + 4 * g * p.nb_atoms) | (k4 << 30),
+                                            (ki > 0 || kb > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                 }
@@ -507,31 +549,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             it += static_cast<uint32_t>(I.nk);
             if (gnext >= it) continue;
             const int first = static_cast<int>(gnext - it_unit);
-            // A rows of this lane: m = lane + 32 j
+            // A rows of this lane: m = lane + 32 j of sub-tile i
             int ra_h[4], ra_w[4], ra_off[4], ra_aw[4];
             bool ra_ok[4];
+            auto set_rows = [&](int i) {
+                int q0 = I.q0, p0 = I.p0, n0 = I.n0;
+                if (KIND == kConv && i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int m = lane + 32 * j;
-                if (KIND == kConv) {
-                    int aw, iq, ip, in;
-                    conv_row(p, m, aw, iq, ip, in);
-                    const int q = I.q0 + iq, pr = I.p0 + ip, n = I.n0 + in;
-                    ra_ok[j] = m < p.sub * p.bq * p.bp * p.bn && p.sub * q + aw < p.ph_Qe[I.ph] &&
-                               pr < p.ph_Pe[I.ph] && n < p.Ne;
-                    ra_h[j] = p.a_st_h * pr;
-                    ra_w[j] = p.a_st_w * q;
-                    ra_aw[j] = aw;
-                    ra_off[j] = (n >> p.sfa.row_shift) * p.sfa.row_pitch;
-                } else {
-                    const int k = I.m0 + m;
-                    ra_ok[j] = k < p.sfa.rows;
-                    ra_h[j] = 0;
-                    ra_w[j] = 0;
-                    ra_aw[j] = 0;
-                    ra_off[j] = (k >> p.sfa.row_shift) * p.sfa.row_pitch;
+                for (int j = 0; j < 4; ++j) {
+                    const int m = lane + 32 * j;
+                    if (KIND == kConv) {
+                        int aw, iq, ip, in;
+                        conv_row(p, m, aw, iq, ip, in);
+                        const int q = q0 + iq, pr = p0 + ip, n = n0 + in;
+                        ra_ok[j] = m < p.sub * p.bq * p.bp * p.bn && p.sub * q + aw < p.ph_Qe[I.ph] &&
+                                   pr < p.ph_Pe[I.ph] && n < p.Ne;
+                        ra_h[j] = p.a_st_h * pr;
+                        ra_w[j] = p.a_st_w * q;
+                        ra_aw[j] = aw;
+                        ra_off[j] = (n >> p.sfa.row_shift) * p.sfa.row_pitch;
+                    } else {
+                        const int k = I.m0 + m;
+                        ra_ok[j] = k < p.sfa.rows;
+                        ra_h[j] = 0;
+                        ra_w[j] = 0;
+                        ra_aw[j] = 0;
+                        ra_off[j] = (k >> p.sfa.row_shift) * p.sfa.row_pitch;
+                    }
                 }
-            }
+            };
+            set_rows(0);
             // B rows of this lane: col0 + 128 at + 32 j + lane
             // (WGRAD: with tap groups a B row is (tap, channel) and carries
             // its tap's pixel offset; otherwise every row has the unit's tap)
@@ -571,7 +618,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 KbWalker k2 = kw;
                 KitWalker k3 = kt;
                 bool slot = false;
-                for (int g = 0; g < GA; ++g) {
+                for (int g = 0; g < GA && ok; ++g) {
+                  const KbWalker kg = k2;                 // start of the group (each sub-tile walks it)
+                  for (int i = 0; i < UM; ++i) {
+                    if (UM > 1) {
+                        set_rows(i);
+                        k2 = kg;
+                    }
+                    const bool gb = i == 0 && !skip_b;      // B atoms: once per group
                     uint32_t wa[4] = {0u, 0u, 0u, 0u};      // [row j]
                     uint32_t wb[2][4] = {};                 // [atom][row j]
                     if (g < ngr) {
@@ -587,7 +641,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                                         p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
                                         ra_off[j] + cb));
                             }
-                            if (!skip_b) {
+                            if (gb) {
                                 const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb;
 #pragma unroll
                                 for (int at = 0; at < 2; ++at)
@@ -612,7 +666,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                                                      ra_off[j] + cb * p.sfa.kb_pitch))
                                                  << (8 * kb);
                                 }
-                                if (!skip_b) {
+                                if (gb) {
                                     const uint8_t *bsrc =
                                         p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
 #pragma unroll
@@ -674,15 +728,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         }
                         slot = true;
                     }
-                    *reinterpret_cast<uint4 *>(sSFA + s * sfa_stage + g * 512 + lane * 16) =
+                    *reinterpret_cast<uint4 *>(sSFA + s * sfa_stage + (g * UM + i) * 512 + lane * 16) =
                         make_uint4(wa[0], wa[1], wa[2], wa[3]);
-                    if (!skip_b) {
+                    if (gb) {
                         *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + (g * p.nb_atoms) * 512 + lane * 16) =
                             make_uint4(wb[0][0], wb[0][1], wb[0][2], wb[0][3]);
                         if (p.nb_atoms > 1)
                             *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + (g * p.nb_atoms + 1) * 512 + lane * 16) =
                                 make_uint4(wb[1][0], wb[1][1], wb[1][2], wb[1][3]);
                     }
+                  }
                 }
                 if (!ok) break;
                 if (KIND == kConv) kw.advance(KS * nsf, p.CB);
@@ -706,68 +761,79 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         uint32_t tcount = 0;
         for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
+            // output row of this thread in sub-tile i
             bool row_ok;
             int64_t row_off;
-            if (KIND == kConv) {
-                int aw, iq, ip, in;
-                conv_row(p, m, aw, iq, ip, in);
-                const int q = p.sub * (I.q0 + iq) + aw, pr = I.p0 + ip, n = I.n0 + in;
-                row_ok = m < p.sub * p.bq * p.bp * p.bn && q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
-                row_off = p.ph_out_base[I.ph] + n * p.os_n + pr * p.os_p + q * p.os_q;
-            } else {
-                const int k = I.m0 + m;
-                row_ok = k < p.Mrows;
-                row_off = p.out_base + I.split * p.split_pitch + k * p.os_m + (p.ntg == 1 ? p.taps[I.tap].btap : 0);
-            }
+            auto set_row = [&](int i) {
+                if (KIND == kConv) {
+                    int q0 = I.q0, p0 = I.p0, n0 = I.n0;
+                    if (i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
+                    int aw, iq, ip, in;
+                    conv_row(p, m, aw, iq, ip, in);
+                    const int q = p.sub * (q0 + iq) + aw, pr = p0 + ip, n = n0 + in;
+                    row_ok = m < p.sub * p.bq * p.bp * p.bn && q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
+                    row_off = p.ph_out_base[I.ph] + n * p.os_n + pr * p.os_p + q * p.os_q;
+                } else {
+                    const int k = I.m0 + m;
+                    row_ok = k < p.Mrows;
+                    row_off = p.out_base + I.split * p.split_pitch + k * p.os_m + (p.ntg == 1 ? p.taps[I.tap].btap : 0);
+                }
+            };
             const bool tap_cols = KIND == kWgrad && p.ntg > 1;   // columns are (tap, channel)
             if (I.nk == 0) {
-                if (row_ok)
-                    for (int n = 0; n < p.BN; ++n) {
-                        if (tap_cols) {
-                            const int t = static_cast<int>(p.fd_cpad.div(n)), c = n - t * p.cpad;
-                            if (t < I.tig && c < p.Ncols) p.out[row_off + c * p.os_c + p.taps[I.tap + t].btap] = 0.0f;
-                        } else if (I.col0 + n < p.Ncols) {
-                            p.out[row_off + (I.col0 + n) * p.os_c] = 0.0f;
+                for (int i = 0; i < UM; ++i) {
+                    set_row(i);
+                    if (row_ok)
+                        for (int n = 0; n < p.BN; ++n) {
+                            if (tap_cols) {
+                                const int t = static_cast<int>(p.fd_cpad.div(n)), c = n - t * p.cpad;
+                                if (t < I.tig && c < p.Ncols) p.out[row_off + c * p.os_c + p.taps[I.tap + t].btap] = 0.0f;
+                            } else if (I.col0 + n < p.Ncols) {
+                                p.out[row_off + (I.col0 + n) * p.os_c] = 0.0f;
+                            }
                         }
-                    }
+                }
                 continue;
             }
-            const uint32_t acc = tcount & 1u & static_cast<uint32_t>(p.nacc - 1);
-            const uint32_t aph = (p.nacc == 2 ? (tcount >> 1) : tcount) & 1u;
+            const uint32_t acc = tcount & static_cast<uint32_t>(p.nacc - 1);
+            const uint32_t aph = (tcount >> p.lg_nacc) & 1u;
             if (!mbar_wait(&acc_full[acc], aph, lim, abort_flag)) break;
             tc_fence_after();
-            const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16) + acc * p.BN;
-            float *orow = p.out + row_off;
-            // 32 columns at a time (one TMEM load, one wait); the accumulator
-            // is released after the last load, before its global stores, so
-            // the MMA issuer can start the next tile on it.  The loop body is
-            // kept small: it runs once per 32 columns of every tile, next to
-            // the code of the other roles.
-            for (int c0 = 0; c0 < p.BN; c0 += 32) {
-                uint32_t r[32];
-                tc_ld_32x32b_x32(t_row + c0, r);
-                tc_wait_ld();
-                if (c0 + 32 >= p.BN) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&acc_empty[acc]);
-                }
-                if (tap_cols) {
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int n = c0 + jj;
-                        const int t = static_cast<int>(p.fd_cpad.div(n)), c = n - t * p.cpad;
-                        if (row_ok && n < p.BN && t < I.tig && c < p.Ncols)
-                            orow[c * p.os_c + p.taps[I.tap + t].btap] = __uint_as_float(r[jj]);
+            // 32 columns at a time (one TMEM load, one wait); the accumulators
+            // are released after the last load of the last sub-tile, before
+            // its global stores, so the MMA issuer can start the next unit on
+            // them.  The loop body is kept small: it runs once per 32 columns
+            // of every sub-tile, next to the code of the other roles.
+            for (int i = 0; i < UM; ++i) {
+                set_row(i);
+                const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16) + (acc * UM + i) * p.BN;
+                float *orow = p.out + row_off;
+                for (int c0 = 0; c0 < p.BN; c0 += 32) {
+                    uint32_t r[32];
+                    tc_ld_32x32b_x32(t_row + c0, r);
+                    tc_wait_ld();
+                    if (i + 1 == UM && c0 + 32 >= p.BN) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc_empty[acc]);
                     }
-                    continue;
-                }
-                const int cb = I.col0 + c0;
-                const int nv = row_ok ? min(32, p.Ncols - cb) : 0;
-                float *op = orow + static_cast<int64_t>(cb) * p.os_c;
+                    if (tap_cols) {
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj)
-                    if (jj < nv) op[jj * p.os_c] = __uint_as_float(r[jj]);
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int n = c0 + jj;
+                            const int t = static_cast<int>(p.fd_cpad.div(n)), c = n - t * p.cpad;
+                            if (row_ok && n < p.BN && t < I.tig && c < p.Ncols)
+                                orow[c * p.os_c + p.taps[I.tap + t].btap] = __uint_as_float(r[jj]);
+                        }
+                        continue;
+                    }
+                    const int cb = I.col0 + c0;
+                    const int nv = row_ok ? min(32, p.Ncols - cb) : 0;
+                    float *op = orow + static_cast<int64_t>(cb) * p.os_c;
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        if (jj < nv) op[jj * p.os_c] = __uint_as_float(r[jj]);
+                }
             }
             ++tcount;
         }

@@ -86,7 +86,7 @@ int conv_Q(const mqc_conv *c) { return (c->W + 2 * c->pad_w - c->S) / c->stride_
 struct DevInfo {
     int sms = 0;
     int max_smem = 0;
-    bool gemm_attr[4] = {false, false, false, false};   // [KIND * 2 + SFV4]
+    bool gemm_attr[7] = {};   // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind
     bool quant_attr[24] = {};                             // staged quantizer, [(fmt*3 + blk)*4 + tile]
 };
 std::mutex g_dev_mu;
@@ -232,10 +232,31 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     // the 32-bit scale path reads B four bytes at a time unless B is cached
     if (!P.sfb_cached && !P.sfb_vec4) P.sf_vec4 = 0;
     const int fixed = 1024 + 64 * 8 + 64 + (P.sfb_cached ? cache : 0);
+    // CONV with few K-blocks per tile and narrow column tiles: units of
+    // um = 2 or 4 row tiles, so that the per-unit work of every role (decode,
+    // barrier round trips, B loads, scale atoms of B) is shared by um MMAs;
+    // only while there are still at least two units per SM.  Measured on the
+    // YOLOv8n layers: a gain up to 9 K-blocks and 32 columns, a loss with 12
+    // K-blocks (the scale gather redoes the rows of every sub-tile per stage)
+    // or 64 columns.
+    P.um = 1;
+    if (KIND == kConv) {
+        P.MTILES = P.TQ * P.TP * P.TN;
+        if (P.total_kb <= 9 && P.BN <= 32) {
+            for (int um = 4; um >= 2; um /= 2) {
+                const int64_t units = ceil_div(P.MTILES, um) * int64_t(P.nph) * P.NT;
+                if (2 * um * P.BN <= 256 && units >= 2 * d.sms) {
+                    P.um = um;
+                    break;
+                }
+            }
+        }
+        P.num_units = static_cast<int32_t>(ceil_div(P.MTILES, P.um) * int64_t(P.nph) * P.NT);
+    }
     auto stages_for = [&](int kbs, int &S) {
         const int ga = kbs / 4;
-        const int per_stage = 128 * 32 * kbs + P.BN * 32 * kbs + 512 * ga + 512 * ga * P.nb_atoms;
-        const int sf_cols = ga * (4 + 4 * P.nb_atoms);
+        const int per_stage = P.um * 128 * 32 * kbs + P.BN * 32 * kbs + 512 * ga * P.um + 512 * ga * P.nb_atoms;
+        const int sf_cols = ga * (4 * P.um + 4 * P.nb_atoms);
         S = std::min(8, (d.max_smem - fixed) / per_stage);
         S = std::min(S, (kTmemCols - kSfTmemBase) / sf_cols);
         return per_stage;
@@ -245,7 +266,7 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     int S8 = 0, S4 = 0;
     const int ps8 = stages_for(8, S8), ps4 = stages_for(4, S4);
     const bool long_k = KIND == kConv ? P.total_kb > 4 : P.kiters_total > 1;
-    P.kbs = (long_k && S8 >= 3) ? 8 : 4;
+    P.kbs = (long_k && S8 >= 3 && P.um == 1) ? 8 : 4;
     const int S = P.kbs == 8 ? S8 : S4;
     const int per_stage = P.kbs == 8 ? ps8 : ps4;
     if (S < 3) return fail(MQC_ERR_UNSUPPORTED, "tile does not fit in shared memory");
@@ -265,12 +286,21 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     P.fd_splits = make_fastdiv(P.splits);
     if (KIND == kWgrad && int64_t(P.kiters_total) * (P.splits + 1) >= (1ll << 31))
         return fail(MQC_ERR_UNSUPPORTED, "weight gradient: reduction too long");
-    P.nacc = (P.BN <= 128) ? 2 : 1;
+    // accumulators in TMEM columns [0, 256): as many as fit, up to 4, so that
+    // several tiles can wait between the MMA issuer and the epilogue
+    const int acc_cols = P.um * P.BN;   // TMEM columns of one unit's accumulators
+    P.nacc = acc_cols <= 64 ? 4 : (acc_cols <= 128 ? 2 : 1);
+    P.lg_nacc = P.nacc == 4 ? 2 : (P.nacc == 2 ? 1 : 0);
     P.timeout_ns = kDefaultTimeoutNs;
     const int smem = fixed + S * per_stage;
     const bool v4 = KIND == kConv && P.sf_vec4;
-    auto kernel = v4 ? conv_gemm_kernel<KIND, true> : conv_gemm_kernel<KIND, false>;
-    const int ai = KIND * 2 + (v4 ? 1 : 0);
+    auto kernel = conv_gemm_kernel<kWgrad, false, 1>;
+    if (KIND == kConv) {
+        if (P.um == 4) kernel = v4 ? conv_gemm_kernel<kConv, true, 4> : conv_gemm_kernel<kConv, false, 4>;
+        else if (P.um == 2) kernel = v4 ? conv_gemm_kernel<kConv, true, 2> : conv_gemm_kernel<kConv, false, 2>;
+        else kernel = v4 ? conv_gemm_kernel<kConv, true, 1> : conv_gemm_kernel<kConv, false, 1>;
+    }
+    const int ai = KIND == kConv ? 1 + (v4 ? 3 : 0) + (P.um == 4 ? 2 : P.um - 1) : 0;
     if (!d.gemm_attr[ai]) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.max_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");

@@ -217,8 +217,18 @@ class LayerBuffers:
         self.y = torch.empty((L.N, L.K, L.P, L.Q), dtype=torch.float32, device=dev)
         self.gx = torch.empty((L.N, L.C, L.H, L.W), dtype=torch.float32, device=dev)
         self.gw = torch.empty((L.K, L.C, L.R, L.S), dtype=torch.float32, device=dev)
-        self.ws_bytes = mqc.conv2d_bwd_weight_workspace_bytes(self.cv, self.q["g"].other_order().mx,
-                                                              self.q["x"].other_order().mx)
+        qx, qw, qg = self.q["x"], self.q["w"], self.q["g"]
+        self.ws_fwd = mqc.mqc_conv2d_fwd_workspace_bytes(self.cv, qx.mx, qw.mx)
+        self.ws_dgrad = mqc.mqc_conv2d_bwd_data_workspace_bytes(self.cv, qw.other_order().mx, qg.mx)
+        self.ws_wgrad = mqc.conv2d_bwd_weight_workspace_bytes(self.cv, qg.other_order().mx, qx.other_order().mx)
+        # E2M1 operands are widened to E4M3 codes inside each GEMM call (one
+        # launch per widened operand); the weight gradient reduces split-K
+        # partials when its workspace holds more than the widened copies
+        widen = {k: (2 * self.q[k].codes.numel() + 255) // 256 * 256 if self.q[k].mx.fmt == mqc.E2M1 else 0
+                 for k in ("x", "w", "g")}
+        self.n_widen = 2 * sum(1 for v in widen.values() if v)
+        self.split_k = self.ws_wgrad > widen["g"] + widen["x"]
+        self.ws_bytes = max(self.ws_fwd, self.ws_dgrad, self.ws_wgrad)
         self.host_out = None
         if want_host:
             self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (self.y, self.gx, self.gw)]
@@ -246,7 +256,7 @@ class LayerBuffers:
         up to 4 height phases), the weight-gradient GEMM and, with split-K
         partials, their reduction."""
         L = self.L
-        return 3 + 1 + -(-L.stride // 4) + (2 if self.ws_bytes > 0 else 1)
+        return 3 + 1 + -(-L.stride // 4) + (2 if self.split_k else 1) + self.n_widen
 
 
 def run_layer(mqc, lb: LayerBuffers, workspace, stream, events=None, only=None):
@@ -275,13 +285,14 @@ def run_layer(mqc, lb: LayerBuffers, workspace, stream, events=None, only=None):
             P(t), lb.desc[name], q.mx, P(q.codes), P(q.scales), P(q.codes_alt), stream))
     qx, qw, qg = lb.q["x"], lb.q["w"], lb.q["g"]
     wq_ab, gq_ab, xq_ab = qw.other_order(), qg.other_order(), qx.other_order()
+    wsp = P(workspace) if lb.ws_bytes else None
     timed("fwd", lambda: mqc.mqc_conv2d_fwd(P(qx.codes), P(qx.scales), qx.mx, P(qw.codes), P(qw.scales), qw.mx,
-                                            lb.cv, P(lb.y), stream))
+                                            lb.cv, P(lb.y), wsp, lb.ws_fwd, stream))
     timed("dgrad", lambda: mqc.mqc_conv2d_bwd_data(P(wq_ab.codes), P(wq_ab.scales), wq_ab.mx, P(qg.codes),
-                                                   P(qg.scales), qg.mx, lb.cv, P(lb.gx), stream))
+                                                   P(qg.scales), qg.mx, lb.cv, P(lb.gx), wsp, lb.ws_dgrad, stream))
     timed("wgrad", lambda: mqc.mqc_conv2d_bwd_weight(P(gq_ab.codes), P(gq_ab.scales), gq_ab.mx, P(xq_ab.codes),
                                                      P(xq_ab.scales), xq_ab.mx, lb.cv, P(lb.gw),
-                                                     P(workspace) if lb.ws_bytes else None, lb.ws_bytes, stream))
+                                                     wsp, lb.ws_wgrad, stream))
 
 
 # --------------------------------------------------------------------------- CPU oracle

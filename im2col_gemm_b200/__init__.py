@@ -32,7 +32,7 @@ EXPORTS = ("mqc_codes_bytes", "mqc_scales_bytes", "mqc_tensor_dims", "mqc_quanti
            "mqc_im2col_cbf_scales_bytes", "mqc_im2col_cbf_codes_bytes", "mqc_conv2d_fwd", "mqc_conv2d_bwd_data",
            "mqc_conv2d_bwd_weight", "mqc_conv2d_bwd_weight_workspace_bytes", "mqc_get_device_status",
            "mqc_debug_expire_wait", "mqc_status_string", "mqc_last_error_message", "mqc_version",
-           "mqc_conv2d_bwd_weight_noalloc")
+           "mqc_conv2d_bwd_weight_noalloc", "mqc_conv2d_fwd_workspace_bytes", "mqc_conv2d_bwd_data_workspace_bytes")
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -71,8 +71,10 @@ def _load() -> ctypes.CDLL:
         "mqc_im2col_cbf": (i32, [vp, vp, P(Conv), P(MX), vp, vp, vp]),
         "mqc_im2col_cbf_scales_bytes": (i64, [P(Conv), P(MX)]),
         "mqc_im2col_cbf_codes_bytes": (i64, [P(Conv), P(MX)]),
-        "mqc_conv2d_fwd": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp]),
-        "mqc_conv2d_bwd_data": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp]),
+        "mqc_conv2d_fwd": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp, sz, vp]),
+        "mqc_conv2d_fwd_workspace_bytes": (sz, [P(Conv), P(MX), P(MX)]),
+        "mqc_conv2d_bwd_data": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp, sz, vp]),
+        "mqc_conv2d_bwd_data_workspace_bytes": (sz, [P(Conv), P(MX), P(MX)]),
         "mqc_conv2d_bwd_weight": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp, sz, vp]),
         "mqc_conv2d_bwd_weight_workspace_bytes": (sz, [P(Conv), P(MX), P(MX)]),
         "mqc_conv2d_bwd_weight_noalloc": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp]),
@@ -116,13 +118,22 @@ def mqc_im2col_cbf(codes_ptr, scales_ptr, conv: Conv, mx: MX, codes_out_ptr, sca
                               scales_out_ptr, stream)
 
 
-def mqc_conv2d_fwd(xq, xs, xf: MX, wq, ws, wf: MX, conv: Conv, y, stream) -> int:
-    return lib.mqc_conv2d_fwd(xq, xs, ctypes.byref(xf), wq, ws, ctypes.byref(wf), ctypes.byref(conv), y, stream)
+def mqc_conv2d_fwd(xq, xs, xf: MX, wq, ws, wf: MX, conv: Conv, y, workspace, workspace_bytes, stream) -> int:
+    return lib.mqc_conv2d_fwd(xq, xs, ctypes.byref(xf), wq, ws, ctypes.byref(wf), ctypes.byref(conv), y, workspace,
+                              workspace_bytes, stream)
 
 
-def mqc_conv2d_bwd_data(wq, ws, wf: MX, gq, gs, gf: MX, conv: Conv, gx, stream) -> int:
+def mqc_conv2d_fwd_workspace_bytes(conv: Conv, xf: MX, wf: MX) -> int:
+    return lib.mqc_conv2d_fwd_workspace_bytes(ctypes.byref(conv), ctypes.byref(xf), ctypes.byref(wf))
+
+
+def mqc_conv2d_bwd_data(wq, ws, wf: MX, gq, gs, gf: MX, conv: Conv, gx, workspace, workspace_bytes, stream) -> int:
     return lib.mqc_conv2d_bwd_data(wq, ws, ctypes.byref(wf), gq, gs, ctypes.byref(gf), ctypes.byref(conv), gx,
-                                   stream)
+                                   workspace, workspace_bytes, stream)
+
+
+def mqc_conv2d_bwd_data_workspace_bytes(conv: Conv, wf: MX, gf: MX) -> int:
+    return lib.mqc_conv2d_bwd_data_workspace_bytes(ctypes.byref(conv), ctypes.byref(wf), ctypes.byref(gf))
 
 
 def mqc_conv2d_bwd_weight(gq, gs, gf: MX, xq, xs, xf: MX, conv: Conv, gw, workspace, workspace_bytes,
@@ -229,21 +240,27 @@ def im2col_cbf(xq: Quantized, cv: Conv):
     return co, so
 
 
-def conv2d_fwd(xq: Quantized, wq: Quantized, cv: Conv, out=None):
+def conv2d_fwd(xq: Quantized, wq: Quantized, cv: Conv, out=None, workspace=None):
     torch = _torch()
     P, Q = conv_out_hw(cv)
     y = out if out is not None else torch.empty((cv.N, cv.K, P, Q), dtype=torch.float32, device=xq.codes.device)
+    nws = mqc_conv2d_fwd_workspace_bytes(cv, xq.mx, wq.mx)
+    if workspace is None and nws > 0:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=xq.codes.device)
     check(mqc_conv2d_fwd(_ptr(xq.codes), _ptr(xq.scales), xq.mx, _ptr(wq.codes), _ptr(wq.scales), wq.mx, cv,
-                         _ptr(y), _stream()))
+                         _ptr(y), _ptr(workspace), nws, _stream()))
     return y
 
 
-def conv2d_bwd_data(wq: Quantized, gq: Quantized, cv: Conv, out=None):
+def conv2d_bwd_data(wq: Quantized, gq: Quantized, cv: Conv, out=None, workspace=None):
     torch = _torch()
     gx = out if out is not None else torch.empty((cv.N, cv.C, cv.H, cv.W), dtype=torch.float32,
                                                  device=gq.codes.device)
+    nws = mqc_conv2d_bwd_data_workspace_bytes(cv, wq.mx, gq.mx)
+    if workspace is None and nws > 0:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=gq.codes.device)
     check(mqc_conv2d_bwd_data(_ptr(wq.codes), _ptr(wq.scales), wq.mx, _ptr(gq.codes), _ptr(gq.scales), gq.mx, cv,
-                              _ptr(gx), _stream()))
+                              _ptr(gx), _ptr(workspace), nws, _stream()))
     return gx
 
 

@@ -17,6 +17,7 @@
 #include "conv_gemm.cuh"
 #include "im2col.cuh"
 #include "quantize.cuh"
+#include "widen.cuh"
 
 using namespace mqc;
 
@@ -87,7 +88,7 @@ struct DevInfo {
     int sms = 0;
     int max_smem = 0;
     bool gemm_attr[7] = {};   // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind
-    bool quant_attr[24] = {};                             // staged quantizer, [(fmt*3 + blk)*4 + tile]
+    bool quant_attr[36] = {};                             // staged quantizer, [(fmt*3 + blk)*4 + tile]
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
@@ -319,13 +320,62 @@ void split_tap(int off, int st, int &d, int &ph) {
     d = (off - ph) / st;
 }
 
-bool gemm_fmt_ok(const mqc_mx *m) { return m->fmt == MQC_E4M3 || m->fmt == MQC_E5M2; }
+bool gemm_fmt_ok(const mqc_mx *m) { return m->fmt == MQC_E4M3 || m->fmt == MQC_E5M2 || m->fmt == MQC_E2M1; }
+
+// A GEMM operand as the kernel reads it: FP8 codes as given; E2M1 codes
+// rewritten as the E4M3 codes of the same values into the workspace (same
+// layout, one byte per element), so the tensor core runs every format
+// through kind::mxf8f6f4 with unchanged E8M0 scales.
+struct GemmOperand {
+    const uint8_t *codes;
+    int mma_fmt;       // element format the MMA reads (E4M3 or E5M2)
+    int64_t inner;     // padded innermost extent: elements = bytes of one row
+};
+
+// Workspace bytes of the widened copy of an operand [d0=B][d1=A][d2][d3].
+size_t widened_bytes(const mqc_mx *m, int64_t d0, int64_t d1, int64_t d2, int64_t d3) {
+    if (m->fmt != MQC_E2M1) return 0;
+    return static_cast<size_t>(round_up(2 * codes_bytes(MQC_E2M1, m->order, d0, d1, d2, d3), 256));
+}
+
+mqc_status check_workspace(const char *name, const void *ws, size_t bytes, size_t need) {
+    if (need == 0) return MQC_OK;
+    if (ws == nullptr || bytes < need) return fail(MQC_ERR_WORKSPACE, "%s: needs %zu workspace bytes", name, need);
+    if (!aligned16(ws)) return fail(MQC_ERR_ALIGNMENT, "%s: workspace not 16-byte aligned", name);
+    return MQC_OK;
+}
+
+// Fills o for the operand [d0][d1][d2][d3] with codes q; an E2M1 operand is
+// widened into *wsp, which then advances past the copy.
+mqc_status gemm_operand(const void *q, const mqc_mx *m, int64_t d0, int64_t d1, int64_t d2, int64_t d3, uint8_t *&wsp,
+                        cudaStream_t s, GemmOperand &o) {
+    int64_t Ap, Bp;
+    padded(m->fmt, m->order, d1, d0, Ap, Bp);
+    o.inner = m->order == MQC_ORDER_BA ? Ap : Bp;
+    if (m->fmt != MQC_E2M1) {
+        o.codes = static_cast<const uint8_t *>(q);
+        o.mma_fmt = m->fmt;
+        return MQC_OK;
+    }
+    const int64_t nb = codes_bytes(MQC_E2M1, m->order, d0, d1, d2, d3);   // a multiple of 16 (16-byte rows)
+    const int64_t chunks = nb / 16;
+    if (chunks > 0) {
+        const int blocks = static_cast<int>(std::min<int64_t>(ceil_div(chunks, 256), 148 * 16));
+        widen_e2m1_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint8_t *>(q), wsp, chunks);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "widen_e2m1_kernel launch");
+    }
+    o.codes = wsp;
+    o.mma_fmt = MQC_E4M3;
+    wsp += widened_bytes(m, d0, d1, d2, d3);
+    return MQC_OK;
+}
 
 mqc_status check_gemm_operand(const char *name, const void *q, const uint8_t *s, const mqc_mx *m, int want_order,
                               bool along_first) {
     if (q == nullptr || s == nullptr || !mx_ok(m)) return fail(MQC_ERR_INVALID, "%s: null pointer or bad mx", name);
     if (!aligned16(q)) return fail(MQC_ERR_ALIGNMENT, "%s codes not 16-byte aligned", name);
-    if (!gemm_fmt_ok(m)) return fail(MQC_ERR_UNSUPPORTED, "%s: only E4M3/E5M2 operands in the GEMMs of this build", name);
+    if (!gemm_fmt_ok(m)) return fail(MQC_ERR_UNSUPPORTED, "%s: unknown element format", name);
     if (m->order != want_order)
         return fail(MQC_ERR_UNSUPPORTED, "%s: code order must be %s", name, want_order == 0 ? "BA" : "AB");
     const int want_block = along_first ? MQC_BLOCK_A32 : MQC_BLOCK_B32;
@@ -434,11 +484,11 @@ mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, 
     const bool dual = codes_alt != nullptr;
     // staged kernel: FP8, positions contiguous (element stride 1 along W,
     // W along H), every plane 16-byte aligned
-    if (!fp4 && d->s3 == 1 && d->s2 == d->d3 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && d->s0 % 4 == 0 &&
+    if (d->s3 == 1 && d->s2 == d->d3 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && d->s0 % 4 == 0 &&
         d->s1 % 4 == 0) {
         StagedParams sp{};
         sp.q = p;
-        sp.IT = p.I1 <= 16 ? 16 : 32;
+        sp.IT = (!fp4 && p.I1 <= 16) ? 16 : 32;     // FP4 rows are 32 codes
         sp.OT = (dual ? std::max(p.O, p.O2) : p.O) <= 16 ? 16 : 32;
         sp.PT = kStagedTileBytes / (4 * sp.OT * sp.IT);
         sp.nPT = static_cast<int32_t>(ceil_div(p.npix, sp.PT));
@@ -453,7 +503,8 @@ mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, 
         const int ai = (p.fmt * 3 + blk) * 4 + (sp.OT == 32 ? 2 : 0) + (sp.IT == 32 ? 1 : 0);
         cudaError_t ae = cudaSuccess;
         if (p.fmt == MQC_E4M3) launch_staged<0>(sp, static_cast<unsigned>(ntiles), smem, s, ae, !dv->quant_attr[ai]);
-        else launch_staged<1>(sp, static_cast<unsigned>(ntiles), smem, s, ae, !dv->quant_attr[ai]);
+        else if (p.fmt == MQC_E5M2) launch_staged<1>(sp, static_cast<unsigned>(ntiles), smem, s, ae, !dv->quant_attr[ai]);
+        else launch_staged<2>(sp, static_cast<unsigned>(ntiles), smem, s, ae, !dv->quant_attr[ai]);
         if (ae != cudaSuccess) return cuda_fail(ae, "cudaFuncSetAttribute");
         dv->quant_attr[ai] = true;
         cudaError_t e = cudaGetLastError();
@@ -547,8 +598,14 @@ mqc_status mqc_im2col_cbf(const void *codes, const uint8_t *scales, const mqc_co
 }
 
 // ------------------------------------------------------------------ forward
+size_t mqc_conv2d_fwd_workspace_bytes(const mqc_conv *c, const mqc_mx *xf, const mqc_mx *wf) {
+    if (!conv_ok(c) || !mx_ok(xf) || !mx_ok(wf)) return 0;
+    return widened_bytes(xf, c->N, c->C, c->H, c->W) + widened_bytes(wf, c->K, c->C, c->R, c->S);
+}
+
 mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, const void *wq, const uint8_t *ws,
-                          const mqc_mx *wf, const mqc_conv *c, float *y, void *stream) {
+                          const mqc_mx *wf, const mqc_conv *c, float *y, void *workspace, size_t workspace_bytes,
+                          void *stream) {
     if (!conv_ok(c) || y == nullptr) return fail(MQC_ERR_INVALID, "conv2d_fwd: bad conv descriptor or null output");
     mqc_status st = check_gemm_operand("X", xq, xs, xf, MQC_ORDER_BA, true);
     if (st != MQC_OK) return st;
@@ -560,7 +617,14 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
 
     const int N = c->N, C = c->C, H = c->H, W = c->W, K = c->K, R = c->R, S = c->S;
     const int sh = c->stride_h, sw = c->stride_w, P = conv_P(c), Q = conv_Q(c);
-    const int64_t Cp = round_up(C, 16);
+    if ((st = check_workspace("conv2d_fwd", workspace, workspace_bytes, mqc_conv2d_fwd_workspace_bytes(c, xf, wf))) !=
+        MQC_OK)
+        return st;
+    uint8_t *wsp = static_cast<uint8_t *>(workspace);
+    GemmOperand ox, ow;
+    if ((st = gemm_operand(xq, xf, N, C, H, W, wsp, static_cast<cudaStream_t>(stream), ox)) != MQC_OK) return st;
+    if ((st = gemm_operand(wq, wf, K, C, R, S, wsp, static_cast<cudaStream_t>(stream), ow)) != MQC_OK) return st;
+    const int64_t Cp = ox.inner, Cpw = ow.inner;   // padded channel extents of X and W rows
     GemmParams G;
     memset(&G, 0, sizeof G);
     G.CB = static_cast<int32_t>(nb32(Cp));
@@ -576,7 +640,7 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     G.Ncols = K;
     G.a_st_h = sh;
     G.a_st_w = sw;
-    G.idesc = make_idesc_mx(mma_fmt(xf->fmt), mma_fmt(wf->fmt), 128, G.BN);
+    G.idesc = make_idesc_mx(mma_fmt(ox.mma_fmt), mma_fmt(ow.mma_fmt), 128, G.BN);
     if (sh * sw > 4) return fail(MQC_ERR_UNSUPPORTED, "conv2d_fwd: stride product above 4");
     // A: one map per stride phase; dims (C, W', H', N) so that rows run along q
     bool phase_ok[16] = {};
@@ -588,7 +652,7 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
                 const int64_t Hh = ceil_div(H - a, sh), Ww = ceil_div(W - b, sw);
                 phase_ok[a * sw + b] = Hh > 0 && Ww > 0;
                 if (!phase_ok[a * sw + b]) continue;
-                const uint8_t *base = static_cast<const uint8_t *>(xq) + (int64_t(a) * W + b) * N * Cp;
+                const uint8_t *base = ox.codes + (int64_t(a) * W + b) * N * Cp;
                 if (!G.rows_nfirst) {
                     const uint64_t dims[4] = {uint64_t(Cp), uint64_t(Ww), uint64_t(Hh), uint64_t(N)};
                     const uint64_t strd[3] = {uint64_t(sw) * N * Cp, uint64_t(sh) * W * N * Cp, uint64_t(Cp)};
@@ -605,10 +669,10 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     }
     if (st != MQC_OK) return st;
     {
-        const uint64_t dims[3] = {uint64_t(Cp), uint64_t(K), uint64_t(R) * S};
-        const uint64_t strd[2] = {uint64_t(Cp), uint64_t(K) * Cp};
+        const uint64_t dims[3] = {uint64_t(Cpw), uint64_t(K), uint64_t(R) * S};
+        const uint64_t strd[2] = {uint64_t(Cpw), uint64_t(K) * Cpw};
         const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(box_rows(K, G.BN)), 1u};
-        if ((st = encode_codes_map(&G.bmap[0], wq, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
+        if ((st = encode_codes_map(&G.bmap[0], ow.codes, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
     }
     G.ntaps = 0;
     for (int r = 0; r < R; ++r)
@@ -673,8 +737,14 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
 }
 
 // ------------------------------------------------------------------ input gradient
+size_t mqc_conv2d_bwd_data_workspace_bytes(const mqc_conv *c, const mqc_mx *wf, const mqc_mx *gf) {
+    if (!conv_ok(c) || !mx_ok(wf) || !mx_ok(gf)) return 0;
+    return widened_bytes(wf, c->K, c->C, c->R, c->S) + widened_bytes(gf, c->N, c->K, conv_P(c), conv_Q(c));
+}
+
 mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *wf, const void *gq, const uint8_t *gs,
-                               const mqc_mx *gf, const mqc_conv *c, float *gx, void *stream) {
+                               const mqc_mx *gf, const mqc_conv *c, float *gx, void *workspace, size_t workspace_bytes,
+                               void *stream) {
     if (!conv_ok(c) || gx == nullptr) return fail(MQC_ERR_INVALID, "conv2d_bwd_data: bad conv descriptor or null output");
     mqc_status st = check_gemm_operand("W", wq, ws, wf, MQC_ORDER_AB, false);
     if (st != MQC_OK) return st;
@@ -685,7 +755,14 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
     if ((st = dev_info(dv)) != MQC_OK) return st;
     const int N = c->N, C = c->C, H = c->H, W = c->W, K = c->K, R = c->R, S = c->S;
     const int sh = c->stride_h, sw = c->stride_w, P = conv_P(c), Q = conv_Q(c);
-    const int64_t Kp = round_up(K, 16);
+    if ((st = check_workspace("conv2d_bwd_data", workspace, workspace_bytes,
+                              mqc_conv2d_bwd_data_workspace_bytes(c, wf, gf))) != MQC_OK)
+        return st;
+    uint8_t *wsp = static_cast<uint8_t *>(workspace);
+    GemmOperand ow, og;
+    if ((st = gemm_operand(wq, wf, K, C, R, S, wsp, static_cast<cudaStream_t>(stream), ow)) != MQC_OK) return st;
+    if ((st = gemm_operand(gq, gf, N, K, P, Q, wsp, static_cast<cudaStream_t>(stream), og)) != MQC_OK) return st;
+    const int64_t Kp = og.inner, Kpw = ow.inner;   // padded output-channel extents of G_Y and W rows
     const bool sqg = gf->block == MQC_BLOCK_SQ32, sqw = wf->block == MQC_BLOCK_SQ32;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     // output stride phases (ah, aw) with at least one row; the first one has
@@ -715,7 +792,7 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
         G.Ncols = C;
         G.a_st_h = 1;
         G.a_st_w = 1;
-        G.idesc = make_idesc_mx(mma_fmt(gf->fmt), mma_fmt(wf->fmt), 128, G.BN);
+        G.idesc = make_idesc_mx(mma_fmt(og.mma_fmt), mma_fmt(ow.mma_fmt), 128, G.BN);
         st = MQC_ERR_CUDA;
         if (sub > 1) {
             // (C, slot, q, p, n): the slot dimension has extent 1 and a box of
@@ -725,7 +802,7 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
             const uint64_t strd[4] = {uint64_t(Kp), uint64_t(N) * Kp, uint64_t(Q) * N * Kp, uint64_t(Kp)};
             const uint32_t box[5] = {uint32_t(32 * G.wkb), uint32_t(sub), uint32_t(G.bq), uint32_t(G.bp),
                                      uint32_t(G.bn)};
-            st = encode_codes_map(&G.amap[0], gq, 5, dims, strd, box, G.wkb);
+            st = encode_codes_map(&G.amap[0], og.codes, 5, dims, strd, box, G.wkb);
         } else {
             for (int attempt = 0; attempt < 2 && st != MQC_OK; ++attempt) {
                 G.rows_nfirst = attempt;
@@ -733,21 +810,21 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
                     const uint64_t dims[4] = {uint64_t(Kp), uint64_t(Q), uint64_t(P), uint64_t(N)};
                     const uint64_t strd[3] = {uint64_t(N) * Kp, uint64_t(Q) * N * Kp, uint64_t(Kp)};
                     const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bq), uint32_t(G.bp), uint32_t(G.bn)};
-                    st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
+                    st = encode_codes_map(&G.amap[0], og.codes, 4, dims, strd, box, G.wkb);
                 } else {
                     const uint64_t dims[4] = {uint64_t(Kp), uint64_t(N), uint64_t(Q), uint64_t(P)};
                     const uint64_t strd[3] = {uint64_t(Kp), uint64_t(N) * Kp, uint64_t(Q) * N * Kp};
                     const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bn), uint32_t(G.bq), uint32_t(G.bp)};
-                    st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb);
+                    st = encode_codes_map(&G.amap[0], og.codes, 4, dims, strd, box, G.wkb);
                 }
             }
         }
         if (st != MQC_OK) return st;
         {
-            const uint64_t dims[3] = {uint64_t(Kp), uint64_t(C), uint64_t(R) * S};
-            const uint64_t strd[2] = {uint64_t(Kp), uint64_t(C) * Kp};
+            const uint64_t dims[3] = {uint64_t(Kpw), uint64_t(C), uint64_t(R) * S};
+            const uint64_t strd[2] = {uint64_t(Kpw), uint64_t(C) * Kpw};
             const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(box_rows(C, G.BN)), 1u};
-            if ((st = encode_codes_map(&G.bmap[0], wq, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
+            if ((st = encode_codes_map(&G.bmap[0], ow.codes, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
         }
         // taps of phase ah: kernel rows r with (ah + pad - r) divisible by sh,
         // every kernel column s; tap (r, s) feeds slot aw = (s - pad) mod sw
@@ -846,15 +923,20 @@ static WgradPlan wgrad_plan(const mqc_conv *c, const DevInfo &d) {
     return w;
 }
 
+// Split-K partial sums (when the reduction is split) at the start of the
+// workspace, then the widened copies of E2M1 operands.
+static size_t wgrad_partial_bytes(const mqc_conv *c, const WgradPlan &w) {
+    if (w.splits <= 1) return 0;
+    return static_cast<size_t>(round_up(int64_t(w.splits) * c->K * c->C * c->R * c->S * int64_t(sizeof(float)), 256));
+}
+
 size_t mqc_conv2d_bwd_weight_workspace_bytes(const mqc_conv *c, const mqc_mx *gf, const mqc_mx *xf) {
-    (void)gf;
-    (void)xf;
-    if (!conv_ok(c)) return 0;
+    if (!conv_ok(c) || !mx_ok(gf) || !mx_ok(xf)) return 0;
     DevInfo *dv;
     if (dev_info(dv) != MQC_OK) return 0;
     const WgradPlan w = wgrad_plan(c, *dv);
-    if (w.splits <= 1) return 0;
-    return size_t(w.splits) * size_t(c->K) * c->C * c->R * c->S * sizeof(float);
+    return wgrad_partial_bytes(c, w) + widened_bytes(gf, c->N, c->K, conv_P(c), conv_Q(c)) +
+           widened_bytes(xf, c->N, c->C, c->H, c->W);
 }
 
 mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx *gf, const void *xq,
@@ -870,7 +952,6 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     if ((st = dev_info(dv)) != MQC_OK) return st;
     const int N = c->N, C = c->C, H = c->H, W = c->W, K = c->K, R = c->R, S = c->S;
     const int sh = c->stride_h, sw = c->stride_w, P = conv_P(c), Q = conv_Q(c);
-    const int64_t Np = round_up(N, 16);
     GemmParams G;
     memset(&G, 0, sizeof G);
     if (sh * sw > 4) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_weight: stride product above 4");
@@ -881,10 +962,14 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     G.ntg = plan.ntg;
     G.ngroups = plan.ngroups;
     G.cpad = plan.cpad;
-    const size_t need = G.splits > 1 ? size_t(G.splits) * K * C * R * S * sizeof(float) : 0;
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
-        return fail(MQC_ERR_WORKSPACE, "conv2d_bwd_weight: needs %zu workspace bytes", need);
-    if (need > 0 && !aligned16(workspace)) return fail(MQC_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+    if ((st = check_workspace("conv2d_bwd_weight", workspace, workspace_bytes,
+                              mqc_conv2d_bwd_weight_workspace_bytes(c, gf, xf))) != MQC_OK)
+        return st;
+    uint8_t *wsp = static_cast<uint8_t *>(workspace) + wgrad_partial_bytes(c, plan);
+    GemmOperand og, ox;
+    if ((st = gemm_operand(gq, gf, N, K, P, Q, wsp, static_cast<cudaStream_t>(stream), og)) != MQC_OK) return st;
+    if ((st = gemm_operand(xq, xf, N, C, H, W, wsp, static_cast<cudaStream_t>(stream), ox)) != MQC_OK) return st;
+    const int64_t Np = og.inner, Npx = ox.inner;   // padded batch extents of G_Y and X rows
     const int64_t NB = nb32(Np);
     G.wkb = largest_wkb(NB);
     G.bqk = 4 / G.wkb;
@@ -900,12 +985,12 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     G.Ncols = C;
     G.x_st_h = sh;
     G.x_st_w = sw;
-    G.idesc = make_idesc_mx(mma_fmt(gf->fmt), mma_fmt(xf->fmt), 128, G.BN);
+    G.idesc = make_idesc_mx(mma_fmt(og.mma_fmt), mma_fmt(ox.mma_fmt), 128, G.BN);
     {
         const uint64_t dims[4] = {uint64_t(Np), uint64_t(K), uint64_t(Q), uint64_t(P)};
         const uint64_t strd[3] = {uint64_t(Np), uint64_t(K) * Np, uint64_t(Q) * K * Np};
         const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(box_rows(K, 128)), uint32_t(G.bqk), 1u};
-        if ((st = encode_codes_map(&G.amap[0], gq, 4, dims, strd, box, G.wkb)) != MQC_OK) return st;
+        if ((st = encode_codes_map(&G.amap[0], og.codes, 4, dims, strd, box, G.wkb)) != MQC_OK) return st;
     }
     bool phase_ok[16] = {};
     for (int a = 0; a < sh; ++a)
@@ -913,9 +998,9 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
             const int64_t Hh = ceil_div(H - a, sh), Ww = ceil_div(W - b, sw);
             phase_ok[a * sw + b] = Hh > 0 && Ww > 0;
             if (!phase_ok[a * sw + b]) continue;
-            const uint8_t *base = static_cast<const uint8_t *>(xq) + (int64_t(a) * W + b) * C * Np;
-            const uint64_t dims[4] = {uint64_t(Np), uint64_t(C), uint64_t(Ww), uint64_t(Hh)};
-            const uint64_t strd[3] = {uint64_t(Np), uint64_t(sw) * C * Np, uint64_t(sh) * W * C * Np};
+            const uint8_t *base = ox.codes + (int64_t(a) * W + b) * C * Npx;
+            const uint64_t dims[4] = {uint64_t(Npx), uint64_t(C), uint64_t(Ww), uint64_t(Hh)};
+            const uint64_t strd[3] = {uint64_t(Npx), uint64_t(sw) * C * Npx, uint64_t(sh) * W * C * Npx};
             // one tap: a box over the kit's bqk pixels; tap groups: one pixel
             // of one tap per box (cpad rows), placed at that tap's rows
             const uint32_t box[4] = {uint32_t(32 * G.wkb),

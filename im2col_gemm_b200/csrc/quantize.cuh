@@ -353,6 +353,28 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+// Four codes of v[0..3] (element k of the group in code position k): 32
+// bits for FP8, 16 bits (nibbles, low first) for FP4.
+template <int FMT>
+__device__ __forceinline__ uint32_t pack4(const float (&v)[4]) {
+    if (FMT == 2) return cvt_pair<FMT>(v[0], v[1]) | (cvt_pair<FMT>(v[2], v[3]) << 8);
+    return cvt_pair<FMT>(v[0], v[1]) | (cvt_pair<FMT>(v[2], v[3]) << 16);
+}
+
+// Stores the packed codes of one row of 16 or 32 codes: h[q] holds codes
+// 4q..4q+3 as pack4 gives them; `bytes` = 16 or 32 (FP8) or 16 (FP4, 32 codes).
+template <int FMT, int NQ>
+__device__ __forceinline__ void store_row(uint8_t *dst, const uint32_t (&h)[NQ], int bytes) {
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+    if (FMT == 2) {
+        d[0] = make_uint4(h[0] | (h[1 % NQ] << 16), h[2 % NQ] | (h[3 % NQ] << 16), h[4 % NQ] | (h[5 % NQ] << 16),
+                          h[6 % NQ] | (h[7 % NQ] << 16));
+        return;
+    }
+    d[0] = make_uint4(h[0], h[1 % NQ], h[2 % NQ], h[3 % NQ]);
+    if (NQ == 8 && bytes == 32) d[1] = make_uint4(h[4 % NQ], h[5 % NQ], h[6 % NQ], h[7 % NQ]);
+}
+
 // OT, IT: tile extents (16 or 32); PT = positions per tile; NS = threads per
 // position.  A thread owns o-rows {sub, sub + NS, ...} in the primary pass and
 // i-columns {sub, sub + NS, ...} in the second-order pass (64 values each).
@@ -473,18 +495,17 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
             const int o = sub + NS * r;
             if (o0 + o >= p.O) break;
             const float inv_row = BLK == kAlongI ? s_inv[o * PT + pos] : inv_sq;
-            uint32_t w[IT / 4];
+            uint32_t h[IT / 4];
 #pragma unroll
             for (int q = 0; q < IT / 4; ++q) {
                 float v[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     v[k] = tp[(o * IT + 4 * q + k) * PT] * (BLK == kAlongO ? inv_i[(4 * q + k) % (BLK == kAlongO ? IT : 1)] : inv_row);
-                w[q] = cvt_pair<FMT>(v[0], v[1]) | (cvt_pair<FMT>(v[2], v[3]) << 16);
+                h[q] = pack4<FMT>(v);
             }
-            uint4 *dst = reinterpret_cast<uint4 *>(p.codes + (static_cast<int64_t>(pix) * p.O + o0 + o) * p.I1 + i0);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            if (IT == 32 && full_row) dst[1] = make_uint4(w[4 % (IT / 4)], w[5 % (IT / 4)], w[6 % (IT / 4)], w[7 % (IT / 4)]);
+            const int64_t off = (static_cast<int64_t>(pix) * p.O + o0 + o) * p.I1 + i0;   // in codes
+            store_row<FMT, IT / 4>(p.codes + (FMT == 2 ? off / 2 : off), h, full_row ? IT : 16);
         }
     }
     if (p.codes_alt == nullptr) return;
@@ -503,18 +524,17 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
             const int i = sub + NS * r;
             if (i0 + i >= p.I) break;
             const float inv_col = BLK == kAlongO ? s_inv[i * PT + pos] : inv_sq;
-            uint32_t w[OT / 4];
+            uint32_t h[OT / 4];
 #pragma unroll
             for (int q = 0; q < OT / 4; ++q) {
                 float v[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     v[k] = tp[((4 * q + k) * IT + i) * PT] * (BLK == kAlongI ? inv_o[(4 * q + k) % (BLK == kAlongI ? OT : 1)] : inv_col);
-                w[q] = cvt_pair<FMT>(v[0], v[1]) | (cvt_pair<FMT>(v[2], v[3]) << 16);
+                h[q] = pack4<FMT>(v);
             }
-            uint4 *dst = reinterpret_cast<uint4 *>(p.codes_alt + (static_cast<int64_t>(pix) * p.I + i0 + i) * p.O2 + o0);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            if (OT == 32 && full_row) dst[1] = make_uint4(w[4 % (OT / 4)], w[5 % (OT / 4)], w[6 % (OT / 4)], w[7 % (OT / 4)]);
+            const int64_t off = (static_cast<int64_t>(pix) * p.I + i0 + i) * p.O2 + o0;   // in codes
+            store_row<FMT, OT / 4>(p.codes_alt + (FMT == 2 ? off / 2 : off), h, full_row ? OT : 16);
         }
     }
 }
@@ -529,10 +549,15 @@ inline void launch_staged_tiles(const StagedParams &sp, unsigned grid, int smem,
         }
         kernel<<<grid, 256, smem, s>>>(sp);
     };
-    if (sp.OT == 16 && sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 16>);
-    else if (sp.OT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 32>);
-    else if (sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 32, 16>);
-    else pick(mx_quantize_staged_kernel<FMT, BLK, 32, 32>);
+    if constexpr (FMT == 2) {            // FP4 rows are 32 codes (16 bytes): IT = 32
+        if (sp.OT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 32>);
+        else pick(mx_quantize_staged_kernel<FMT, BLK, 32, 32>);
+    } else {
+        if (sp.OT == 16 && sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 16>);
+        else if (sp.OT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 32>);
+        else if (sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 32, 16>);
+        else pick(mx_quantize_staged_kernel<FMT, BLK, 32, 32>);
+    }
 }
 
 template <int FMT>

@@ -144,18 +144,30 @@ MQC_API mqc_status mqc_im2col_cbf(const void *codes, const uint8_t *scales, cons
 MQC_API int64_t mqc_im2col_cbf_scales_bytes(const mqc_conv *conv, const mqc_mx *mx);
 MQC_API int64_t mqc_im2col_cbf_codes_bytes(const mqc_conv *conv, const mqc_mx *mx);
 
-/* Forward convolution, Eq. 1, as the block-scaled GEMM
+/* The three GEMMs below take E4M3, E5M2 or E2M1 operands, in any mix.
+ * Accumulation is fp32 in tensor memory (tcgen05.mma kind::mxf8f6f4 with
+ * E8M0 block scales).  An E2M1 operand is first rewritten, in the caller's
+ * workspace, as the E4M3 codes of the same values (every E2M1 value is an
+ * E4M3 value; same layout, one byte per element); the products and the
+ * scales are unchanged.  Each GEMM has a *_workspace_bytes query: 0 when no
+ * operand is E2M1 (and, for the weight gradient, no split-K partials are
+ * needed), in which case workspace may be NULL.  The workspace must be
+ * 16-byte aligned; it is scratch, overwritten by the call.
+ *
+ * Forward convolution, Eq. 1, as the block-scaled GEMM
  * Y_f{Cout,N} = W_f{Cout,Cin} . X'_{Cin,N} of section IV-B, with the im2col
  * folded into the tensor-core operand staging.
  *   xq, xs  X quantized with blocks along C: block A32 or SQ32, order BA.
  *   wq, ws  W quantized with blocks along C: block A32 or SQ32, order BA.
  *   y       fp32 output [N][K][P][Q] (overwritten).
- * Accumulation is fp32 in tensor memory.  Formats: E4M3 or E5M2 for either
- * operand (MQC_ERR_UNSUPPORTED for E2M1 in this build).
- * Errors: MQC_ERR_INVALID, MQC_ERR_UNSUPPORTED, MQC_ERR_ALIGNMENT, MQC_ERR_CUDA. */
+ *   workspace, workspace_bytes: at least mqc_conv2d_fwd_workspace_bytes().
+ * Errors: MQC_ERR_INVALID, MQC_ERR_UNSUPPORTED, MQC_ERR_ALIGNMENT, MQC_ERR_CUDA,
+ * MQC_ERR_WORKSPACE. */
 MQC_API mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf,
                           const void *wq, const uint8_t *ws, const mqc_mx *wf,
-                          const mqc_conv *conv, float *y, void *stream);
+                          const mqc_conv *conv, float *y,
+                          void *workspace, size_t workspace_bytes, void *stream);
+MQC_API size_t mqc_conv2d_fwd_workspace_bytes(const mqc_conv *conv, const mqc_mx *xf, const mqc_mx *wf);
 
 /* Input gradient, Eq. 2: G_X = W^T * G_Y as the GEMM
  * G_X'{Cin,N} = W_f^T . G_Yf{Cout,N} of section IV-B, computed directly as a
@@ -166,10 +178,13 @@ MQC_API mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_m
  *   wq, ws  W quantized with blocks along K: block B32 or SQ32, order AB.
  *   gq, gs  G_Y quantized with blocks along K: block A32 or SQ32, order BA.
  *   gx      fp32 output [N][C][H][W] (overwritten).
+ *   workspace, workspace_bytes: at least mqc_conv2d_bwd_data_workspace_bytes().
  * Errors: as mqc_conv2d_fwd. */
 MQC_API mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *wf,
                                const void *gq, const uint8_t *gs, const mqc_mx *gf,
-                               const mqc_conv *conv, float *gx, void *stream);
+                               const mqc_conv *conv, float *gx,
+                               void *workspace, size_t workspace_bytes, void *stream);
+MQC_API size_t mqc_conv2d_bwd_data_workspace_bytes(const mqc_conv *conv, const mqc_mx *wf, const mqc_mx *gf);
 
 /* Weight gradient, Eq. 3: G_W[k,c] = sum_n G_Y[n,k] * X[n,c] as the GEMM
  * G_Wf{Cout,Cin} = G_Yf{Cout,N} . X'^T_{Cin,N} of section IV-B, reducing over
@@ -177,11 +192,12 @@ MQC_API mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const 
  *   gq, gs  G_Y quantized with blocks along N: block B32 or SQ32, order AB.
  *   xq, xs  X quantized with blocks along N: block B32 or SQ32, order AB.
  *   gw      fp32 output [K][C][R][S] (overwritten).
- *   workspace, workspace_bytes: device scratch for the split-K partial sums,
- *           at least mqc_conv2d_bwd_weight_workspace_bytes(); may be NULL
- *           when that size is 0.
+ *   workspace, workspace_bytes: device scratch for the split-K partial sums
+ *           and widened E2M1 operands, at least
+ *           mqc_conv2d_bwd_weight_workspace_bytes(); may be NULL when that
+ *           size is 0.
  * The split-K reduction is deterministic (fixed order).
- * Errors: as mqc_conv2d_fwd, plus MQC_ERR_WORKSPACE. */
+ * Errors: as mqc_conv2d_fwd. */
 MQC_API mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx *gf,
                                  const void *xq, const uint8_t *xs, const mqc_mx *xf,
                                  const mqc_conv *conv, float *gw,
@@ -205,9 +221,9 @@ MQC_API size_t mqc_conv2d_bwd_weight_workspace_bytes(const mqc_conv *conv, const
  *   - The first call on each device looks up that device's copy of the array
  *     (with the device current) and caches its address; make that first call
  *     before any stream capture.
- *   - A problem whose split-K scratch (mqc_conv2d_bwd_weight_workspace_bytes)
- *     exceeds MQC_NOALLOC_SCRATCH_BYTES is rejected with MQC_ERR_WORKSPACE
- *     and nothing is launched.
+ *   - A problem whose scratch (mqc_conv2d_bwd_weight_workspace_bytes: split-K
+ *     partials and widened E2M1 operands) exceeds MQC_NOALLOC_SCRATCH_BYTES
+ *     is rejected with MQC_ERR_WORKSPACE and nothing is launched.
  *   - Every call on a device shares the one array, which keeps the previous
  *     call's partial sums; each call overwrites every partial it later reads,
  *     so nothing needs to start at zero.  Calls that can overlap on the GPU

@@ -87,10 +87,28 @@ def test_invalid_arguments_rejected_before_launch(mqc):
     # GEMM operand in the wrong block mode / order / format
     cv = mqc.conv_desc(2, 32, 8, 8, 32, 3, 3, 1, 1)
     p = ctypes.c_void_p(256)
-    assert mqc.mqc_conv2d_fwd(p, p, mqc.MX(0, 1, 0), p, p, mqc.MX(0, 0, 0), cv, p, None) == -2
-    assert mqc.mqc_conv2d_fwd(p, p, mqc.MX(0, 0, 1), p, p, mqc.MX(0, 0, 0), cv, p, None) == -2
-    assert mqc.mqc_conv2d_bwd_data(p, p, mqc.MX(0, 0, 1), p, p, mqc.MX(1, 0, 0), cv, p, None) == -2
+    assert mqc.mqc_conv2d_fwd(p, p, mqc.MX(0, 1, 0), p, p, mqc.MX(0, 0, 0), cv, p, None, 0, None) == -2
+    assert mqc.mqc_conv2d_fwd(p, p, mqc.MX(0, 0, 1), p, p, mqc.MX(0, 0, 0), cv, p, None, 0, None) == -2
+    assert mqc.mqc_conv2d_bwd_data(p, p, mqc.MX(0, 0, 1), p, p, mqc.MX(1, 0, 0), cv, p, None, 0, None) == -2
     assert mqc.mqc_conv2d_bwd_weight(p, p, mqc.MX(1, 0, 1), p, p, mqc.MX(0, 1, 1), cv, p, None, 0, None) == -2
     # a convolution whose kernel is larger than the padded input
-    assert mqc.mqc_conv2d_fwd(p, p, mx, p, p, mx, mqc.conv_desc(1, 32, 2, 2, 8, 5, 5, 1, 1), p, None) == -1
+    assert mqc.mqc_conv2d_fwd(p, p, mx, p, p, mx, mqc.conv_desc(1, 32, 2, 2, 8, 5, 5, 1, 1), p, None, 0, None) == -1
     assert mqc.lib.mqc_debug_expire_wait(10, None) == -1
+
+
+def test_gemm_workspace_sizes_cover_widened_fp4_operands(mqc):
+    """E2M1 GEMM operands are widened to one byte per element in the caller's
+    workspace: the size queries give twice the packed code bytes (rounded up
+    to 256), and nothing for FP8 operands."""
+    cv = mqc.conv_desc(4, 40, 9, 11, 24, 3, 3, 2, 1)
+    P, Q = (9 + 2 - 3) // 2 + 1, (11 + 2 - 3) // 2 + 1
+    fp8_a, fp4_a = mqc.MX(0, 2, 0), mqc.MX(2, 2, 0)
+    fp8_b, fp4_b = mqc.MX(0, 2, 1), mqc.MX(2, 2, 1)
+    r = lambda n: (2 * n + 255) // 256 * 256
+    assert mqc.mqc_conv2d_fwd_workspace_bytes(cv, fp8_a, fp8_a) == 0
+    assert mqc.mqc_conv2d_fwd_workspace_bytes(cv, fp4_a, fp8_a) == r(mqc.mqc_codes_bytes(fp4_a, 4, 40, 9, 11))
+    assert mqc.mqc_conv2d_fwd_workspace_bytes(cv, fp4_a, fp4_a) == (r(mqc.mqc_codes_bytes(fp4_a, 4, 40, 9, 11))
+                                                                     + r(mqc.mqc_codes_bytes(fp4_a, 24, 40, 3, 3)))
+    assert mqc.mqc_conv2d_bwd_data_workspace_bytes(cv, fp8_b, fp8_a) == 0
+    assert mqc.mqc_conv2d_bwd_data_workspace_bytes(cv, fp4_b, fp4_a) == (r(mqc.mqc_codes_bytes(fp4_b, 24, 40, 3, 3))
+                                                                          + r(mqc.mqc_codes_bytes(fp4_a, 4, 24, P, Q)))

@@ -127,6 +127,36 @@ def test_conv_bwd_weight_parity(mqc, orc, case, sq):
     _check(f"wgrad {case} sq={sq}", _host(gw), ref, refabs)
 
 
+# FP4 (E2M1) operands, alone or mixed with FP8: (case, format of the first
+# operand, format of the second) for each GEMM
+FP4_CASES = [((4, 48, 9, 11, 40, 3, 3, 2, 1), 2, 0), ((16, 16, 12, 12, 32, 3, 3, 2, 1), 2, 2),
+             ((3, 128, 10, 9, 160, 3, 3, 1, 1), 0, 2), ((40, 96, 5, 6, 130, 1, 1, 1, 0), 2, 1)]
+
+
+@pytest.mark.parametrize("case,fa,fb", FP4_CASES)
+def test_conv_fp4_operands(mqc, orc, case, fa, fb):
+    """E2M1 operands run through the same tensor-core path (widened to the
+    E4M3 codes of the same values): forward (X, W), input gradient (W, G_Y)
+    and weight gradient (G_Y, X) against the oracle on its own E2M1
+    dequantization."""
+    N, C, H, W, K, R, S, st, pad = case
+    P, Q = orc.out_hw(H, W, R, S, st, st, pad, pad)
+    x = synth.random_tensor((N, C, H, W), seed=950 + C, dist="student_t")
+    w = synth.random_tensor((K, C, R, S), seed=951 + K, scale=0.05)
+    g = synth.random_tensor((N, K, P, Q), seed=952 + N, scale=1e-3)
+    cv = mqc.conv_desc(N, C, H, W, K, R, S, st, pad)
+    deq = lambda t, f, o: orc.dequantize(*orc.quantize(t, f, 2, o), t.shape, f, 2, o)
+    y = mqc.conv2d_fwd(mqc.quantize_mx(_dev(x), fa, 2, 0), mqc.quantize_mx(_dev(w), fb, 2, 0), cv)
+    ref, refabs = orc.conv_fwd(deq(x, fa, 0), deq(w, fb, 0), st, st, pad, pad)
+    _check(f"fwd fp4 {case} {fa}/{fb}", _host(y), ref, refabs)
+    gx = mqc.conv2d_bwd_data(mqc.quantize_mx(_dev(w), fa, 2, 1), mqc.quantize_mx(_dev(g), fb, 2, 0), cv)
+    ref, refabs = orc.conv_dgrad(deq(w, fa, 1), deq(g, fb, 0), H, W, st, st, pad, pad)
+    _check(f"dgrad fp4 {case} {fa}/{fb}", _host(gx), ref, refabs)
+    gw = mqc.conv2d_bwd_weight(mqc.quantize_mx(_dev(g), fa, 2, 1), mqc.quantize_mx(_dev(x), fb, 2, 1), cv)
+    ref, refabs = orc.conv_wgrad(deq(g, fa, 1), deq(x, fb, 1), R, S, st, st, pad, pad)
+    _check(f"wgrad fp4 {case} {fa}/{fb}", _host(gw), ref, refabs)
+
+
 def test_training_step_shares_one_quantization(mqc, orc):
     """SQ32: each tensor is quantized once, in both code orders, and the
     three GEMMs read those copies (paper, section IV-B: quantized once)."""

@@ -1,6 +1,7 @@
 """Parity at the benchmark's full sizes, in the launch configuration the
 benchmark times: every layer of the YOLOv8n-shaped N=16 640x640 training
-stack and the N=128, C=128, 80x80 MXFP8 layer, with the benchmark's own
+stack, the N=128, C=128, 80x80 MXFP8 and MXFP4 layers (MXFP4 also at
+N=32) and the latent-replay block (E2M1 activations), with the benchmark's own
 seeded inputs and the same C-ABI entry points (the library picks the tiling
 from the problem shape, so these are the benchmark's kernel launches).
 
@@ -19,7 +20,7 @@ import synth
 
 pytestmark = pytest.mark.gpu
 RTOL, ATOL = 1e-3, 1e-6
-CASES = [(3, i) for i in range(8)] + [((5, "fp8", 128), 0)]
+CASES = [(3, i) for i in range(8)] + [((5, "fp8", 128), 0), (4, 0), ((5, "fp4", 32), 0), ((5, "fp4", 128), 0)]
 # mid-sized layers (YOLO-like, N = 16) whose tile count gives units of two
 # 128-row sub-tiles rather than four
 MID = [synth.Layer(16, 16, 160, 160, 32, 3, 3, 2, 1), synth.Layer(16, 32, 80, 80, 32, 1, 1, 1, 0)]

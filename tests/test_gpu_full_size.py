@@ -8,10 +8,11 @@ from the problem shape, so these are the benchmark's kernel launches).
 - Quantization (MicroQonv paper, section III-A, Eq. 5-7): the codes of X,
   W and G_Y in both orders and their E8M0 scales are compared with the
   oracle's in full, bit for bit.
-- Convolutions (section II-C3, Eq. 1-3): the forward output, the input
-  gradient and the weight gradient on a seeded sample of elements, each
-  computed by the oracle on its own dequantized operands as a sum in double,
-  within |err| <= 1e-3 * sum|a*b| + 1e-6.
+- Convolutions (section II-C3, Eq. 1-3): the forward output and the input
+  gradient on 65,536 seeded elements plus every border pixel of image 0,
+  the weight gradient on 768 seeded elements (each a sum over N x P x Q);
+  each computed by the oracle on its own dequantized operands as a sum in
+  double, within |err| <= 1e-3 * sum|a*b| + 1e-6.
 """
 import numpy as np
 import pytest
@@ -46,10 +47,19 @@ def _host(t):
     return t.cpu().numpy()
 
 
-def _sample(shape, n, seed):
+def _sample(shape, n, seed, border=False):
+    """Seeded flat indices into an output of `shape`; with border, also every
+    border pixel (first/last row and column) of image 0, all channels."""
     rng = np.random.default_rng(seed)
     size = int(np.prod(shape))
-    return np.unique(rng.integers(0, size, size=min(n, size), dtype=np.int64))
+    idx = [rng.integers(0, size, size=min(n, size), dtype=np.int64)]
+    if border:
+        _, ch, hh, ww = shape
+        m = np.zeros((hh, ww), dtype=bool)
+        m[0, :] = m[-1, :] = m[:, 0] = m[:, -1] = True
+        pix = np.flatnonzero(m)
+        idx.append((np.arange(ch, dtype=np.int64)[:, None] * (hh * ww) + pix[None, :]).ravel())
+    return np.unique(np.concatenate(idx))
 
 
 def _check(name, got, idx, ref, refabs):
@@ -102,11 +112,11 @@ def _layer_parity(mqc, orc, wl, layer):
         deq[name] = orc.dequantize(rc, rs, t.shape, f, wl.block, BA)
 
     st, pd = L.stride, L.pad
-    yi = _sample(y.shape, 4096, 11 + layer)
+    yi = _sample(y.shape, 65536, 11 + layer, border=True)
     ref, refabs = orc.conv_fwd_at(deq["X"], deq["W"], yi, st, st, pd, pd)
     _check(f"fwd {wl.name} layer {layer}", _host(y), yi, ref, refabs)
 
-    gi = _sample(gx.shape, 4096, 12 + layer)
+    gi = _sample(gx.shape, 65536, 12 + layer, border=True)
     ref, refabs = orc.conv_dgrad_at(deq["W"], deq["G_Y"], L.H, L.W, gi, st, st, pd, pd)
     _check(f"dgrad {wl.name} layer {layer}", _host(gx), gi, ref, refabs)
 

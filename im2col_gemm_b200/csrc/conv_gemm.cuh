@@ -103,6 +103,7 @@ struct alignas(64) GemmParams {
     int32_t sf_vec4;             // A: each group of 4 K-blocks is 4 aligned consecutive scale bytes (one tap)
     int32_t sfb_vec4;            // B: likewise (the weights' scales along C)
     int32_t sfb_cached;          // CONV: B scale atoms of every (column tile, group) built once per CTA
+    int32_t sq_gather;           // WGRAD: square blocks on both operands, 32-row groups of an atom aligned
     int32_t groups;              // CONV: groups of 4 K-blocks per tile
     // CONV: a unit is um consecutive 128-row tiles (sub-tiles) sharing the
     // B operand, the pipeline stages and the per-unit bookkeeping; each
@@ -265,11 +266,15 @@ struct KitWalker {
     }
 };
 
-// SFV4 (CONV only): the A scales of 4 consecutive K-blocks are 4 aligned
-// bytes of one tap and are read with one 32-bit load per row; otherwise one
-// byte per (row, K-block).  The choice is a template parameter so that each
-// kernel carries only one gather path (the per-stage code of all roles has to
-// share the instruction cache).
+// SFV4, CONV: the A scales of 4 consecutive K-blocks are 4 aligned bytes of
+// one tap and are read with one 32-bit load per row; otherwise one byte per
+// (row, K-block).  SFV4, WGRAD: both operands have 32x32 square blocks and
+// every 32-row group of an atom shares one scale per K-block, so a group of 4
+// K-blocks needs 4 x 4 A bytes and 2 x 4 x 4 B bytes: one per lane, merged by
+// warp shuffles (instead of one load per row group and K-block in every lane).
+// The choice is a template parameter so that each kernel carries only one
+// gather path (the per-stage code of all roles has to share the instruction
+// cache).
 //
 // UMT (CONV only): 128-row sub-tiles per unit (1, 2 or 4; p.um equals it).
 // A template parameter as well, so that the one-tile kernel carries no
@@ -553,6 +558,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             int ra_h[4], ra_w[4], ra_off[4], ra_aw[4];
             bool ra_ok[4];
             auto set_rows = [&](int i) {
+                if (KIND == kWgrad && SFV4) {
+                    // this lane's A byte: row group (lane >> 2) & 3 (lanes 0-15)
+                    const int k = I.m0 + 32 * ((lane >> 2) & 3);
+                    ra_ok[0] = lane < 16 && k < p.sfa.rows;
+                    ra_off[0] = (k >> 5) * p.sfa.row_pitch;
+                    return;
+                }
                 int q0 = I.q0, p0 = I.p0, n0 = I.n0;
                 if (KIND == kConv && i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
 #pragma unroll
@@ -584,6 +596,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             // its tap's pixel offset; otherwise every row has the unit's tap)
             int rb_off[2][4], rb_dh[2][4], rb_dw[2][4];
             bool rb_ok[2][4];
+            if (KIND == kWgrad && SFV4) {
+                // this lane's B byte: atom lane >> 4, row group (lane >> 2) & 3
+                const int rl = 128 * (lane >> 4) + 32 * ((lane >> 2) & 3);
+                const int t = p.ntg > 1 ? static_cast<int>(p.fd_cpad.div(rl)) : 0;
+                const int r = I.col0 + rl - t * p.cpad;
+                rb_ok[0][0] = (lane >> 4) < p.nb_atoms && rl < p.BN && r < p.sfb.rows && t < I.tig;
+                rb_off[0][0] = (r >> 5) * p.sfb.row_pitch;
+                const ConvTap T = p.taps[I.tap + (rb_ok[0][0] ? t : 0)];
+                rb_dh[0][0] = T.sf_dh;
+                rb_dw[0][0] = T.sf_dw;
+            } else {
 #pragma unroll
             for (int at = 0; at < 2; ++at)
 #pragma unroll
@@ -604,6 +627,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         rb_dh[at][j] = rb_dw[at][j] = 0;
                     }
                 }
+            }
             KbWalker kw{I.tap0, 0};
             KitWalker kt{0, 0, 0};
             if (KIND == kConv) kw.advance(KS * first, p.CB);
@@ -678,6 +702,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                                 }
                                 k2.advance(1, p.CB);
                             }
+                        } else if (SFV4) {
+                            // lane: K-block lane & 3 of A row group (lane >> 2) & 3
+                            // and of B atom lane >> 4, row group (lane >> 2) & 3
+                            const int kbl = lane & 3;
+                            const int q = k3.qg * p.bqk + (kbl >> lg_wkb);
+                            const int nb = k3.nc * p.wkb + (kbl & (p.wkb - 1));
+                            uint32_t va = 0u, vb = 0u;
+                            if (q < p.Q) {
+                                const int64_t pix = static_cast<int64_t>(k3.pp) * p.Q + q;
+                                if (ra_ok[0])
+                                    va = __ldg(p.sfa.base + pix * p.sfa.pix_pitch + nb * p.sfa.kb_pitch + ra_off[0]);
+                                const int hh = p.x_st_h * k3.pp + rb_dh[0][0], ww = p.x_st_w * q + rb_dw[0][0];
+                                if (rb_ok[0][0] && hh >= 0 && hh < p.sfb.H && ww >= 0 && ww < p.sfb.W)
+                                    vb = __ldg(p.sfb.base +
+                                               (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
+                                               nb * p.sfb.kb_pitch + rb_off[0][0]);
+                            }
+                            va <<= 8 * kbl;
+                            vb <<= 8 * kbl;
+                            va |= __shfl_xor_sync(0xFFFFFFFFu, va, 1);
+                            vb |= __shfl_xor_sync(0xFFFFFFFFu, vb, 1);
+                            va |= __shfl_xor_sync(0xFFFFFFFFu, va, 2);
+                            vb |= __shfl_xor_sync(0xFFFFFFFFu, vb, 2);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                wa[j] = __shfl_sync(0xFFFFFFFFu, va, 4 * j);
+                                wb[0][j] = __shfl_sync(0xFFFFFFFFu, vb, 4 * j);
+                                wb[1][j] = __shfl_sync(0xFFFFFFFFu, vb, 16 + 4 * j);
+                            }
+                            k3.next(p);
                         } else {
                             for (int kb = 0; kb < 4; ++kb) {
                                 const int q = k3.qg * p.bqk + (kb >> lg_wkb);

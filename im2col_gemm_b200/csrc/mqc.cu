@@ -87,7 +87,7 @@ int conv_Q(const mqc_conv *c) { return (c->W + 2 * c->pad_w - c->S) / c->stride_
 struct DevInfo {
     int sms = 0;
     int max_smem = 0;
-    bool gemm_attr[7] = {};   // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind
+    bool gemm_attr[8] = {};   // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind, [7] SFV4 weight gradient
     bool quant_attr[36] = {};                             // staged quantizer, [(fmt*3 + blk)*4 + tile]
 };
 std::mutex g_dev_mu;
@@ -295,13 +295,13 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     P.timeout_ns = kDefaultTimeoutNs;
     const int smem = fixed + S * per_stage;
     const bool v4 = KIND == kConv && P.sf_vec4;
-    auto kernel = conv_gemm_kernel<kWgrad, false, 1>;
+    auto kernel = P.sq_gather ? conv_gemm_kernel<kWgrad, true, 1> : conv_gemm_kernel<kWgrad, false, 1>;
     if (KIND == kConv) {
         if (P.um == 4) kernel = v4 ? conv_gemm_kernel<kConv, true, 4> : conv_gemm_kernel<kConv, false, 4>;
         else if (P.um == 2) kernel = v4 ? conv_gemm_kernel<kConv, true, 2> : conv_gemm_kernel<kConv, false, 2>;
         else kernel = v4 ? conv_gemm_kernel<kConv, true, 1> : conv_gemm_kernel<kConv, false, 1>;
     }
-    const int ai = KIND == kConv ? 1 + (v4 ? 3 : 0) + (P.um == 4 ? 2 : P.um - 1) : 0;
+    const int ai = KIND == kConv ? 1 + (v4 ? 3 : 0) + (P.um == 4 ? 2 : P.um - 1) : (P.sq_gather ? 7 : 0);
     if (!d.gemm_attr[ai]) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.max_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -1057,6 +1057,9 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     G.sfb.rows = C;
     G.sfb.H = H;
     G.sfb.W = W;
+    // square blocks on both sides and every 32-column group of an atom inside
+    // one tap at a multiple of 32 channels: one scale per 32-row group
+    G.sq_gather = sqg && sqx && (G.ntg > 1 ? G.cpad % 32 == 0 : (G.NT == 1 || G.BN % 32 == 0));
     G.out = G.splits > 1 ? static_cast<float *>(workspace) : gw;
     G.out_base = 0;
     G.os_m = int64_t(C) * R * S;

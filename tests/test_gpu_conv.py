@@ -81,6 +81,7 @@ BWD_CASES = [
     (16, 16, 12, 12, 32, 3, 3, 2, 1),
     (40, 96, 5, 6, 130, 3, 3, 1, 1),
     (64, 32, 6, 6, 32, 3, 3, 1, 0),
+    (6, 160, 5, 5, 48, 3, 3, 1, 1),       # C > 128: one tap per weight-gradient unit, two column tiles
 ]
 
 

@@ -103,7 +103,8 @@ struct alignas(64) GemmParams {
     int32_t sf_vec4;             // A: each group of 4 K-blocks is 4 aligned consecutive scale bytes (one tap)
     int32_t sfb_vec4;            // B: likewise (the weights' scales along C)
     int32_t sfb_cached;          // CONV: B scale atoms of every (column tile, group) built once per CTA
-    int32_t sq_gather;           // WGRAD: square blocks on both operands, 32-row groups of an atom aligned
+    int32_t sq_gather;           // WGRAD: square blocks on both operands, 16-row groups of an atom aligned
+    int32_t sq16;                // WGRAD, sq_gather: a 32-row group of B may hold two taps (cpad = 16 mod 32)
     int32_t groups;              // CONV: groups of 4 K-blocks per tile
     // CONV: a unit is um consecutive 128-row tiles (sub-tiles) sharing the
     // B operand, the pipeline stages and the per-unit bookkeeping; each
@@ -131,6 +132,16 @@ struct alignas(64) GemmParams {
     // input channel), cpad rows per tap (a multiple of 8), so one MMA per
     // K-block covers ntg taps.  ntg = 1: the columns are channels of one tap.
     int32_t ntg, ngroups, cpad;
+    // WGRAD window boxes (tap groups of whole kernel rows): bmap[0] covers the
+    // unphased X as (batch, C, W, H), and one box of (batch, cpad, S, ntg / S)
+    // at the pixel's window origin lands every (tap, channel) row of the
+    // group in the column order of the GEMM; wb_S = S, wb_ph/wb_pw = padding
+    int32_t wbox, wb_S, wb_ph, wb_pw;
+    // WGRAD k16 (batch of at most 16): every operand row holds 16 batch codes
+    // in HBM, so a K-block row is 16 bytes in shared memory (the MMA reads its
+    // other 16 from a zero block) and the TMA views take 16 rows of 16 bytes
+    // as one 256-byte row: (256, rows / 16, ...) boxes, row coordinates / 16
+    int32_t k16;
     // the divisions of the unit and row decoding, by launch constants
     FastDiv fd_NT, fd_nph, fd_TQ, fd_TP, fd_sub, fd_bq, fd_bp, fd_bn, fd_MT, fd_ngroups, fd_splits, fd_cpad;
     int32_t x_st_h, x_st_w;      // stride of X pixels per output pixel
@@ -268,10 +279,12 @@ struct KitWalker {
 
 // SFV4, CONV: the A scales of 4 consecutive K-blocks are 4 aligned bytes of
 // one tap and are read with one 32-bit load per row; otherwise one byte per
-// (row, K-block).  SFV4, WGRAD: both operands have 32x32 square blocks and
-// every 32-row group of an atom shares one scale per K-block, so a group of 4
-// K-blocks needs 4 x 4 A bytes and 2 x 4 x 4 B bytes: one per lane, merged by
-// warp shuffles (instead of one load per row group and K-block in every lane).
+// (row, K-block).  SFV4, WGRAD: both operands have 32x32 square blocks, so
+// every 32-row group of an A atom and every 16-row group of a B atom (16 | cpad:
+// a group stays inside one tap and one channel block) shares one scale per
+// K-block; a group of 4 K-blocks needs 4 x 4 A bytes and 2 x 8 x 4 B bytes,
+// loaded one or two per lane and merged by warp shuffles (instead of one load
+// per row group and K-block in every lane).
 // The choice is a template parameter so that each kernel carries only one
 // gather path (the per-stage code of all roles has to share the instruction
 // cache).
@@ -288,11 +301,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     const int KS = p.kbs;                     // K-blocks per stage
     const int GA = KS / 4;                    // groups of 4 K-blocks (one scale atom) per stage
     const int row_bytes = 32 * p.wkb;         // bytes of one operand row of a TMA box
+    const int kb_bytes = p.k16 ? 16 : 32;     // shared-memory bytes of one row of one K-block
+    const int srow = p.k16 ? 16 : row_bytes;  // shared-memory bytes of one row of a TMA box (wkb K-blocks)
+    const int rsh = p.k16 ? 4 : 0;            // row coordinate shift of the 16-row TMA views
     const int lg_wkb = p.wkb == 4 ? 2 : (p.wkb == 2 ? 1 : 0);
     constexpr int UM = KIND == kConv ? UMT : 1;   // 128-row sub-tiles per unit
-    const int a_sub_stage = 128 * 32 * KS;     // one sub-tile's A rows of a stage
+    const int a_sub_stage = 128 * kb_bytes * KS;   // one sub-tile's A rows of a stage
     const int a_stage = UM * a_sub_stage;
-    const int b_stage = p.BN * 32 * KS;
+    const int b_stage = p.BN * kb_bytes * KS;
     const int sfa_stage = 512 * GA * UM;       // A atoms [group][sub-tile]
     const int sfb_stage = 512 * GA * p.nb_atoms;
     uint8_t *sA = smem;
@@ -309,6 +325,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
     uint64_t *acc_empty = acc_full + kMaxAcc;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + kMaxAcc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    // k16: the upper 16 bytes of every operand row (batch 16..31 of a K-block)
+    // are read by the MMA from this zero block (256 rows x 16 bytes)
+    uint8_t *sZ = reinterpret_cast<uint8_t *>(full) + 1024;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -362,6 +381,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         }
         fence_proxy_async_smem();
     }
+    if (p.k16) {
+        for (int i = threadIdx.x; i < 4096 / 16; i += kGemmThreads)
+            reinterpret_cast<uint4 *>(sZ)[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -382,6 +406,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             KbWalker kw{I.tap0, 0};
             KitWalker kt{0, 0, 0};
             if (KIND == kWgrad) kt.init(p, I.kbase);
+            // window boxes: input row of the group's first kernel row at output row 0
+            const int wb_h0 = KIND == kWgrad && p.wbox ? I.tap / p.wb_S - p.wb_ph : 0;
             int oq[4], op[4], on[4];             // sub-tile origins
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -427,23 +453,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     const int nkit = min(GA, I.nkit - GA * ki);
                     // B: one box over the kit's pixels (one tap), or one box
                     // per (tap, pixel) of a tap group
-                    const int bmul = p.ntg > 1 ? I.tig * p.bqk : 1;
+                    const int bmul = p.ntg > 1 ? (p.wbox ? 1 : I.tig) * p.bqk : 1;
                     if (leader)
                         mbar_arrive_expect_tx(&full[s],
                                               static_cast<uint32_t>(nkit * (p.a_box_bytes + bmul * p.b_box_bytes)));
                     for (int g = 0; g < nkit; ++g) {
                         const int nx = kt.nc * row_bytes;
                         if (leader) {
-                            tma_load_4d(a_dst + g * 128 * 128, &p.amap[0], &full[s], nx, I.m0, kt.qg * p.bqk, kt.pp);
+                            tma_load_4d(a_dst + g * 128 * 4 * kb_bytes, &p.amap[0], &full[s], nx, I.m0 >> rsh,
+                                        kt.qg * p.bqk, kt.pp);
                             if (p.ntg == 1) {
                                 const ConvTap T = p.taps[I.tap];
-                                tma_load_4d(b_dst + g * p.BN * 128, &p.bmap[T.map], &full[s], nx, I.col0,
-                                            kt.qg * p.bqk + T.dw, kt.pp + T.dh);
+                                tma_load_4d(b_dst + g * p.BN * 4 * kb_bytes, &p.bmap[T.map], &full[s], nx,
+                                            I.col0 >> rsh, kt.qg * p.bqk + T.dw, kt.pp + T.dh);
+                            } else if (p.wbox) {
+                                // the group's kernel rows r0.. and all S columns, one box per pixel
+                                const int h = p.x_st_h * kt.pp + wb_h0;
+                                for (int jq = 0; jq < p.bqk; ++jq)
+                                    tma_load_4d(b_dst + g * p.BN * 4 * kb_bytes + jq * p.BN * srow, &p.bmap[0], &full[s],
+                                                nx, 0, p.x_st_w * (kt.qg * p.bqk + jq) - p.wb_pw, h);
                             } else {
                                 for (int t = 0; t < I.tig; ++t) {
                                     const ConvTap T = p.taps[I.tap + t];
                                     for (int jq = 0; jq < p.bqk; ++jq)
-                                        tma_load_4d(b_dst + g * p.BN * 128 + (jq * p.BN + t * p.cpad) * row_bytes,
+                                        tma_load_4d(b_dst + g * p.BN * 4 * kb_bytes + (jq * p.BN + t * p.cpad) * srow,
                                                     &p.bmap[T.map], &full[s], nx, 0, kt.qg * p.bqk + jq + T.dw,
                                                     kt.pp + T.dh);
                                 }
@@ -471,15 +504,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         int s = 0;
         uint32_t ph = 0;
         bool ok = true;
-        const uint32_t swz = swizzle_of(p.wkb);
-        // descriptors of stage 0, sub-tile 0; other positions add (byte offset >> 4)
-        const uint64_t adesc0 = make_smem_desc(smem_u32(sA), 16, 8 * row_bytes, swz);
-        const uint64_t bdesc0 = make_smem_desc(smem_u32(sB), 16, 8 * row_bytes, swz);
+        // descriptors of stage 0, sub-tile 0; other positions add (byte offset
+        // >> 4).  k16: no swizzle, 8-row core matrices of 16-byte rows (SBO 128),
+        // the second 16 bytes of K at the zero block (LBO = its distance, so an
+        // offset added to the start address is taken off the LBO field)
+        const uint32_t swz = p.k16 ? static_cast<uint32_t>(kSwizzleNone) : swizzle_of(p.wkb);
+        const uint64_t adesc0 = p.k16 ? make_smem_desc(smem_u32(sA), smem_u32(sZ) - smem_u32(sA), 128, swz)
+                                      : make_smem_desc(smem_u32(sA), 16, 8 * row_bytes, swz);
+        const uint64_t bdesc0 = p.k16 ? make_smem_desc(smem_u32(sB), smem_u32(sZ) - smem_u32(sB), 128, swz)
+                                      : make_smem_desc(smem_u32(sB), 16, 8 * row_bytes, swz);
+        const uint64_t lbo_step = p.k16 ? (1ull << 16) : 0ull;   // LBO change per 16 bytes of offset
         const uint64_t sfa_desc0 = make_smem_desc(smem_u32(sSFA), 0, 128, kSwizzleNone);
         const uint64_t sfb_desc0 = make_smem_desc(smem_u32(sSFB), 0, 128, kSwizzleNone);
         const uint64_t sfbc_desc0 = make_smem_desc(smem_u32(sSFBc), 0, 128, kSwizzleNone);
-        const uint32_t a_sub = (p.a_slab * row_bytes) >> 4, b_sub = (p.b_slab * row_bytes) >> 4;
-        const uint32_t a_grp = (128 * 128) >> 4, b_grp = (p.BN * 128) >> 4;   // one group of 4 K-blocks
+        const uint32_t a_sub = (p.a_slab * srow) >> 4, b_sub = (p.b_slab * srow) >> 4;
+        const uint32_t a_grp = (128 * 4 * kb_bytes) >> 4, b_grp = (p.BN * 4 * kb_bytes) >> 4;   // 4 K-blocks
         for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
             if (I.nk == 0) continue;
@@ -499,8 +538,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 const uint32_t sfb_t = sf_t + 4 * GA * UM;
                 const int nkb = KIND == kConv ? min(KS, I.tkb - KS * ki) : 4 * min(GA, I.nkit - GA * ki);
                 const int ngr = (nkb + 3) >> 2;
-                const uint64_t a_s = adesc0 + static_cast<uint64_t>((s * a_stage) >> 4);
-                const uint64_t b_s = bdesc0 + static_cast<uint64_t>((s * b_stage) >> 4);
+                const uint32_t a_s = static_cast<uint32_t>(s * a_stage) >> 4;
+                const uint32_t b_s = static_cast<uint32_t>(s * b_stage) >> 4;
                 if (leader) {
                     for (int g = 0; g < ngr; ++g) {
                         for (int i = 0; i < UM; ++i)
@@ -518,12 +557,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         const uint32_t g = static_cast<uint32_t>(kb >> 2), k4 = static_cast<uint32_t>(kb & 3);
                         const uint32_t j = k4 >> lg_wkb;                       // sub-tile within the group
                         const uint32_t within = k4 & static_cast<uint32_t>(p.wkb - 1);
-                        for (int i = 0; i < UM; ++i)
-                            tc_mma_mxf8f6f4(d_tmem + i * p.BN,
-                                            a_s + static_cast<uint64_t>((i * a_sub_stage) >> 4) + g * a_grp + j * a_sub + within * 2,
-                                            b_s + g * b_grp + j * b_sub + within * 2, p.idesc | (k4 << 29) | (k4 << 4),
+                        const uint32_t bo = b_s + g * b_grp + j * b_sub + within * 2;
+                        for (int i = 0; i < UM; ++i) {
+                            const uint32_t ao = a_s + ((i * a_sub_stage) >> 4) + g * a_grp + j * a_sub + within * 2;
+                            tc_mma_mxf8f6f4(d_tmem + i * p.BN, adesc0 + ao - ao * lbo_step, bdesc0 + bo - bo * lbo_step,
+                                            p.idesc | (k4 << 29) | (k4 << 4),
                                             (sf_t + 4 * (g * UM + i)) | (k4 << 30), (sfb_t + 4 * g * p.nb_atoms) | (k4 << 30),
                                             (ki > 0 || kb > 0) ? 1u : 0u);
+                        }
                     }
                     tc_commit(&empty[s]);
                 }
@@ -597,15 +638,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             int rb_off[2][4], rb_dh[2][4], rb_dw[2][4];
             bool rb_ok[2][4];
             if (KIND == kWgrad && SFV4) {
-                // this lane's B byte: atom lane >> 4, row group (lane >> 2) & 3
-                const int rl = 128 * (lane >> 4) + 32 * ((lane >> 2) & 3);
-                const int t = p.ntg > 1 ? static_cast<int>(p.fd_cpad.div(rl)) : 0;
-                const int r = I.col0 + rl - t * p.cpad;
-                rb_ok[0][0] = (lane >> 4) < p.nb_atoms && rl < p.BN && r < p.sfb.rows && t < I.tig;
-                rb_off[0][0] = (r >> 5) * p.sfb.row_pitch;
-                const ConvTap T = p.taps[I.tap + (rb_ok[0][0] ? t : 0)];
-                rb_dh[0][0] = T.sf_dh;
-                rb_dw[0][0] = T.sf_dw;
+                // this lane's B bytes: with 16-row groups, group 2 ((lane >> 3) & 3) +
+                // ((lane >> 2) & 1) of atom 0 and of atom 1; with 32-row groups,
+                // group (lane >> 2) & 3 of atom lane >> 4 (one byte)
+#pragma unroll
+                for (int at = 0; at < 2; ++at) {
+                    const int atom = p.sq16 ? at : lane >> 4;
+                    const int rl = p.sq16 ? 128 * at + 32 * ((lane >> 3) & 3) + 16 * ((lane >> 2) & 1)
+                                          : 128 * atom + 32 * ((lane >> 2) & 3);
+                    const int t = p.ntg > 1 ? static_cast<int>(p.fd_cpad.div(rl)) : 0;
+                    const int r = I.col0 + rl - t * p.cpad;
+                    rb_ok[at][0] = atom < p.nb_atoms && rl < p.BN && r < p.sfb.rows && t < I.tig;
+                    rb_off[at][0] = (r >> 5) * p.sfb.row_pitch;
+                    const ConvTap T = p.taps[I.tap + (rb_ok[at][0] ? t : 0)];
+                    rb_dh[at][0] = T.sf_dh;
+                    rb_dw[at][0] = T.sf_dw;
+                }
             } else {
 #pragma unroll
             for (int at = 0; at < 2; ++at)
@@ -703,33 +751,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                                 k2.advance(1, p.CB);
                             }
                         } else if (SFV4) {
-                            // lane: K-block lane & 3 of A row group (lane >> 2) & 3
-                            // and of B atom lane >> 4, row group (lane >> 2) & 3
+                            // lane: K-block lane & 3; A row group (lane >> 2) & 3
+                            // (lanes 0-15); B 16-row group of each atom as above
                             const int kbl = lane & 3;
                             const int q = k3.qg * p.bqk + (kbl >> lg_wkb);
                             const int nb = k3.nc * p.wkb + (kbl & (p.wkb - 1));
-                            uint32_t va = 0u, vb = 0u;
+                            uint32_t va = 0u, vb[2] = {0u, 0u};
                             if (q < p.Q) {
                                 const int64_t pix = static_cast<int64_t>(k3.pp) * p.Q + q;
                                 if (ra_ok[0])
                                     va = __ldg(p.sfa.base + pix * p.sfa.pix_pitch + nb * p.sfa.kb_pitch + ra_off[0]);
-                                const int hh = p.x_st_h * k3.pp + rb_dh[0][0], ww = p.x_st_w * q + rb_dw[0][0];
-                                if (rb_ok[0][0] && hh >= 0 && hh < p.sfb.H && ww >= 0 && ww < p.sfb.W)
-                                    vb = __ldg(p.sfb.base +
-                                               (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
-                                               nb * p.sfb.kb_pitch + rb_off[0][0]);
+#pragma unroll
+                                for (int at = 0; at < 2; ++at) {
+                                    if (at == 1 && !p.sq16) break;
+                                    const int hh = p.x_st_h * k3.pp + rb_dh[at][0], ww = p.x_st_w * q + rb_dw[at][0];
+                                    if (rb_ok[at][0] && hh >= 0 && hh < p.sfb.H && ww >= 0 && ww < p.sfb.W)
+                                        vb[at] = __ldg(p.sfb.base +
+                                                       (static_cast<int64_t>(hh) * p.sfb.W + ww) * p.sfb.pix_pitch +
+                                                       nb * p.sfb.kb_pitch + rb_off[at][0]);
+                                }
                             }
                             va <<= 8 * kbl;
-                            vb <<= 8 * kbl;
-                            va |= __shfl_xor_sync(0xFFFFFFFFu, va, 1);
-                            vb |= __shfl_xor_sync(0xFFFFFFFFu, vb, 1);
-                            va |= __shfl_xor_sync(0xFFFFFFFFu, va, 2);
-                            vb |= __shfl_xor_sync(0xFFFFFFFFu, vb, 2);
+                            vb[0] <<= 8 * kbl;
+                            vb[1] <<= 8 * kbl;
+#pragma unroll
+                            for (int x = 1; x <= 2; x <<= 1) {
+                                va |= __shfl_xor_sync(0xFFFFFFFFu, va, x);
+                                vb[0] |= __shfl_xor_sync(0xFFFFFFFFu, vb[0], x);
+                                if (p.sq16) vb[1] |= __shfl_xor_sync(0xFFFFFFFFu, vb[1], x);
+                            }
+                            if (!p.sq16) vb[1] = vb[0];
+                            // row lane + 32 j of B atom `at`: 16-row group 2 j + (lane >> 4)
+                            // of vb[at], or 32-row group j of atom at in vb[0]
+                            const int b0 = p.sq16 ? 4 * (lane >> 4) : 0, b1 = p.sq16 ? b0 : 16;
+                            const int bstep = p.sq16 ? 8 : 4;
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 wa[j] = __shfl_sync(0xFFFFFFFFu, va, 4 * j);
-                                wb[0][j] = __shfl_sync(0xFFFFFFFFu, vb, 4 * j);
-                                wb[1][j] = __shfl_sync(0xFFFFFFFFu, vb, 16 + 4 * j);
+                                wb[0][j] = __shfl_sync(0xFFFFFFFFu, vb[0], b0 + bstep * j);
+                                wb[1][j] = __shfl_sync(0xFFFFFFFFu, vb[1], b1 + bstep * j);
                             }
                             k3.next(p);
                         } else {

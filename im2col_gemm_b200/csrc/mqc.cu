@@ -152,8 +152,10 @@ mqc_status encode_codes_map(CUtensorMap *map, const void *base, int rank, const 
         if (strides[i] % 16 != 0) return fail(MQC_ERR_ALIGNMENT, "tensor stride %llu not a multiple of 16 bytes",
                                               (unsigned long long)strides[i]);
     }
-    const CUtensorMapSwizzle sw = wkb == 4 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                           : (wkb == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    const CUtensorMapSwizzle sw = wkb == 4   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : wkb == 2 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : wkb == 1 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                             : CU_TENSOR_MAP_SWIZZLE_NONE;   // wkb 0: plain rows
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void *>(base), gd, gs, bx, es,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -232,7 +234,8 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     P.sfb_cached = KIND == kConv && cache <= 16384 && !P.sfb_vec4;
     // the 32-bit scale path reads B four bytes at a time unless B is cached
     if (!P.sfb_cached && !P.sfb_vec4) P.sf_vec4 = 0;
-    const int fixed = 1024 + 64 * 8 + 64 + (P.sfb_cached ? cache : 0);
+    // k16: the zero block (4 KB) 1 KB past the barriers
+    const int fixed = 1024 + (P.k16 ? 1024 + 4096 : 64 * 8 + 64) + (P.sfb_cached ? cache : 0);
     // CONV with few K-blocks per tile and narrow column tiles: units of
     // um = 2 or 4 row tiles, so that the per-unit work of every role (decode,
     // barrier round trips, B loads, scale atoms of B) is shared by um MMAs;
@@ -256,7 +259,9 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     }
     auto stages_for = [&](int kbs, int &S) {
         const int ga = kbs / 4;
-        const int per_stage = P.um * 128 * 32 * kbs + P.BN * 32 * kbs + 512 * ga * P.um + 512 * ga * P.nb_atoms;
+        const int kb_bytes = P.k16 ? 16 : 32;
+        const int per_stage =
+            P.um * 128 * kb_bytes * kbs + P.BN * kb_bytes * kbs + 512 * ga * P.um + 512 * ga * P.nb_atoms;
         const int sf_cols = ga * (4 * P.um + 4 * P.nb_atoms);
         S = std::min(8, (d.max_smem - fixed) / per_stage);
         S = std::min(S, (kTmemCols - kSfTmemBase) / sf_cols);
@@ -893,6 +898,7 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
 // of them instead of one narrow MMA per tap.
 struct WgradPlan {
     int BN, splits, ntg, ngroups, cpad;
+    bool wbox;      // tap groups of whole kernel rows, loaded as window boxes
     int64_t kiters;
 };
 
@@ -906,8 +912,24 @@ static WgradPlan wgrad_plan(const mqc_conv *c, const DevInfo &d) {
     const int ntaps = c->R * c->S;
     w.kiters = int64_t(P) * ceil_div(Q, bqk) * (NB / wkb);
     w.cpad = static_cast<int>(round_up(c->C, 8));
-    if (ntaps > 1 && c->C <= 128) {
-        const int most = std::max(1, 256 / w.cpad);
+    const int most = std::max(1, 256 / w.cpad);   // taps whose columns fit 256
+    if (ntaps > 1 && c->C <= 128 && most >= c->S) {
+        // groups of kr whole kernel rows: one TMA box per pixel brings every
+        // (tap, channel) row of the group (the taps of a kernel row are
+        // neighbouring pixels of X, whatever the stride).  kr: the fewest GEMM
+        // columns over all groups (a partial last group still computes whole
+        // rows), then the fewest groups.  Measured on the YOLOv8n layers:
+        // C = 16 one group of 3 rows, C = 32 three groups of one row.
+        int kr = 1;
+        for (int k = 1; k <= std::min(c->R, most / c->S); ++k)
+            if (ceil_div(c->R, k) * round_up(c->S * k * w.cpad, 16) <=
+                ceil_div(c->R, kr) * round_up(c->S * kr * w.cpad, 16))
+                kr = k;
+        w.ngroups = static_cast<int>(ceil_div(c->R, kr));
+        w.ntg = c->S * kr;
+        w.wbox = true;
+        w.BN = static_cast<int>(round_up(w.ntg * w.cpad, 16));
+    } else if (ntaps > 1 && c->C <= 128) {
         w.ngroups = static_cast<int>(ceil_div(ntaps, most));
         w.ntg = static_cast<int>(ceil_div(ntaps, w.ngroups));
         w.BN = static_cast<int>(round_up(w.ntg * w.cpad, 16));
@@ -986,12 +1008,25 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     G.x_st_h = sh;
     G.x_st_w = sw;
     G.idesc = make_idesc_mx(mma_fmt(og.mma_fmt), mma_fmt(ox.mma_fmt), 128, G.BN);
-    {
+    // batch of at most 16 (rows of 16 codes) and channel counts in 16s: the
+    // maps take 16 rows of 16 bytes as one 256-byte row, unswizzled
+    G.k16 = Np == 16 && Npx == 16 && K % 16 == 0 && C % 16 == 0 && G.wkb == 1;
+    const int rb = G.k16 ? 16 : 32 * G.wkb;   // bytes of one operand row of a box
+    if (G.k16) {
+        const uint64_t dims[4] = {256, uint64_t(K / 16), uint64_t(Q), uint64_t(P)};
+        const uint64_t strd[3] = {256, uint64_t(K) * 16, uint64_t(Q) * K * 16};
+        const uint32_t box[4] = {256, uint32_t(box_rows(K, 128) / 16), uint32_t(G.bqk), 1u};
+        if ((st = encode_codes_map(&G.amap[0], og.codes, 4, dims, strd, box, 0)) != MQC_OK) return st;
+    } else {
         const uint64_t dims[4] = {uint64_t(Np), uint64_t(K), uint64_t(Q), uint64_t(P)};
         const uint64_t strd[3] = {uint64_t(Np), uint64_t(K) * Np, uint64_t(Q) * K * Np};
         const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(box_rows(K, 128)), uint32_t(G.bqk), 1u};
         if ((st = encode_codes_map(&G.amap[0], og.codes, 4, dims, strd, box, G.wkb)) != MQC_OK) return st;
     }
+    G.wbox = plan.wbox;
+    G.wb_S = S;
+    G.wb_ph = c->pad_h;
+    G.wb_pw = c->pad_w;
     bool phase_ok[16] = {};
     for (int a = 0; a < sh; ++a)
         for (int b = 0; b < sw; ++b) {
@@ -999,14 +1034,21 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
             phase_ok[a * sw + b] = Hh > 0 && Ww > 0;
             if (!phase_ok[a * sw + b]) continue;
             const uint8_t *base = ox.codes + (int64_t(a) * W + b) * C * Npx;
-            const uint64_t dims[4] = {uint64_t(Npx), uint64_t(C), uint64_t(Ww), uint64_t(Hh)};
-            const uint64_t strd[3] = {uint64_t(Npx), uint64_t(sw) * C * Npx, uint64_t(sh) * W * C * Npx};
+            const int rows = G.ntg > 1 ? G.cpad : box_rows(C, G.BN);
             // one tap: a box over the kit's bqk pixels; tap groups: one pixel
             // of one tap per box (cpad rows), placed at that tap's rows
-            const uint32_t box[4] = {uint32_t(32 * G.wkb),
-                                     uint32_t(G.ntg > 1 ? G.cpad : box_rows(C, G.BN)),
+            const uint32_t box[4] = {uint32_t(G.k16 ? 256 : 32 * G.wkb), uint32_t(G.k16 ? rows / 16 : rows),
                                      uint32_t(G.ntg > 1 ? 1 : G.bqk), 1u};
-            if ((st = encode_codes_map(&G.bmap[a * sw + b], base, 4, dims, strd, box, G.wkb)) != MQC_OK) return st;
+            if (G.k16) {
+                const uint64_t dims[4] = {256, uint64_t(C / 16), uint64_t(Ww), uint64_t(Hh)};
+                const uint64_t strd[3] = {256, uint64_t(sw) * C * 16, uint64_t(sh) * W * C * 16};
+                if ((st = encode_codes_map(&G.bmap[a * sw + b], base, 4, dims, strd, box, 0)) != MQC_OK) return st;
+            } else {
+                const uint64_t dims[4] = {uint64_t(Npx), uint64_t(C), uint64_t(Ww), uint64_t(Hh)};
+                const uint64_t strd[3] = {uint64_t(Npx), uint64_t(sw) * C * Npx, uint64_t(sh) * W * C * Npx};
+                if ((st = encode_codes_map(&G.bmap[a * sw + b], base, 4, dims, strd, box, G.wkb)) != MQC_OK)
+                    return st;
+            }
         }
     G.ntaps = 0;
     for (int r = 0; r < R; ++r)
@@ -1036,10 +1078,20 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
                 if (phase_ok[j]) { G.bmap[i] = G.bmap[j]; break; }
     G.n_amaps = 1;
     G.n_bmaps = sh * sw;
+    if (G.wbox) {
+        // (batch, C, W, H) of the whole X; a box of cpad channels x S x kr pixels
+        const uint64_t dims[4] = {G.k16 ? 256 : uint64_t(Npx), uint64_t(G.k16 ? C / 16 : C), uint64_t(W), uint64_t(H)};
+        const uint64_t strd[3] = {G.k16 ? 256 : uint64_t(Npx), uint64_t(C) * Npx, uint64_t(W) * C * Npx};
+        const uint32_t box[4] = {uint32_t(G.k16 ? 256 : 32 * G.wkb), uint32_t(G.k16 ? G.cpad / 16 : G.cpad),
+                                 uint32_t(S), uint32_t(G.ntg / S)};
+        if ((st = encode_codes_map(&G.bmap[0], ox.codes, 4, dims, strd, box, G.k16 ? 0 : G.wkb)) != MQC_OK)
+            return st;
+        G.n_bmaps = 1;
+    }
     G.a_slab = box_rows(K, 128);
     G.b_slab = G.ntg > 1 ? G.BN : box_rows(C, G.BN);
-    G.a_box_bytes = 32 * G.wkb * G.a_slab * G.bqk;
-    G.b_box_bytes = G.ntg > 1 ? 32 * G.wkb * G.cpad : 32 * G.wkb * G.b_slab * G.bqk;
+    G.a_box_bytes = rb * G.a_slab * G.bqk;
+    G.b_box_bytes = G.wbox ? rb * G.cpad * G.ntg : (G.ntg > 1 ? rb * G.cpad : rb * G.b_slab * G.bqk);
     const bool sqg = gf->block == MQC_BLOCK_SQ32, sqx = xf->block == MQC_BLOCK_SQ32;
     G.sfa.base = gs;
     G.sfa.pix_pitch = nb32(Np) * (sqg ? nb32(K) : K);
@@ -1057,9 +1109,10 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     G.sfb.rows = C;
     G.sfb.H = H;
     G.sfb.W = W;
-    // square blocks on both sides and every 32-column group of an atom inside
-    // one tap at a multiple of 32 channels: one scale per 32-row group
-    G.sq_gather = sqg && sqx && (G.ntg > 1 ? G.cpad % 32 == 0 : (G.NT == 1 || G.BN % 32 == 0));
+    // square blocks on both sides and every 16-column group of an atom inside
+    // one tap: one scale per 16-row group (columns start at multiples of 16)
+    G.sq_gather = sqg && sqx && (G.ntg == 1 || G.cpad % 16 == 0);
+    G.sq16 = G.ntg > 1 ? G.cpad % 32 != 0 : G.BN % 32 != 0 && G.NT > 1;
     G.out = G.splits > 1 ? static_cast<float *>(workspace) : gw;
     G.out_base = 0;
     G.os_m = int64_t(C) * R * S;

@@ -112,7 +112,17 @@ def test_conv_bwd_data_parity(mqc, orc, case, sq):
     _check(f"dgrad {case} sq={sq}", _host(gx), ref, refabs)
 
 
-@pytest.mark.parametrize("case", BWD_CASES)
+# weight-gradient cases beyond the shared ones: tap groups of whole kernel
+# rows loaded as one window box per pixel with channels beyond C (C = 3), with
+# 128-byte rows (N = 128), and with a partial last group (5x5, two rows each)
+WGRAD_CASES = BWD_CASES + [
+    (2, 3, 16, 16, 16, 3, 3, 2, 1),
+    (128, 16, 6, 6, 32, 3, 3, 2, 1),
+    (4, 24, 11, 10, 40, 5, 5, 2, 2),
+]
+
+
+@pytest.mark.parametrize("case", WGRAD_CASES)
 @pytest.mark.parametrize("sq", [False, True])
 def test_conv_bwd_weight_parity(mqc, orc, case, sq):
     N, C, H, W, K, R, S, st, pad = case

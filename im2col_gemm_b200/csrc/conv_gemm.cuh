@@ -142,6 +142,11 @@ struct alignas(64) GemmParams {
     // other 16 from a zero block) and the TMA views take 16 rows of 16 bytes
     // as one 256-byte row: (256, rows / 16, ...) boxes, row coordinates / 16
     int32_t k16;
+    // CONV d2s (input gradient as one sub-pixel GEMM): GEMM column n is
+    // (phase n / cpad, channel n % cpad) and lands at channel offset
+    // (n % cpad) * os_c + d2s_off[phase]; cpad is a multiple of 16
+    int32_t d2s;
+    int64_t d2s_off[kMaxPhases];
     // the divisions of the unit and row decoding, by launch constants
     FastDiv fd_NT, fd_nph, fd_TQ, fd_TP, fd_sub, fd_bq, fd_bp, fd_bn, fd_MT, fd_ngroups, fd_splits, fd_cpad;
     int32_t x_st_h, x_st_w;      // stride of X pixels per output pixel
@@ -899,7 +904,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                     set_row(i);
                     if (row_ok)
                         for (int n = 0; n < p.BN; ++n) {
-                            if (tap_cols) {
+                            if (KIND == kConv && p.d2s) {
+                                const int cs = I.col0 + n;
+                                const int ph = static_cast<int>(p.fd_cpad.div(cs));
+                                if (cs < p.Ncols) p.out[row_off + (cs - ph * p.cpad) * p.os_c + p.d2s_off[ph]] = 0.0f;
+                            } else if (tap_cols) {
                                 const int t = static_cast<int>(p.fd_cpad.div(n)), c = n - t * p.cpad;
                                 if (t < I.tig && c < p.Ncols) p.out[row_off + c * p.os_c + p.taps[I.tap + t].btap] = 0.0f;
                             } else if (I.col0 + n < p.Ncols) {
@@ -930,6 +939,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                    }
+                    if (KIND == kConv && p.d2s) {
+                        // 16 columns at a time: one phase, consecutive channels
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int n0 = I.col0 + c0 + 16 * h;
+                            if (!row_ok || n0 >= p.Ncols) continue;
+                            const int ph = static_cast<int>(p.fd_cpad.div(n0));
+                            float *op = orow + static_cast<int64_t>(n0 - ph * p.cpad) * p.os_c + p.d2s_off[ph];
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj) op[jj * p.os_c] = __uint_as_float(r[16 * h + jj]);
+                        }
+                        continue;
                     }
                     if (tap_cols) {
 #pragma unroll

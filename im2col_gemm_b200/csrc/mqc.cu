@@ -18,6 +18,7 @@
 #include "im2col.cuh"
 #include "quantize.cuh"
 #include "widen.cuh"
+#include "subpixel.cuh"
 
 using namespace mqc;
 
@@ -742,9 +743,71 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
 }
 
 // ------------------------------------------------------------------ input gradient
+// Input gradient of a strided convolution as one sub-pixel GEMM (see
+// subpixel.cuh): used when the stride phases number 2 to 4, tile the input
+// exactly (H, W multiples of the stride) and C is a multiple of 16 (columns
+// of one phase come in 16s).  Measured on the YOLOv8n layers (3x3, stride 2):
+// one launch with 4 x C columns instead of phase launches with C columns.
+struct SubpixPlan {
+    bool on = false;
+    SubpixGeom g{};
+    size_t codes_bytes = 0, scale_bytes = 0;
+};
+
+static SubpixPlan subpix_plan(const mqc_conv *c, const mqc_mx *wf) {
+    SubpixPlan sp;
+    const int sh = c->stride_h, sw = c->stride_w;
+    if (sh * sw < 2 || sh * sw > kMaxPhases || c->H % sh != 0 || c->W % sw != 0 || c->C % 16 != 0) return sp;
+    int dh0 = 1 << 30, dh1 = -(1 << 30), dw0 = 1 << 30, dw1 = -(1 << 30);
+    for (int a = 0; a < sh; ++a)
+        for (int r = 0; r < c->R; ++r) {
+            const int t = a + c->pad_h - r;
+            if ((t % sh + sh) % sh != 0) continue;
+            dh0 = std::min(dh0, t / sh);
+            dh1 = std::max(dh1, t / sh);
+        }
+    for (int a = 0; a < sw; ++a)
+        for (int s = 0; s < c->S; ++s) {
+            const int t = a + c->pad_w - s;
+            if ((t % sw + sw) % sw != 0) continue;
+            dw0 = std::min(dw0, t / sw);
+            dw1 = std::max(dw1, t / sw);
+        }
+    if (dh0 > dh1 || dw0 > dw1 || (dh1 - dh0 + 1) * (dw1 - dw0 + 1) > kMaxTaps) return sp;
+    int64_t Ap, Bp;
+    padded(wf->fmt, wf->order, c->C, c->K, Ap, Bp);
+    const int64_t kpw = wf->order == MQC_ORDER_BA ? Ap : Bp;
+    const bool sqw = wf->block == MQC_BLOCK_SQ32;
+    SubpixGeom &g = sp.g;
+    g.C = c->C;
+    g.Cs = sh * sw * c->C;
+    g.R = c->R;
+    g.S = c->S;
+    g.sh = sh;
+    g.sw = sw;
+    g.ph = c->pad_h;
+    g.pw = c->pad_w;
+    g.dh0 = dh0;
+    g.dw0 = dw0;
+    g.Rs = dh1 - dh0 + 1;
+    g.Ss = dw1 - dw0 + 1;
+    g.kpw = static_cast<int32_t>(kpw);
+    g.nkb = static_cast<int32_t>(nb32(kpw));
+    g.w_kb_pitch = static_cast<int32_t>(sqw ? nb32(c->C) : c->C);
+    g.w_tap_pitch = nb32(kpw) * g.w_kb_pitch;
+    g.w_row_shift = sqw ? 5 : 0;
+    const int64_t ntap = int64_t(g.Rs) * g.Ss;
+    sp.codes_bytes = static_cast<size_t>(round_up(ntap * g.Cs * kpw, 256));
+    sp.scale_bytes = static_cast<size_t>(round_up(ntap * g.nkb * g.Cs, 256));
+    sp.on = kpw % 16 == 0;
+    return sp;
+}
+
 size_t mqc_conv2d_bwd_data_workspace_bytes(const mqc_conv *c, const mqc_mx *wf, const mqc_mx *gf) {
     if (!conv_ok(c) || !mx_ok(wf) || !mx_ok(gf)) return 0;
-    return widened_bytes(wf, c->K, c->C, c->R, c->S) + widened_bytes(gf, c->N, c->K, conv_P(c), conv_Q(c));
+    const SubpixPlan sp = subpix_plan(c, wf);
+    return widened_bytes(wf, c->K, c->C, c->R, c->S) + widened_bytes(gf, c->N, c->K, conv_P(c), conv_Q(c)) +
+           (sp.on ? sp.codes_bytes + sp.scale_bytes : 0);
 }
 
 mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *wf, const void *gq, const uint8_t *gs,
@@ -770,6 +833,106 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
     const int64_t Kp = og.inner, Kpw = ow.inner;   // padded output-channel extents of G_Y and W rows
     const bool sqg = gf->block == MQC_BLOCK_SQ32, sqw = wf->block == MQC_BLOCK_SQ32;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    const SubpixPlan sp = subpix_plan(c, wf);
+    if (sp.on) {
+        if (ow.inner != sp.g.kpw) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_data: weight row padding mismatch");
+        uint8_t *scodes = wsp, *sscales = wsp + sp.codes_bytes;
+        const SubpixGeom &g = sp.g;
+        const int64_t work = (int64_t(g.Rs) * g.Ss * g.Cs * g.kpw) / 16 + int64_t(g.Rs) * g.Ss * g.nkb * g.Cs;
+        const int blocks = static_cast<int>(std::min<int64_t>(ceil_div(work, 256), int64_t(dv->sms) * 4));
+        subpix_weights_kernel<<<blocks, 256, 0, strm>>>(ow.codes, ws, scodes, sscales, g);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "subpix_weights_kernel launch");
+        const int ntap = g.Rs * g.Ss, Cs = g.Cs, Qs = W / sw, Ps = H / sh;
+        GemmParams G;
+        memset(&G, 0, sizeof G);
+        G.CB = static_cast<int32_t>(nb32(Kp));
+        G.wkb = largest_wkb(G.CB);
+        G.sub = 1;
+        choose_rows(Qs, Ps, N, G.bq, G.bp, G.bn);
+        G.BN = choose_bn(Cs);
+        G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
+        G.Ne = N;
+        G.TQ = static_cast<int32_t>(ceil_div(Qs, G.bq));
+        G.TP = static_cast<int32_t>(ceil_div(Ps, G.bp));
+        G.TN = static_cast<int32_t>(ceil_div(N, G.bn));
+        G.NT = static_cast<int32_t>(ceil_div(Cs, G.BN));
+        G.Ncols = Cs;
+        G.a_st_h = 1;
+        G.a_st_w = 1;
+        G.idesc = make_idesc_mx(mma_fmt(og.mma_fmt), mma_fmt(ow.mma_fmt), 128, G.BN);
+        st = MQC_ERR_CUDA;
+        for (int attempt = 0; attempt < 2 && st != MQC_OK; ++attempt) {
+            G.rows_nfirst = attempt;
+            if (!G.rows_nfirst) {
+                const uint64_t dims[4] = {uint64_t(Kp), uint64_t(Q), uint64_t(P), uint64_t(N)};
+                const uint64_t strd[3] = {uint64_t(N) * Kp, uint64_t(Q) * N * Kp, uint64_t(Kp)};
+                const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bq), uint32_t(G.bp), uint32_t(G.bn)};
+                st = encode_codes_map(&G.amap[0], og.codes, 4, dims, strd, box, G.wkb);
+            } else {
+                const uint64_t dims[4] = {uint64_t(Kp), uint64_t(N), uint64_t(Q), uint64_t(P)};
+                const uint64_t strd[3] = {uint64_t(Kp), uint64_t(N) * Kp, uint64_t(Q) * N * Kp};
+                const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bn), uint32_t(G.bq), uint32_t(G.bp)};
+                st = encode_codes_map(&G.amap[0], og.codes, 4, dims, strd, box, G.wkb);
+            }
+        }
+        if (st != MQC_OK) return st;
+        {
+            const uint64_t dims[3] = {uint64_t(Kpw), uint64_t(Cs), uint64_t(ntap)};
+            const uint64_t strd[2] = {uint64_t(Kpw), uint64_t(Cs) * Kpw};
+            const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(box_rows(Cs, G.BN)), 1u};
+            if ((st = encode_codes_map(&G.bmap[0], scodes, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
+        }
+        G.ntaps = ntap;
+        for (int t = 0; t < ntap; ++t) {
+            ConvTap &T = G.taps[t];
+            T.dh = T.sf_dh = static_cast<int16_t>(g.dh0 + t / g.Ss);
+            T.dw = T.sf_dw = static_cast<int16_t>(g.dw0 + t % g.Ss);
+            T.map = 0;
+            T.aw = 0;
+            T.btap = static_cast<int16_t>(t);
+        }
+        G.nph = 1;
+        G.ph_tap0[0] = 0;
+        G.ph_tkb[0] = ntap * G.CB;
+        G.ph_Pe[0] = Ps;
+        G.ph_Qe[0] = Qs;
+        G.ph_out_base[0] = 0;
+        G.n_amaps = 1;
+        G.n_bmaps = 1;
+        G.a_box_bytes = 32 * G.wkb * G.bq * G.bp * G.bn;
+        G.b_box_bytes = 32 * G.wkb * box_rows(Cs, G.BN);
+        G.a_slab = 128;
+        G.b_slab = G.BN;
+        G.sfa.base = gs;
+        G.sfa.pix_pitch = (sqg ? nb32(N) : N) * nb32(Kp);
+        G.sfa.row_shift = sqg ? 5 : 0;
+        G.sfa.row_pitch = static_cast<int32_t>(nb32(Kp));
+        G.sfa.kb_pitch = 1;
+        G.sfa.rows = N;
+        G.sfa.H = P;
+        G.sfa.W = Q;
+        G.sfb.base = sscales;
+        G.sfb.tap_pitch = int64_t(g.nkb) * Cs;
+        G.sfb.row_shift = 0;
+        G.sfb.row_pitch = 1;
+        G.sfb.kb_pitch = Cs;
+        G.sfb.rows = Cs;
+        G.sf_vec4 = G.CB % 4 == 0 && G.sfa.pix_pitch % 4 == 0 && G.sfa.row_pitch % 4 == 0 &&
+                    (reinterpret_cast<uintptr_t>(gs) & 3u) == 0;
+        G.sfb_vec4 = false;
+        G.out = gx;
+        G.os_q = sw;
+        G.os_p = int64_t(sh) * W;
+        G.os_n = int64_t(C) * H * W;
+        G.os_c = int64_t(H) * W;
+        G.d2s = 1;
+        G.cpad = C;
+        for (int a = 0; a < sh; ++a)
+            for (int b = 0; b < sw; ++b) G.d2s_off[a * sw + b] = int64_t(a) * W + b;
+        G.num_units = G.TQ * G.TP * G.TN * G.NT;
+        return launch_gemm<kConv>(G, *dv, strm);
+    }
     // output stride phases (ah, aw) with at least one row; the first one has
     // the largest extents and sets the tiling shared by a launch
     if (sh > 64 || sw > 64) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_data: stride above 64");

@@ -150,8 +150,9 @@ MQC_API int64_t mqc_im2col_cbf_codes_bytes(const mqc_conv *conv, const mqc_mx *m
  * workspace, as the E4M3 codes of the same values (every E2M1 value is an
  * E4M3 value; same layout, one byte per element); the products and the
  * scales are unchanged.  Each GEMM has a *_workspace_bytes query: 0 when no
- * operand is E2M1 (and, for the weight gradient, no split-K partials are
- * needed), in which case workspace may be NULL.  The workspace must be
+ * operand is E2M1 (and, for the input gradient, the sub-pixel plan does not
+ * apply; for the weight gradient, no split-K partials are needed), in which
+ * case workspace may be NULL.  The workspace must be
  * 16-byte aligned; it is scratch, overwritten by the call.
  *
  * Forward convolution, Eq. 1, as the block-scaled GEMM
@@ -171,10 +172,17 @@ MQC_API size_t mqc_conv2d_fwd_workspace_bytes(const mqc_conv *conv, const mqc_mx
 
 /* Input gradient, Eq. 2: G_X = W^T * G_Y as the GEMM
  * G_X'{Cin,N} = W_f^T . G_Yf{Cout,N} of section IV-B, computed directly as a
- * transposed convolution: one implicit GEMM per output stride phase, up to
- * four phases per kernel launch, their tiles interleaved so that the
- * phases' outputs (which interleave in memory) are written together; no
- * G_X' is materialized.  stride_h * stride_w must be at most 64.
+ * transposed convolution; no G_X' is materialized.  When the stride phases
+ * number 2 to 4, H and W are multiples of the strides and C is a multiple of
+ * 16: ONE sub-pixel GEMM whose rows are the super-pixels (n, i, j) (input
+ * pixels sh*i+ah, sw*j+aw for every phase (ah, aw)) and whose columns are
+ * (phase, c), reducing over the few G_Y pixels (i+dh, j+dw) any phase
+ * reaches; its weights (W's codes and scales rearranged per (dh, dw), zero
+ * where no kernel tap links an offset to a phase) are built in the workspace
+ * first, and the results are stored depth-to-space.  Otherwise one implicit
+ * GEMM per output stride phase, up to four phases per kernel launch, their
+ * tiles interleaved so that the phases' outputs (which interleave in memory)
+ * are written together.  stride_h * stride_w must be at most 64.
  *   wq, ws  W quantized with blocks along K: block B32 or SQ32, order AB.
  *   gq, gs  G_Y quantized with blocks along K: block A32 or SQ32, order BA.
  *   gx      fp32 output [N][C][H][W] (overwritten).

@@ -99,7 +99,8 @@ def test_invalid_arguments_rejected_before_launch(mqc):
 def test_gemm_workspace_sizes_cover_widened_fp4_operands(mqc):
     """E2M1 GEMM operands are widened to one byte per element in the caller's
     workspace: the size queries give twice the packed code bytes (rounded up
-    to 256), and nothing for FP8 operands."""
+    to 256), and nothing for FP8 operands unless the input gradient runs as a
+    sub-pixel GEMM (its window weights)."""
     cv = mqc.conv_desc(4, 40, 9, 11, 24, 3, 3, 2, 1)
     P, Q = (9 + 2 - 3) // 2 + 1, (11 + 2 - 3) // 2 + 1
     fp8_a, fp4_a = mqc.MX(0, 2, 0), mqc.MX(2, 2, 0)
@@ -110,5 +111,10 @@ def test_gemm_workspace_sizes_cover_widened_fp4_operands(mqc):
     assert mqc.mqc_conv2d_fwd_workspace_bytes(cv, fp4_a, fp4_a) == (r(mqc.mqc_codes_bytes(fp4_a, 4, 40, 9, 11))
                                                                      + r(mqc.mqc_codes_bytes(fp4_a, 24, 40, 3, 3)))
     assert mqc.mqc_conv2d_bwd_data_workspace_bytes(cv, fp8_b, fp8_a) == 0
+    # sub-pixel input gradient (C = 32, even H and W, stride 2): the window
+    # weights, 2 x 2 offsets x (4 phases x 32 channels) rows of 48 code bytes,
+    # and their scales, 2 K-blocks per row
+    sub = mqc.conv_desc(2, 32, 8, 8, 48, 3, 3, 2, 1)
+    assert mqc.mqc_conv2d_bwd_data_workspace_bytes(sub, fp8_b, fp8_a) == 4 * 128 * 48 + (4 * 2 * 128 + 255) // 256 * 256
     assert mqc.mqc_conv2d_bwd_data_workspace_bytes(cv, fp4_b, fp4_a) == (r(mqc.mqc_codes_bytes(fp4_b, 24, 40, 3, 3))
                                                                           + r(mqc.mqc_codes_bytes(fp4_a, 4, 24, P, Q)))

@@ -94,6 +94,15 @@ DGRAD_CASES = BWD_CASES + [
     (3, 16, 13, 12, 32, 5, 5, 2, 2),
     (2, 64, 7, 9, 160, 3, 3, 2, 1),
 ]
+# the sub-pixel GEMM (stride 2, even H and W, C in 16s): phases no tap reaches
+# (1x1), a 3x3 window of offsets (5x5), column tiles that split the phases
+# (C = 48, 192 columns) with ragged K, a 4x4 kernel
+DGRAD_CASES += [
+    (4, 32, 10, 8, 32, 1, 1, 2, 0),
+    (3, 16, 12, 10, 32, 5, 5, 2, 2),
+    (2, 48, 6, 8, 40, 3, 3, 2, 1),
+    (2, 16, 8, 8, 32, 4, 4, 2, 1),
+]
 
 
 @pytest.mark.parametrize("case", DGRAD_CASES)

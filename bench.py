@@ -252,11 +252,15 @@ class LayerBuffers:
 
     def launches(self, mqc):
         """Kernels one pass of this layer launches: 3 quantizations, the
-        forward GEMM, the input gradient (its stride phases share launches of
-        up to 4 height phases), the weight-gradient GEMM and, with split-K
-        partials, their reduction."""
+        forward GEMM, the input gradient (as one sub-pixel GEMM after the
+        kernel that builds its window weights when the 2 to 4 stride phases
+        tile the input and C is a multiple of 16; else its stride phases
+        share launches of up to 4 height phases), the weight-gradient GEMM
+        and, with split-K partials, their reduction."""
         L = self.L
-        return 3 + 1 + -(-L.stride // 4) + (2 if self.split_k else 1) + self.n_widen
+        subpix = 2 <= L.stride * L.stride <= 4 and L.H % L.stride == 0 and L.W % L.stride == 0 and L.C % 16 == 0
+        dgrad = 2 if subpix else -(-L.stride // 4)
+        return 3 + 1 + dgrad + (2 if self.split_k else 1) + self.n_widen
 
 
 def run_layer(mqc, lb: LayerBuffers, workspace, stream, events=None, only=None):

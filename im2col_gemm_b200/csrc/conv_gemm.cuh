@@ -40,9 +40,13 @@ constexpr int kMaxTaps = 64;
 constexpr int kMaxPhases = 4;   // CONV: output stride phases sharing one launch
 constexpr int kGemmThreads = 384;
 // Warp roles (a warp's SM sub-partition is its index modulo 4):
-//   0 TMA producer, 1 MMA issuer (alone on its sub-partition apart from one
-//   epilogue warp), 4-7 epilogue (one per TMEM lane quadrant), and the
+//   0 TMA producer, 1 MMA issuer (alone on its sub-partition apart from the
+//   epilogue warps), 4-7 epilogue (one per TMEM lane quadrant), and the
 //   scale-factor gather warps below; warp 9 only joins the final barrier.
+//   CONV kernels have 16 warps: 12-15 are a second epilogue team, the two
+//   teams taking alternate accumulators (when there are at least two).
+template <int KIND>
+__host__ __device__ constexpr int gemm_threads() { return KIND == 0 ? 512 : kGemmThreads; }
 constexpr int kNumSfWarps = 5;
 __device__ __forceinline__ int sf_warp_index(int warp) {
     return warp == 2 ? 0 : warp == 3 ? 1 : warp == 8 ? 2 : warp == 10 ? 3 : warp == 11 ? 4 : -1;
@@ -298,7 +302,7 @@ struct KitWalker {
 // A template parameter as well, so that the one-tile kernel carries no
 // sub-tile loops.
 template <int KIND, bool SFV4, int UMT>
-__global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -361,7 +365,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         // every thread helps build the B scale atoms once: item = (column tile,
         // group of 4 K-blocks, atom); lane l writes rows l, l+32, l+64, l+96
         const int items = p.NT * p.groups * p.nb_atoms;
-        for (int item = warp; item < items; item += kGemmThreads / 32) {
+        for (int item = warp; item < items; item += gemm_threads<KIND>() / 32) {
             const int at = item % p.nb_atoms;
             const int gq = (item / p.nb_atoms) % p.groups;
             const int nt = item / (p.nb_atoms * p.groups);
@@ -387,7 +391,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
         fence_proxy_async_smem();
     }
     if (p.k16) {
-        for (int i = threadIdx.x; i < 4096 / 16; i += kGemmThreads)
+        for (int i = threadIdx.x; i < 4096 / 16; i += gemm_threads<KIND>())
             reinterpret_cast<uint4 *>(sZ)[i] = make_uint4(0u, 0u, 0u, 0u);
         fence_proxy_async_smem();
     }
@@ -873,12 +877,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                 }
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if ((warp >= 4 && warp < 8) || (KIND == kConv && warp >= 12)) {
         // ------------------------------------------------------------ epilogue
         const int qd = warp & 3;               // TMEM lane quadrant of this warp
         const int m = qd * 32 + lane;
+        const int team = warp >= 12 ? 1 : 0;   // team t: accumulators t, t + 2 (tiles t modulo 2)
+        const int nteams = KIND == kConv && p.nacc >= 2 ? 2 : 1;
         uint32_t tcount = 0;
-        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+        for (int u = blockIdx.x; u < p.num_units && team < nteams; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
             // output row of this thread in sub-tile i
             bool row_ok;
@@ -900,6 +906,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
             };
             const bool tap_cols = KIND == kWgrad && p.ntg > 1;   // columns are (tap, channel)
             if (I.nk == 0) {
+                if (team != 0) continue;
                 for (int i = 0; i < UM; ++i) {
                     set_row(i);
                     if (row_ok)
@@ -916,6 +923,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) conv_gemm_kernel(const __grid
                             }
                         }
                 }
+                continue;
+            }
+            if (nteams == 2 && static_cast<int>(tcount & 1u) != team) {
+                ++tcount;
                 continue;
             }
             const uint32_t acc = tcount & static_cast<uint32_t>(p.nacc - 1);

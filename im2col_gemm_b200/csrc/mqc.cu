@@ -314,7 +314,7 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
         const_cast<DevInfo &>(d).gemm_attr[ai] = true;
     }
     const int grid = std::max(1, std::min(P.num_units, d.sms));
-    kernel<<<grid, kGemmThreads, smem, stream>>>(P);
+    kernel<<<grid, gemm_threads<KIND>(), smem, stream>>>(P);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "conv_gemm_kernel launch");
     return MQC_OK;

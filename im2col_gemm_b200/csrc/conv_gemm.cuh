@@ -882,7 +882,9 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
         const int qd = warp & 3;               // TMEM lane quadrant of this warp
         const int m = qd * 32 + lane;
         const int team = warp >= 12 ? 1 : 0;   // team t: accumulators t, t + 2 (tiles t modulo 2)
-        const int nteams = KIND == kConv && p.nacc >= 2 ? 2 : 1;
+        // one team for the depth-to-space stores (their half-sector writes
+        // measured slower with twice as many in flight)
+        const int nteams = KIND == kConv && p.nacc >= 2 && !p.d2s ? 2 : 1;
         uint32_t tcount = 0;
         for (int u = blockIdx.x; u < p.num_units && team < nteams; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);

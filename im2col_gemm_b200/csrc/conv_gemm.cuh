@@ -148,7 +148,9 @@ struct alignas(64) GemmParams {
     int32_t k16;
     // CONV d2s (input gradient as one sub-pixel GEMM): GEMM column n is
     // (phase n / cpad, channel n % cpad) and lands at channel offset
-    // (n % cpad) * os_c + d2s_off[phase]; cpad is a multiple of 16
+    // (n % cpad) * os_c + d2s_off[phase]; cpad is a multiple of 16.
+    // d2s = 2: width stride 2 and column tiles of whole phase pairs
+    // (aw = 0, 1): the two are stored together, 8 bytes per lane
     int32_t d2s;
     int64_t d2s_off[kMaxPhases];
     // the divisions of the unit and row decoding, by launch constants
@@ -944,6 +946,35 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                 set_row(i);
                 const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16) + (acc * UM + i) * p.BN;
                 float *orow = p.out + row_off;
+                if (KIND == kConv && p.d2s == 2) {
+                    // 16 channels of a phase pair (aw = 0, 1) per pass: column
+                    // pa and pa + cpad, stored together as 8-byte pairs
+                    for (int c0 = 0; c0 < p.BN; c0 += 32) {
+                        uint32_t r[32];
+                        const int q = c0 >> 5, nblk = p.cpad >> 4;   // 16-channel blocks of a phase
+                        const int pp = q / nblk;
+                        const int pc = (q - pp * nblk) << 4;
+                        const int pa = 2 * pp * p.cpad + pc;
+                        tc_ld_32x32b_x16p(t_row + pa, r);
+                        tc_ld_32x32b_x16p(t_row + pa + p.cpad, r + 16);
+                        tc_wait_ld();
+                        if (i + 1 == UM && c0 + 32 >= p.BN) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                        }
+                        const int n0 = I.col0 + pa;
+                        if (row_ok && n0 < p.Ncols) {
+                            const int ph = static_cast<int>(p.fd_cpad.div(n0));
+                            float *op = orow + static_cast<int64_t>(pc) * p.os_c + p.d2s_off[ph];
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj)
+                                *reinterpret_cast<float2 *>(op + jj * p.os_c) =
+                                    make_float2(__uint_as_float(r[jj]), __uint_as_float(r[16 + jj]));
+                        }
+                    }
+                    continue;
+                }
                 for (int c0 = 0; c0 < p.BN; c0 += 32) {
                     uint32_t r[32];
                     tc_ld_32x32b_x32(t_row + c0, r);

@@ -926,7 +926,8 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
         G.os_p = int64_t(sh) * W;
         G.os_n = int64_t(C) * H * W;
         G.os_c = int64_t(H) * W;
-        G.d2s = 1;
+        // width phases stored in pairs when the column tiles hold whole pairs
+        G.d2s = sw == 2 && G.BN % (2 * C) == 0 && (reinterpret_cast<uintptr_t>(gx) & 7u) == 0 ? 2 : 1;
         G.cpad = C;
         for (int a = 0; a < sh; ++a)
             for (int b = 0; b < sw; ++b) G.d2s_off[a * sw + b] = int64_t(a) * W + b;

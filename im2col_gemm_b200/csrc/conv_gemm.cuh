@@ -1025,13 +1025,20 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-// Deterministic split-K reduction: out[i] = sum over s (in order) of part[s][i].
+// Deterministic split-K reduction: out[i] = the sum of part[s][i] over s in a
+// fixed order: eight running sums (s modulo 8, each in increasing s, so
+// eight loads are in flight per thread), then combined pairwise.
 __global__ void splitk_reduce_kernel(const float *__restrict__ part, float *__restrict__ out, int64_t n, int splits) {
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        float acc = 0.0f;
-        for (int s = 0; s < splits; ++s) acc += part[s * n + i];
-        out[i] = acc;
+        float a[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+        int s = 0;
+        for (; s + 8 <= splits; s += 8) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) a[k] += __ldg(part + (s + k) * n + i);
+        }
+        for (int k = 0; s < splits; ++s, ++k) a[k] += __ldg(part + s * n + i);
+        out[i] = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
     }
 }
 

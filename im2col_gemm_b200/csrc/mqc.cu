@@ -1287,8 +1287,8 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     if ((st = launch_gemm<kWgrad>(G, *dv, strm)) != MQC_OK) return st;
     if (G.splits > 1) {
         const int64_t n = int64_t(K) * C * R * S;
-        const int blocks = static_cast<int>(std::min<int64_t>(ceil_div(n, 256), int64_t(dv->sms) * 8));
-        splitk_reduce_kernel<<<blocks, 256, 0, strm>>>(static_cast<const float *>(workspace), gw, n, G.splits);
+        const int blocks = static_cast<int>(std::min<int64_t>(ceil_div(n, 128), int64_t(dv->sms) * 16));
+        splitk_reduce_kernel<<<blocks, 128, 0, strm>>>(static_cast<const float *>(workspace), gw, n, G.splits);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "splitk_reduce_kernel launch");
     }

@@ -331,6 +331,15 @@ def oracle_sample(wl: synth.Workload, n_images: int = 1, layers=None):
     return flops, t_total, orc.num_threads(), desc
 
 
+def arm_config(wl, world):
+    """The `config` object both arms print: the workload, its sizes and formats."""
+    L0 = wl.layers[0]
+    return {"workload": wl.name, "layers": len(wl.layers), "global_batch": L0.N * world,
+            "input": f"{L0.C}x{L0.H}x{L0.W}", "block": "SQ32", "formats": "X,W e4m3; G_Y e5m2",
+            "l2": "inputs larger than L2 (step working set well above 126 MB); no flush",
+            "parallelism": f"dp{world}"}
+
+
 def reference_arm(args):
     world, rank, local = dist_env()
     if rank != 0:
@@ -350,7 +359,7 @@ def reference_arm(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(1, len(secs)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "sample": desc},
+        "config": dict(arm_config(wl, world), sample=desc),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -624,11 +633,7 @@ def main(argv=None):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "mxfp8 (e4m3/e5m2 x e8m0) -> fp32", "data": "synthetic",
-            "config": {"workload": wl.name, "layers": len(layers), "global_batch": wl.layers[0].N * world,
-                       "input": f"{wl.layers[0].C}x{wl.layers[0].H}x{wl.layers[0].W}",
-                       "block": "SQ32", "formats": "X,W e4m3; G_Y e5m2",
-                       "l2": "inputs larger than L2 (step working set well above 126 MB); no flush",
-                       "parallelism": f"dp{world}"},
+            "config": arm_config(wl, world),
             "quantizer_gbs": quant_gbs, "quantizer_frac_of_hbm": quant_gbs / pk["hbm_gbs"],
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,

@@ -96,6 +96,17 @@ def barrier():
         dist.barrier()
 
 
+def allreduce_weight_grads(tensors):
+    """The data-parallel exchange of the step: every rank's weight gradients
+    (partial sums over its own batch shard) are summed over the ranks in
+    place, so each rank ends with the gradient of the whole global batch.
+    The only collective of the path; nothing when running alone."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        for t in tensors:
+            dist.all_reduce(t, op=dist.ReduceOp.SUM)
+
+
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -489,10 +500,7 @@ def main(argv=None):
     gws = [lb.gw for lb in layers]
 
     def allreduce_gw():
-        import torch.distributed as dist
-        if world > 1:
-            for t in gws:
-                dist.all_reduce(t)
+        allreduce_weight_grads(gws)
 
     def cur_stream():
         return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)

@@ -16,10 +16,14 @@
 //         A tile of a tap is one TMA box of the activation tensor at shifted
 //         coordinates (out-of-range rows are zero-filled: the padding);
 //         strided convolutions use one tensor map per stride phase.
-//   WGRAD (weight gradient): rows = C_out, columns = C_in of one tap,
-//         reduction = (output pixel, batch) with N contiguous; split over K.
+//         The input gradient of a strided convolution can also run as one
+//         sub-pixel GEMM: rows = super-pixels, columns = (stride phase,
+//         channel), stored depth-to-space (d2s below).
+//   WGRAD (weight gradient): rows = C_out, columns = C_in of one tap or
+//         (tap, C_in) of a tap group, reduction = (output pixel, batch) with
+//         N contiguous; split over K.
 //
-// CTA layout (persistent, one CTA per SM, 12 warps):
+// CTA layout (persistent, one CTA per SM; 16 warps for CONV, 12 for WGRAD):
 //   warp 0      TMA producer (codes of A and B, one elected thread)
 //   warp 1      TMEM allocator + MMA issuer (one elected thread): scale
 //               factors smem -> TMEM with tcgen05.cp, then tcgen05.mma
@@ -28,6 +32,7 @@
 //               row and K-block into the 128x4 shared-memory atoms the MMA
 //               expects (one stage per warp in turn)
 //   warps 4-7   epilogue: TMEM -> registers -> fp32 global stores
+//   warps 12-15 (CONV) a second epilogue team, alternate accumulators
 // Every wait is bounded in time; a wait that runs out records a device error
 // and the CTA winds down without hanging.
 #pragma once

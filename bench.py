@@ -447,7 +447,34 @@ def sweep(mqc, torch, wl, args):
                         "gbs": round(byt / (ms * 1e-3) / 1e9, 1),
                         "frac_of_roofline": round(1e3 * t_roof / ms, 4),
                         "frac_of_mxfp8_peak": round(fl / (ms * 1e-3) / 1e12 / fp8_peak, 4) if fl else None})
-        del lb, workspace
+        # the explicit channel-batch-first im2col of quantized X (the GEMMs
+        # never call it): HBM-bound, source codes + scales read once and the
+        # expansion written once, timed after a 256 MiB L2 flush
+        xq = lb.q["x"]
+        nc = mqc.lib.mqc_im2col_cbf_codes_bytes(ctypes.byref(lb.cv), ctypes.byref(xq.mx))
+        ns = mqc.lib.mqc_im2col_cbf_scales_bytes(ctypes.byref(lb.cv), ctypes.byref(xq.mx))
+        co = torch.empty(max(nc, 16), dtype=torch.uint8, device="cuda")
+        so = torch.empty(max(ns, 16), dtype=torch.uint8, device="cuda")
+        ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+        call = lambda: mqc.check(mqc.mqc_im2col_cbf(ptr(xq.codes), ptr(xq.scales), lb.cv, xq.mx, ptr(co), ptr(so),
+                                                   stream))
+        call()
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        ts = []
+        for _ in range(max(3, args.reps)):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        byt = xq.codes.numel() + xq.scales.numel() + nc + ns
+        out.append({"workload": wl.name, "layer": i, "call": "im2col_x", "ms": round(ms, 5), "tflops": None,
+                    "gbs": round(byt / (ms * 1e-3) / 1e9, 1),
+                    "frac_of_roofline": round(byt / (pk["hbm_gbs"] * 1e9) * 1e3 / ms, 4), "frac_of_mxfp8_peak": None})
+        del lb, workspace, co, so, flush
         torch.cuda.empty_cache()
     for o in out:
         print(json.dumps(o), flush=True)

@@ -148,6 +148,102 @@ def test_layout_hand_worked_example(orc):
             assert np.array_equal(scales, exp_s)
 
 
+def test_block_modes_hand_worked_example(orc):
+    """B32 and SQ32 (and A32) on tensors with more than 32 elements along both
+    blocked axes and a short block of 16, both code orders, E4M3 / E5M2 /
+    E2M1: every code and scale byte worked out by hand (golden file)."""
+    g = gold("layout_blocks_example.json")
+    tensors = {}
+    for name, t in g["tensors"].items():
+        x = np.zeros(t["shape"], dtype=np.float32)
+        for b, a, v in t["x_nonzero"]:
+            x[b, a, 0, 0] = v
+        tensors[name] = x
+    for case in g["cases"]:
+        x = tensors[case["tensor"]]
+        codes, scales = orc.quantize(x, FMTS[case["fmt"]], BLOCKS[case["block"]], ORDERS[case["order"]])
+        assert codes.size == case["codes_len"], case["why"]
+        exp = np.zeros(case["codes_len"], dtype=np.uint8)
+        for k, v in case["codes_nonzero"].items():
+            exp[int(k)] = v
+        assert np.array_equal(codes, exp), case["why"]
+        if "scales" in case:
+            assert list(scales) == case["scales"], case["why"]
+        else:
+            exp_s = np.zeros(case["scales_len"], dtype=np.uint8)
+            for k, v in case["scales_nonzero"].items():
+                exp_s[int(k)] = v
+            assert np.array_equal(scales, exp_s), case["why"]
+
+
+def _numpy_blocks_reference(x, fmt, block, order):
+    """Codes and scales of the block modes built another way than the oracle:
+    blocks are numpy reshapes of the zero-padded tensor, the exponent comes
+    from np.frexp of each block's maximum, the codes from torch's saturating
+    float8 cast of x / 2^e, and the layout from transposes (no index formula).
+    Section IV-B directions: A32 blocks run along d1, B32 along d0, SQ32 are
+    32 x 32 squares over (d0, d1)."""
+    tdt = {0: torch.float8_e4m3fn, 1: torch.float8_e5m2}[fmt]
+    emax = {0: 8, 1: 15}[fmt]
+    vmax = {0: 448.0, 1: 57344.0}[fmt]
+    B, A, H, W = x.shape
+    Bq, Aq = -(-B // 32) * 32, -(-A // 32) * 32
+    xp = np.zeros((Bq, Aq, H, W), dtype=np.float64)
+    xp[:B, :A] = x
+    if block == 2:
+        amax = np.abs(xp.reshape(Bq // 32, 32, Aq // 32, 32, H, W)).max(axis=(1, 3))   # [bb][ab][h][w]
+        per_elem = lambda e: np.repeat(np.repeat(e, 32, axis=0), 32, axis=1)
+    elif block == 1:
+        amax = np.abs(xp.reshape(Bq // 32, 32, Aq, H, W)).max(axis=1)                  # [bb][a][h][w]
+        per_elem = lambda e: np.repeat(e, 32, axis=0)
+    else:
+        amax = np.abs(xp.reshape(Bq, Aq // 32, 32, H, W)).max(axis=2)                  # [b][ab][h][w]
+        per_elem = lambda e: np.repeat(e, 32, axis=1)
+    _, ex = np.frexp(amax)                                  # amax = f * 2^ex, f in [0.5, 1)
+    e = np.clip(ex - 1 - emax, -127, 127)
+    sc = np.where(amax == 0, 0, e + 127).astype(np.uint8)
+    ee = per_elem(np.where(amax == 0, -127, e))[:B, :A]
+    v = np.clip(x.astype(np.float64) * np.exp2(-ee), -vmax, vmax).astype(np.float32)
+    codes8 = torch.from_numpy(v).to(tdt).view(torch.uint8).numpy()                   # [B][A][H][W]
+    row = 16
+    if order == 0:
+        Ap = -(-A // row) * row
+        lay = np.zeros((H, W, B, Ap), dtype=np.uint8)
+        lay[..., :A] = codes8.transpose(2, 3, 0, 1)
+    else:
+        Bp = -(-B // row) * row
+        lay = np.zeros((H, W, A, Bp), dtype=np.uint8)
+        lay[..., :B] = codes8.transpose(2, 3, 1, 0)
+    # scales over the layout's extents (the padded innermost extent is at most
+    # the 32-padded one, so slicing keeps exactly the blocks the layout has)
+    if block == 2:
+        s = sc.transpose(2, 3, 0, 1)                                               # [h][w][bb][ab]
+    elif block == 1:
+        Ap = -(-A // row) * row if order == 0 else A
+        s = sc[:, :Ap].transpose(2, 3, 0, 1)                                       # [h][w][bb][a]
+    else:
+        Bp = -(-B // row) * row if order == 1 else B
+        s = sc[:Bp].transpose(2, 3, 0, 1)                                          # [h][w][b][ab]
+    return lay.reshape(-1), s.reshape(-1)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("block", [0, 1, 2])
+@pytest.mark.parametrize("order", [0, 1])
+@pytest.mark.parametrize("shape", [(40, 72, 2, 3), (16, 40, 3, 2), (70, 33, 1, 2)])
+def test_block_modes_match_numpy_blocks_and_torch_cast(orc, fmt, block, order, shape):
+    x = synth.random_tensor(shape, seed=31 + 7 * block + order, dist="student_t")
+    # give each 32 x 32 square its own magnitude so that mixing blocks changes scales
+    B, A = shape[0], shape[1]
+    for bb in range(-(-B // 32)):
+        for ab in range(-(-A // 32)):
+            x[32 * bb:32 * bb + 32, 32 * ab:32 * ab + 32] *= np.float32(2.0 ** (3 * bb - 5 * ab))
+    codes, scales = orc.quantize(x, fmt, block, order)
+    ref_codes, ref_scales = _numpy_blocks_reference(x, fmt, block, order)
+    assert np.array_equal(scales, ref_scales)
+    assert np.array_equal(codes, ref_codes)
+
+
 def _quant_error_bound(orc, fmt, x, xq, e_of_elem):
     """|x - dequant| <= half an ulp of the top binade at the block scale, or the
     saturation gap for elements beyond the largest finite value."""

@@ -72,6 +72,13 @@ def lib():
         L.oracle_im2col_counts.argtypes = [i64] * 10 + [vp]
         L.oracle_im2col_counts.restype = i64
         L.oracle_num_threads.restype = i32
+        u64, u32 = ctypes.c_uint64, ctypes.c_uint32
+        L.oracle_philox4x64.argtypes = [vp, vp, vp]
+        L.oracle_sr_bits.argtypes = [u64, u64, i64, i64, i64, i64, i64]
+        L.oracle_sr_bits.restype = u32
+        L.oracle_encode_sr.argtypes = [i32, dbl, u32]
+        L.oracle_encode_sr.restype = i32
+        L.oracle_quantize_sr.argtypes = [vp, i64, i64, i64, i64, vp, i32, i32, i32, u64, u64, vp, vp]
         _lib = L
     return _lib
 
@@ -141,6 +148,51 @@ def quantize(x: np.ndarray, fmt: int, block: int, order: int) -> tuple[np.ndarra
     scales = np.zeros(scales_bytes(fmt, block, order, d0, d1, d2, d3), dtype=np.uint8)
     lib().oracle_quantize(_p(x), d0, d1, d2, d3, _p(strides), fmt, block, order, _p(codes), _p(scales))
     return codes, scales
+
+
+def philox4x64(ctr, key) -> np.ndarray:
+    """One Philox4x64-10 block (four uint64 words) for a counter and a key."""
+    c = np.ascontiguousarray(ctr, dtype=np.uint64)
+    k = np.ascontiguousarray(key, dtype=np.uint64)
+    out = np.zeros(4, dtype=np.uint64)
+    lib().oracle_philox4x64(_p(c), _p(k), _p(out))
+    return out
+
+
+def sr_bits(seed, offset, B, A, pix, b, a) -> int:
+    """The 16 random bits stochastic rounding uses for element (pix, b, a)."""
+    return int(lib().oracle_sr_bits(seed, offset, B, A, pix, b, a))
+
+
+def encode_sr(fmt: int, v: float, r: int) -> int:
+    return int(lib().oracle_encode_sr(fmt, float(v), int(r)))
+
+
+def quantize_sr(x: np.ndarray, fmt: int, block: int, order: int, seed: int, offset: int = 0):
+    """MX quantization with stochastically rounded elements: (codes, scales)."""
+    assert x.dtype == np.float32 and x.ndim == 4
+    d0, d1, d2, d3 = x.shape
+    strides = np.array([s // 4 for s in x.strides], dtype=np.int64)
+    codes = np.zeros(codes_bytes(fmt, order, d0, d1, d2, d3), dtype=np.uint8)
+    scales = np.zeros(scales_bytes(fmt, block, order, d0, d1, d2, d3), dtype=np.uint8)
+    lib().oracle_quantize_sr(_p(x), d0, d1, d2, d3, _p(strides), fmt, block, order, seed, offset, _p(codes),
+                             _p(scales))
+    return codes, scales
+
+
+ACT_NONE, ACT_RELU, ACT_SILU = 0, 1, 2
+
+
+def activation(y: np.ndarray, act: int) -> np.ndarray:
+    """The activation a layer applies to its convolution output before the
+    result is quantized as the next layer's input (the paper's section V and
+    Fig. 4 flow): none, ReLU max(y, 0), or SiLU y / (1 + exp(-y)), in float64."""
+    y = np.asarray(y, dtype=np.float64)
+    if act == ACT_RELU:
+        return np.maximum(y, 0.0)
+    if act == ACT_SILU:
+        return y / (1.0 + np.exp(-y))
+    return y
 
 
 def dequantize(codes, scales, shape, fmt, block, order) -> np.ndarray:

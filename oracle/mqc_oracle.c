@@ -30,6 +30,9 @@
  *   - Direct convolution forward (Eq. 1), input gradient (Eq. 2) and weight
  *     gradient (Eq. 3), as cross-correlation with stride and zero padding,
  *     each also returning sum |a*b| of its dot product.
+ *   - Stochastic rounding of the elements (section III-A, Eq. 6: the
+ *     gradients are rounded stochastically), with random bits from the
+ *     Philox4x64-10 counter-based generator (Salmon et al., SC 2011).
  *   - The per-element quantization-count and stored-bytes model behind
  *     Table I (section IV-C).
  */
@@ -275,6 +278,120 @@ void oracle_quantize(const float *src, int64_t d0, int64_t d1, int64_t d2, int64
                     for (int64_t a = a0; a < a1; ++a) {
                         double x = src_at(src, d0, d1, strides, b, a, h, w);
                         int code = oracle_encode(fmt, x * inv);
+                        put_code(codes, fmt, code_index(order, pix, b, a, Ap, Bp), code);
+                    }
+            }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Stochastic rounding (paper, section III-A, Eq. 6 and the text after it:    */
+/* gradients are rounded stochastically, activations and weights to nearest) */
+/* ------------------------------------------------------------------------ */
+/* Philox4x64-10, the counter-based generator of Salmon, Moraes, Dror and
+ * Shaw ("Parallel random numbers: as easy as 1, 2, 3", SC 2011): ten rounds
+ * of two 64x64->128-bit multiplications with the published multipliers
+ * and Weyl key increments.  out[i] is word i of the block for (ctr, key). */
+static void mulhilo64(uint64_t a, uint64_t b, uint64_t *hi, uint64_t *lo)
+{
+    unsigned __int128 p = (unsigned __int128)a * b;
+    *hi = (uint64_t)(p >> 64);
+    *lo = (uint64_t)p;
+}
+
+void oracle_philox4x64(const uint64_t ctr[4], const uint64_t key[2], uint64_t out[4])
+{
+    uint64_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint64_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) { k0 += 0x9E3779B97F4A7C15ull; k1 += 0xBB67AE8584CAA73Bull; }
+        uint64_t h0, l0, h1, l1;
+        mulhilo64(0xD2E7470EE14C6C93ull, c0, &h0, &l0);
+        mulhilo64(0xCA5A826395121157ull, c2, &h1, &l1);
+        uint64_t n0 = h1 ^ c1 ^ k0, n1 = l1, n2 = h0 ^ c3 ^ k1, n3 = l0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* The 16 random bits of element (pix, b, a) of a tensor with extents
+ * (d0 = B, d1 = A): element index i = ((pix*B + b)*A16 + a) with A16 = A
+ * rounded up to 16, Philox block i / 16 (counter (i / 16, offset, 0, 0),
+ * key (seed, 0)), bits 16*(j % 4) .. +15 of word j / 4, j = i % 16. */
+uint32_t oracle_sr_bits(uint64_t seed, uint64_t offset, int64_t B, int64_t A, int64_t pix, int64_t b, int64_t a)
+{
+    int64_t A16 = (A + 15) / 16 * 16;
+    uint64_t i = (uint64_t)((pix * B + b) * A16 + a);
+    uint64_t ctr[4] = {i / 16, offset, 0, 0}, key[2] = {seed, 0}, out[4];
+    oracle_philox4x64(ctr, key, out);
+    int j = (int)(i % 16);
+    return (uint32_t)((out[j / 4] >> (16 * (j % 4))) & 0xFFFFu);
+}
+
+/* Stochastic rounding of a real value v to the element format with 16
+ * uniform random bits r: |v| lies between neighbouring finite magnitudes
+ * lo <= |v| < hi; with f = (|v| - lo) / (hi - lo), the magnitude becomes hi
+ * when r < f * 2^16 and lo otherwise (so hi with probability f, up to
+ * 2^-16).  Magnitudes at or beyond the largest finite value saturate to it;
+ * the sign is kept (also for zero). */
+int oracle_encode_sr(int fmt, double v, uint32_t r)
+{
+    const or_table *t = table_of(fmt);
+    int nb = fmt_bits(fmt);
+    if (v != v) return fmt == OR_E2M1 ? 0x7 : 0x7F;
+    int sign = signbit(v) ? 1 : 0;
+    double a = fabs(v);
+    int code;
+    if (a >= t->val[t->n - 1]) {
+        code = t->code[t->n - 1];
+    } else {
+        int lo = 0, hi = t->n - 1;                    /* val[lo] <= a < val[hi] */
+        while (hi - lo > 1) {
+            int mid = (lo + hi) / 2;
+            if (t->val[mid] <= a) lo = mid; else hi = mid;
+        }
+        double f = (a - t->val[lo]) / (t->val[hi] - t->val[lo]);
+        code = ((double)r < f * 65536.0) ? t->code[hi] : t->code[lo];
+    }
+    return (sign << (nb - 1)) | code;
+}
+
+/* MX quantization with stochastic rounding of the elements: the blocks and
+ * E8M0 scales are those of oracle_quantize (section III-A with the OCP
+ * scale), each element x*2^-e is rounded by oracle_encode_sr with the bits
+ * oracle_sr_bits gives for its position. */
+void oracle_quantize_sr(const float *src, int64_t d0, int64_t d1, int64_t d2, int64_t d3,
+                        const int64_t *strides, int fmt, int block, int order,
+                        uint64_t seed, uint64_t offset, uint8_t *codes, uint8_t *scales)
+{
+    int64_t Ap, Bp;
+    oracle_padded_extents(fmt, order, d1, d0, &Ap, &Bp);
+    int64_t nbytes = oracle_codes_bytes(fmt, order, d0, d1, d2, d3);
+    memset(codes, 0, (size_t)nbytes);
+    int64_t eb = (block == OR_A32) ? 1 : 32;
+    int64_t ea = (block == OR_B32) ? 1 : 32;
+    int64_t npix = d2 * d3;
+#pragma omp parallel for schedule(static)
+    for (int64_t pix = 0; pix < npix; ++pix) {
+        int64_t h = pix / d3, w = pix % d3;
+        for (int64_t b0 = 0; b0 < Bp; b0 += eb)
+            for (int64_t a0 = 0; a0 < Ap; a0 += ea) {
+                int64_t b1 = b0 + eb < Bp ? b0 + eb : Bp, a1 = a0 + ea < Ap ? a0 + ea : Ap;
+                double amax = 0.0;
+                for (int64_t b = b0; b < b1; ++b)
+                    for (int64_t a = a0; a < a1; ++a) {
+                        double x = fabs(src_at(src, d0, d1, strides, b, a, h, w));
+                        if (x > amax || x != x) amax = x;
+                    }
+                int sc = oracle_scale_code(fmt, amax);
+                scales[scale_index(block, pix, b0, a0, Ap, Bp)] = (uint8_t)sc;
+                double inv = ldexp(1.0, 127 - sc);
+                for (int64_t b = b0; b < b1; ++b)
+                    for (int64_t a = a0; a < a1; ++a) {
+                        if (b >= d0 || a >= d1) continue;     /* padding stays +0 */
+                        double x = src_at(src, d0, d1, strides, b, a, h, w);
+                        uint32_t r = oracle_sr_bits(seed, offset, d0, d1, pix, b, a);
+                        int code = oracle_encode_sr(fmt, x * inv, r);
                         put_code(codes, fmt, code_index(order, pix, b, a, Ap, Bp), code);
                     }
             }

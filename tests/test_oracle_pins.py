@@ -460,3 +460,17 @@ def test_table1_memory_movement(orc):
     # MXFP8 with B=32: 32 / 8.25 = 3.879 (the paper's "closer to x3.93" is the B=64 figure 32/8.125)
     mx8 = orc.codes_bytes(0, 0, N, C, H, W) + orc.scales_bytes(0, 0, 0, N, C, H, W)
     assert abs(fp32 / mx8 - 32 / 8.25) < 1e-12
+
+
+# ---------------------------------------------------------------- activation
+def test_activation_matches_torch(orc):
+    """The activations of the quantized forward output: torch's relu and silu
+    in float64, and the closed forms silu(0) = 0, silu(x) -> x and -> 0."""
+    y = synth.random_tensor((3, 5, 7, 11), seed=8, dist="student_t").astype(np.float64) * 4
+    t = torch.from_numpy(y)
+    assert np.array_equal(orc.activation(y, orc.ACT_NONE), y)
+    assert np.array_equal(orc.activation(y, orc.ACT_RELU), F.relu(t).numpy())
+    assert np.allclose(orc.activation(y, orc.ACT_SILU), F.silu(t).numpy(), rtol=1e-15, atol=1e-300)
+    big = np.array([0.0, 60.0, -60.0])
+    s = orc.activation(big, orc.ACT_SILU)
+    assert s[0] == 0.0 and abs(s[1] - 60.0) < 1e-20 and abs(s[2]) < 1e-20

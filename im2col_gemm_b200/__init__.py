@@ -32,7 +32,9 @@ EXPORTS = ("mqc_codes_bytes", "mqc_scales_bytes", "mqc_tensor_dims", "mqc_quanti
            "mqc_im2col_cbf_scales_bytes", "mqc_im2col_cbf_codes_bytes", "mqc_conv2d_fwd", "mqc_conv2d_bwd_data",
            "mqc_conv2d_bwd_weight", "mqc_conv2d_bwd_weight_workspace_bytes", "mqc_get_device_status",
            "mqc_debug_expire_wait", "mqc_status_string", "mqc_last_error_message", "mqc_version",
-           "mqc_conv2d_bwd_weight_noalloc", "mqc_conv2d_fwd_workspace_bytes", "mqc_conv2d_bwd_data_workspace_bytes")
+           "mqc_conv2d_bwd_weight_noalloc", "mqc_conv2d_fwd_workspace_bytes", "mqc_conv2d_bwd_data_workspace_bytes",
+           "mqc_quantize_mx_sr", "mqc_conv2d_fwd_quant")
+ACT_NONE, ACT_RELU, ACT_SILU = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -68,11 +70,14 @@ def _load() -> ctypes.CDLL:
         "mqc_scales_bytes": (i64, [P(MX), i32, i32, i32, i32]),
         "mqc_tensor_dims": (i32, [i32, P(Conv), P(i32)]),
         "mqc_quantize_mx": (i32, [vp, P(T4), P(MX), vp, vp, vp, vp]),
+        "mqc_quantize_mx_sr": (i32, [vp, P(T4), P(MX), vp, vp, vp, ctypes.c_uint64, ctypes.c_uint64, vp]),
         "mqc_im2col_cbf": (i32, [vp, vp, P(Conv), P(MX), vp, vp, vp]),
         "mqc_im2col_cbf_scales_bytes": (i64, [P(Conv), P(MX)]),
         "mqc_im2col_cbf_codes_bytes": (i64, [P(Conv), P(MX)]),
         "mqc_conv2d_fwd": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp, sz, vp]),
         "mqc_conv2d_fwd_workspace_bytes": (sz, [P(Conv), P(MX), P(MX)]),
+        "mqc_conv2d_fwd_quant": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), i32, P(MX), vp, vp, vp, vp, vp, sz,
+                                       vp]),
         "mqc_conv2d_bwd_data": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp, sz, vp]),
         "mqc_conv2d_bwd_data_workspace_bytes": (sz, [P(Conv), P(MX), P(MX)]),
         "mqc_conv2d_bwd_weight": (i32, [vp, vp, P(MX), vp, vp, P(MX), P(Conv), vp, vp, sz, vp]),
@@ -113,6 +118,11 @@ def mqc_quantize_mx(src_ptr, desc: T4, mx: MX, codes_ptr, scales_ptr, codes_alt_
                                codes_alt_ptr, stream)
 
 
+def mqc_quantize_mx_sr(src_ptr, desc: T4, mx: MX, codes_ptr, scales_ptr, codes_alt_ptr, seed, offset, stream) -> int:
+    return lib.mqc_quantize_mx_sr(src_ptr, ctypes.byref(desc), ctypes.byref(mx), codes_ptr, scales_ptr,
+                                  codes_alt_ptr, seed, offset, stream)
+
+
 def mqc_im2col_cbf(codes_ptr, scales_ptr, conv: Conv, mx: MX, codes_out_ptr, scales_out_ptr, stream) -> int:
     return lib.mqc_im2col_cbf(codes_ptr, scales_ptr, ctypes.byref(conv), ctypes.byref(mx), codes_out_ptr,
                               scales_out_ptr, stream)
@@ -121,6 +131,12 @@ def mqc_im2col_cbf(codes_ptr, scales_ptr, conv: Conv, mx: MX, codes_out_ptr, sca
 def mqc_conv2d_fwd(xq, xs, xf: MX, wq, ws, wf: MX, conv: Conv, y, workspace, workspace_bytes, stream) -> int:
     return lib.mqc_conv2d_fwd(xq, xs, ctypes.byref(xf), wq, ws, ctypes.byref(wf), ctypes.byref(conv), y, workspace,
                               workspace_bytes, stream)
+
+
+def mqc_conv2d_fwd_quant(xq, xs, xf: MX, wq, ws, wf: MX, conv: Conv, act: int, yf: MX, yq, ys, yq_alt, y, workspace,
+                         workspace_bytes, stream) -> int:
+    return lib.mqc_conv2d_fwd_quant(xq, xs, ctypes.byref(xf), wq, ws, ctypes.byref(wf), ctypes.byref(conv), act,
+                                    ctypes.byref(yf), yq, ys, yq_alt, y, workspace, workspace_bytes, stream)
 
 
 def mqc_conv2d_fwd_workspace_bytes(conv: Conv, xf: MX, wf: MX) -> int:
@@ -206,8 +222,11 @@ class Quantized:
                          self.codes)
 
 
-def quantize_mx(src, fmt: int, block: int, order: int, both_orders: bool = False) -> Quantized:
-    """MX-quantize a 4-D fp32 CUDA tensor [d0=B][d1=A][d2][d3] (any strides)."""
+def quantize_mx(src, fmt: int, block: int, order: int, both_orders: bool = False, sr_seed: int | None = None,
+                sr_offset: int = 0) -> Quantized:
+    """MX-quantize a 4-D fp32 CUDA tensor [d0=B][d1=A][d2][d3] (any strides);
+    with `sr_seed`, the elements are rounded stochastically
+    (mqc_quantize_mx_sr, order BA, NCHW-like source)."""
     torch = _torch()
     assert src.is_cuda and src.dtype == torch.float32 and src.dim() == 4
     d0, d1, d2, d3 = src.shape
@@ -223,7 +242,11 @@ def quantize_mx(src, fmt: int, block: int, order: int, both_orders: bool = False
         alt = torch.empty(mqc_codes_bytes(MX(fmt, block, 1 - order), d0, d1, d2, d3), dtype=torch.uint8,
                           device=src.device)
     desc = T4(d0, d1, d2, d3, *src.stride())
-    check(mqc_quantize_mx(_ptr(src), desc, mx, _ptr(codes), _ptr(scales), _ptr(alt), _stream()))
+    if sr_seed is None:
+        check(mqc_quantize_mx(_ptr(src), desc, mx, _ptr(codes), _ptr(scales), _ptr(alt), _stream()))
+    else:
+        check(mqc_quantize_mx_sr(_ptr(src), desc, mx, _ptr(codes), _ptr(scales), _ptr(alt), sr_seed, sr_offset,
+                                 _stream()))
     return Quantized(codes, scales, (d0, d1, d2, d3), mx, alt)
 
 
@@ -250,6 +273,30 @@ def conv2d_fwd(xq: Quantized, wq: Quantized, cv: Conv, out=None, workspace=None)
     check(mqc_conv2d_fwd(_ptr(xq.codes), _ptr(xq.scales), xq.mx, _ptr(wq.codes), _ptr(wq.scales), wq.mx, cv,
                          _ptr(y), _ptr(workspace), nws, _stream()))
     return y
+
+
+def conv2d_fwd_quant(xq: Quantized, wq: Quantized, cv: Conv, fmt: int, block: int, act: int = ACT_NONE,
+                     both_orders: bool = False, keep_fp32: bool = False, workspace=None):
+    """Forward convolution whose output is returned MX-quantized (order BA,
+    and AB with `both_orders`) as the next layer's input: (Quantized, y)
+    where y is the fp32 activated output when `keep_fp32`, else None."""
+    torch = _torch()
+    P, Q = conv_out_hw(cv)
+    dev = xq.codes.device
+    mx = MX(fmt, block, ORDER_BA)
+    dims = (cv.N, cv.K, P, Q)
+    codes = torch.empty(mqc_codes_bytes(mx, *dims), dtype=torch.uint8, device=dev)
+    scales = torch.empty(mqc_scales_bytes(mx, *dims), dtype=torch.uint8, device=dev)
+    alt = (torch.empty(mqc_codes_bytes(MX(fmt, block, ORDER_AB), *dims), dtype=torch.uint8, device=dev)
+           if both_orders else None)
+    y = torch.empty(dims, dtype=torch.float32, device=dev) if keep_fp32 else None
+    nws = mqc_conv2d_fwd_workspace_bytes(cv, xq.mx, wq.mx)
+    if workspace is None and nws > 0:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=dev)
+    check(mqc_conv2d_fwd_quant(_ptr(xq.codes), _ptr(xq.scales), xq.mx, _ptr(wq.codes), _ptr(wq.scales), wq.mx, cv,
+                               act, mx, _ptr(codes), _ptr(scales), _ptr(alt), _ptr(y), _ptr(workspace), nws,
+                               _stream()))
+    return Quantized(codes, scales, dims, mx, alt), y
 
 
 def conv2d_bwd_data(wq: Quantized, gq: Quantized, cv: Conv, out=None, workspace=None):

@@ -161,6 +161,16 @@ struct alignas(64) GemmParams {
     // the divisions of the unit and row decoding, by launch constants
     FastDiv fd_NT, fd_nph, fd_TQ, fd_TP, fd_sub, fd_bq, fd_bp, fd_bn, fd_MT, fd_ngroups, fd_splits, fd_cpad;
     int32_t x_st_h, x_st_w;      // stride of X pixels per output pixel
+    // CONV QOUT (forward with a quantized output, template flag): the
+    // epilogue applies the activation and writes the result as the next
+    // layer's MX-quantized input [N][K][P][Q] (B-axis N, A-axis K): codes in
+    // order BA [P][Q][N][q_Kp], optionally order AB [P][Q][K][q_Np], one
+    // E8M0 scale per block of 32 channels (A32) or per 32 x 32 square over
+    // (n, k) (SQ32); rows run n fastest within a pixel (rows_nfirst) with bn =
+    // q_lanes (16 or 32), so a square's rows are lanes of one warp
+    uint8_t *q_codes, *q_codes_alt, *q_scales;
+    float *q_y;                  // optional fp32 copy of the activated output (NCHW), else null
+    int32_t q_fmt, q_sq, q_act, q_emax, q_Kp, q_Np, q_nbA, q_nbB, q_lanes;
     // output
     float *out;
     int64_t out_base, os_q, os_p, os_n, os_c, os_m, split_pitch;
@@ -308,7 +318,173 @@ struct KitWalker {
 // UMT (CONV only): 128-row sub-tiles per unit (1, 2 or 4; p.um equals it).
 // A template parameter as well, so that the one-tile kernel carries no
 // sub-tile loops.
-template <int KIND, bool SFV4, int UMT>
+// Activations the quantized forward output can apply before quantizing:
+// 0 none, 1 ReLU, 2 SiLU (x * sigmoid(x), with CUDA's expf and an IEEE
+// division).
+__device__ __forceinline__ float activate(float x, int act) {
+    if (act == 1) return fmaxf(x, 0.0f);
+    if (act == 2) return x / (1.0f + expf(-x));
+    return x;
+}
+
+// E8M0 code of a block maximum and its inverse scale, for the quantized
+// forward output: e = floor(log2 amax) - emax, clamped below at -127 (zero
+// and subnormal maxima give 0x00); the same rule as the quantizer's.
+__device__ __forceinline__ uint32_t qout_scale_code(float amax, int emax) {
+    const uint32_t bits = __float_as_uint(amax);
+    if (bits >= 0x7F800000u) return 0xFFu;
+    const int ex = static_cast<int>(bits >> 23);
+    const int c = ex - emax;
+    return (ex == 0 || c < 0) ? 0u : static_cast<uint32_t>(c);
+}
+__device__ __forceinline__ float qout_inv_scale(uint32_t code) {
+    if (code == 0xFFu) return __uint_as_float(0x00400000u);
+    return __uint_as_float((254u - code) << 23);
+}
+
+// Four codes, one per byte (FP4: a nibble in each byte), round-to-nearest-
+// even with saturation.
+__device__ __forceinline__ uint32_t qout_cvt4(int fmt, float a, float b, float c, float d) {
+    uint16_t lo, hi;
+    if (fmt == 0) {
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+        return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+    if (fmt == 1) {
+        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+        return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+    uint32_t p0, p1;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}" : "=r"(p0) : "f"(b), "f"(a));
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}" : "=r"(p1) : "f"(d), "f"(c));
+    return (p0 & 0xFu) | ((p0 >> 4) << 8) | ((p1 & 0xFu) << 16) | ((p1 >> 4) << 24);
+}
+
+// Packs the bytes of w[0..7] (32 codes, one per byte) into 16 bytes of
+// nibbles, element 2i in the low nibble.
+__device__ __forceinline__ uint4 qout_pack_fp4(const uint32_t (&w)[8]) {
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t a = w[2 * q], b = w[2 * q + 1];
+        o[q] = (a & 0xFu) | ((a >> 4) & 0xF0u) | ((a >> 8) & 0xF00u) | ((a >> 12) & 0xF000u) |
+               ((b & 0xFu) << 16) | (((b >> 8) & 0xFu) << 20) | (((b >> 16) & 0xFu) << 24) | (((b >> 24) & 0xFu) << 28);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// QOUT: the output tile of one epilogue warp, 32 rows x 32 columns
+// (columns k0 .. k0 + 31 of its TMEM lane quadrant) -> activation, block
+// maxima, scales, codes in order BA, and through a per-warp 32 x 36-byte
+// shared-memory transpose the codes in order AB.
+//   v        the 32 accumulator columns of this thread's row
+//   row_ok   the row is an output (n < N, pixel inside the output)
+//   pix, n   next-layer pixel p*Q + q and batch index of the row
+//   k0       first output channel of the 32
+//   s_tr     this warp's transposition scratch (32 x 36 bytes)
+__device__ __forceinline__ void qout_chunk(const GemmParams &p, const uint32_t (&r)[32], bool row_ok, int pix,
+                                           int n, int k0, uint32_t *s_tr, int lane) {
+    const int K = p.Ncols;
+    float v[32];
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const float x = (row_ok && k0 + j < K) ? activate(__uint_as_float(r[j]), p.q_act) : 0.0f;
+        v[j] = x;
+        m = fmaxf(m, fabsf(x));
+    }
+    if (p.q_y != nullptr && row_ok) {
+        // optional fp32 copy, NCHW [N][K][P][Q]: p.os_* give the strides
+        float *op = p.q_y + static_cast<int64_t>(n) * p.os_n + static_cast<int64_t>(pix) + static_cast<int64_t>(k0) * p.os_c;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (k0 + j < K) op[j * p.os_c] = v[j];
+    }
+    if (p.q_sq) {
+        // square block: the rows of one pixel are q_lanes consecutive lanes
+#pragma unroll
+        for (int x = 1; x < 32; x <<= 1)
+            if (x < p.q_lanes) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, x));
+    }
+    const uint32_t code = qout_scale_code(m, p.q_emax);
+    const float inv = qout_inv_scale(code);
+    // pixel validity of the square's first lane (all rows of a pixel share it)
+    if (p.q_sq) {
+        const int lead = lane & ~(p.q_lanes - 1);
+        const bool pix_ok = __shfl_sync(0xFFFFFFFFu, row_ok ? 1 : 0, lead) != 0;
+        if (lane == lead && pix_ok)
+            p.q_scales[(static_cast<int64_t>(pix) * p.q_nbB + (n >> 5)) * p.q_nbA + (k0 >> 5)] = static_cast<uint8_t>(code);
+    } else if (row_ok) {
+        p.q_scales[(static_cast<int64_t>(pix) * p.Ne + n) * p.q_nbA + (k0 >> 5)] = static_cast<uint8_t>(code);
+    }
+    uint32_t w[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) w[q] = qout_cvt4(p.q_fmt, v[4 * q] * inv, v[4 * q + 1] * inv, v[4 * q + 2] * inv, v[4 * q + 3] * inv);
+    const bool fp4 = p.q_fmt == 2;
+    // order BA: row (pix, n), channels k0 .. k0 + 31 (clipped to the padded q_Kp)
+    if (row_ok) {
+        const int64_t off = (static_cast<int64_t>(pix) * p.Ne + n) * p.q_Kp + k0;   // in codes
+        if (fp4) {
+            *reinterpret_cast<uint4 *>(p.q_codes + off / 2) = qout_pack_fp4(w);
+        } else {
+            uint4 *d = reinterpret_cast<uint4 *>(p.q_codes + off);
+            d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            if (p.q_Kp - k0 >= 32) d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+    }
+    if (p.q_codes_alt == nullptr) return;
+    // order AB: lane L takes channel k0 + L and the codes of the 32 rows
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) s_tr[lane * 9 + q] = w[q];
+    __syncwarp();
+    const uint8_t *tb = reinterpret_cast<const uint8_t *>(s_tr);
+    uint32_t t[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        t[q] = 0u;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) t[q] |= static_cast<uint32_t>(tb[(4 * q + b) * 36 + lane]) << (8 * b);
+    }
+    // pixels and row validity of the lanes' groups
+    const int pix0 = __shfl_sync(0xFFFFFFFFu, pix, 0), pix1 = __shfl_sync(0xFFFFFFFFu, pix, 16);
+    const int n0 = __shfl_sync(0xFFFFFFFFu, n, 0), n1 = __shfl_sync(0xFFFFFFFFu, n, 16);
+    const bool ok0 = __shfl_sync(0xFFFFFFFFu, row_ok ? 1 : 0, 0) != 0;
+    const bool ok1 = __shfl_sync(0xFFFFFFFFu, row_ok ? 1 : 0, 16) != 0;
+    const int k = k0 + lane;
+    if (k >= K) return;
+    if (p.q_lanes == 32) {
+        // one pixel, batch n0 .. n0 + 31 (clipped to the padded q_Np)
+        if (!ok0) return;
+        const int64_t off = (static_cast<int64_t>(pix0) * K + k) * p.q_Np + n0;
+        if (fp4) {
+            *reinterpret_cast<uint4 *>(p.q_codes_alt + off / 2) = qout_pack_fp4(t);
+        } else {
+            uint4 *d = reinterpret_cast<uint4 *>(p.q_codes_alt + off);
+            d[0] = make_uint4(t[0], t[1], t[2], t[3]);
+            if (p.q_Np - n0 >= 32) d[1] = make_uint4(t[4], t[5], t[6], t[7]);
+        }
+    } else {
+        // two pixels of 16 rows each (a batch of at most 16: q_Np = 16 FP8 or
+        // 32 FP4 codes, the rows past N are zero codes)
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            if (!(g == 0 ? ok0 : ok1)) continue;
+            const int64_t off = (static_cast<int64_t>(g == 0 ? pix0 : pix1) * K + k) * p.q_Np;
+            if (fp4) {
+                uint32_t h[8] = {t[4 * g], t[4 * g + 1], t[4 * g + 2], t[4 * g + 3], 0u, 0u, 0u, 0u};
+                *reinterpret_cast<uint4 *>(p.q_codes_alt + off / 2) = qout_pack_fp4(h);
+            } else {
+                *reinterpret_cast<uint4 *>(p.q_codes_alt + off) = make_uint4(t[4 * g], t[4 * g + 1], t[4 * g + 2], t[4 * g + 3]);
+            }
+        }
+        (void)n1;
+    }
+}
+
+template <int KIND, bool SFV4, int UMT, bool QOUT = false>
 __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
@@ -344,6 +520,8 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
     // k16: the upper 16 bytes of every operand row (batch 16..31 of a K-block)
     // are read by the MMA from this zero block (256 rows x 16 bytes)
     uint8_t *sZ = reinterpret_cast<uint8_t *>(full) + 1024;
+    // QOUT: eight 32 x 36-byte transposition buffers (one per epilogue warp)
+    uint32_t *sTr = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(full) + 1024);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -915,7 +1093,7 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
             };
             const bool tap_cols = KIND == kWgrad && p.ntg > 1;   // columns are (tap, channel)
             if (I.nk == 0) {
-                if (team != 0) continue;
+                if (team != 0 || QOUT) continue;   // (a forward tile always has K-blocks)
                 for (int i = 0; i < UM; ++i) {
                     set_row(i);
                     if (row_ok)
@@ -950,6 +1128,27 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
             for (int i = 0; i < UM; ++i) {
                 set_row(i);
                 const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16) + (acc * UM + i) * p.BN;
+                if constexpr (KIND == kConv && QOUT) {
+                    // next-layer pixel and batch index of this row
+                    int q0 = I.q0, p0 = I.p0, n0 = I.n0;
+                    if (i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
+                    int aw, iq, ip, in;
+                    conv_row(p, m, aw, iq, ip, in);
+                    const int qpix = (p0 + ip) * p.ph_Qe[0] + (q0 + iq);
+                    for (int c0 = 0; c0 < p.BN; c0 += 32) {
+                        uint32_t r[32];
+                        tc_ld_32x32b_x32(t_row + c0, r);
+                        tc_wait_ld();
+                        if (i + 1 == UM && c0 + 32 >= p.BN) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                        }
+                        if (I.col0 + c0 < p.Ncols)
+                            qout_chunk(p, r, row_ok, qpix, n0 + in, I.col0 + c0, sTr + (team * 4 + qd) * (32 * 9), lane);
+                    }
+                    continue;
+                }
                 float *orow = p.out + row_off;
                 if (KIND == kConv && p.d2s == 2) {
                     // 16 channels of a phase pair (aw = 0, 1) per pass: column

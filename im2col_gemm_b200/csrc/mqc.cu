@@ -88,8 +88,9 @@ int conv_Q(const mqc_conv *c) { return (c->W + 2 * c->pad_w - c->S) / c->stride_
 struct DevInfo {
     int sms = 0;
     int max_smem = 0;
-    bool gemm_attr[8] = {};   // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind, [7] SFV4 weight gradient
-    bool quant_attr[36] = {};                             // staged quantizer, [(fmt*3 + blk)*4 + tile]
+    bool gemm_attr[16] = {};  // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind, [7] SFV4 weight
+                              // gradient, [8 + 1 + 3 * SFV4 + log2(um)] forward with a quantized output
+    bool quant_attr[72] = {};    // staged quantizer, [36*sr + (fmt*3 + blk)*4 + tile]
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
@@ -235,8 +236,11 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     P.sfb_cached = KIND == kConv && cache <= 16384 && !P.sfb_vec4;
     // the 32-bit scale path reads B four bytes at a time unless B is cached
     if (!P.sfb_cached && !P.sfb_vec4) P.sf_vec4 = 0;
-    // k16: the zero block (4 KB) 1 KB past the barriers
-    const int fixed = 1024 + (P.k16 ? 1024 + 4096 : 64 * 8 + 64) + (P.sfb_cached ? cache : 0);
+    // k16: the zero block (4 KB) 1 KB past the barriers; quantized output:
+    // eight 32 x 36-byte transposition buffers there
+    const bool qout = KIND == kConv && P.q_codes != nullptr;
+    const int fixed = 1024 + (P.k16 ? 1024 + 4096 : (qout ? 1024 + 8 * 32 * 36 : 64 * 8 + 64)) +
+                      (P.sfb_cached ? cache : 0);
     // CONV with few K-blocks per tile and narrow column tiles: units of
     // um = 2 or 4 row tiles, so that the per-unit work of every role (decode,
     // barrier round trips, B loads, scale atoms of B) is shared by um MMAs;
@@ -302,12 +306,17 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     const int smem = fixed + S * per_stage;
     const bool v4 = KIND == kConv && P.sf_vec4;
     auto kernel = P.sq_gather ? conv_gemm_kernel<kWgrad, true, 1> : conv_gemm_kernel<kWgrad, false, 1>;
-    if (KIND == kConv) {
+    if (KIND == kConv && !qout) {
         if (P.um == 4) kernel = v4 ? conv_gemm_kernel<kConv, true, 4> : conv_gemm_kernel<kConv, false, 4>;
         else if (P.um == 2) kernel = v4 ? conv_gemm_kernel<kConv, true, 2> : conv_gemm_kernel<kConv, false, 2>;
         else kernel = v4 ? conv_gemm_kernel<kConv, true, 1> : conv_gemm_kernel<kConv, false, 1>;
+    } else if (KIND == kConv) {
+        if (P.um == 4) kernel = v4 ? conv_gemm_kernel<kConv, true, 4, true> : conv_gemm_kernel<kConv, false, 4, true>;
+        else if (P.um == 2) kernel = v4 ? conv_gemm_kernel<kConv, true, 2, true> : conv_gemm_kernel<kConv, false, 2, true>;
+        else kernel = v4 ? conv_gemm_kernel<kConv, true, 1, true> : conv_gemm_kernel<kConv, false, 1, true>;
     }
-    const int ai = KIND == kConv ? 1 + (v4 ? 3 : 0) + (P.um == 4 ? 2 : P.um - 1) : (P.sq_gather ? 7 : 0);
+    const int ai = KIND == kConv ? (qout ? 8 : 0) + 1 + (v4 ? 3 : 0) + (P.um == 4 ? 2 : P.um - 1)
+                                 : (P.sq_gather ? 7 : 0);
     if (!d.gemm_attr[ai]) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.max_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -431,9 +440,34 @@ mqc_status mqc_tensor_dims(mqc_role role, const mqc_conv *c, int32_t dims[4]) {
     return fail(MQC_ERR_INVALID, "bad role %d", (int)role);
 }
 
+}  // extern "C"
+
 // ------------------------------------------------------------------ quantize
+// Stochastic rounding request: Philox key and stream offset.
+struct SrArgs {
+    uint64_t seed, offset;
+};
+
+static mqc_status quantize_impl(const float *src, const mqc_t4 *d, const mqc_mx *mx, void *codes, uint8_t *scales,
+                                void *codes_alt, void *stream, const SrArgs *sr);
+
+extern "C" {
+
 mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, void *codes, uint8_t *scales,
                            void *codes_alt, void *stream) {
+    return quantize_impl(src, d, mx, codes, scales, codes_alt, stream, nullptr);
+}
+
+mqc_status mqc_quantize_mx_sr(const float *src, const mqc_t4 *d, const mqc_mx *mx, void *codes, uint8_t *scales,
+                              void *codes_alt, uint64_t seed, uint64_t offset, void *stream) {
+    const SrArgs sr{seed, offset};
+    return quantize_impl(src, d, mx, codes, scales, codes_alt, stream, &sr);
+}
+
+}  // extern "C"
+
+static mqc_status quantize_impl(const float *src, const mqc_t4 *d, const mqc_mx *mx, void *codes, uint8_t *scales,
+                                void *codes_alt, void *stream, const SrArgs *sr) {
     if (src == nullptr || d == nullptr || codes == nullptr || scales == nullptr || !mx_ok(mx))
         return fail(MQC_ERR_INVALID, "quantize: null pointer or bad mx descriptor");
     if (d->d0 <= 0 || d->d1 <= 0 || d->d2 <= 0 || d->d3 <= 0)
@@ -443,6 +477,13 @@ mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, 
         return fail(MQC_ERR_ALIGNMENT, "quantize: codes not 16-byte aligned");
     if (static_cast<int64_t>(d->d2) * d->d3 > (int64_t(1) << 31) - 64)
         return fail(MQC_ERR_INVALID, "quantize: too many spatial positions");
+    // staged kernel: positions contiguous (element stride 1 along W, W along
+    // H), every plane 16-byte aligned
+    const bool staged = d->s3 == 1 && d->s2 == d->d3 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 &&
+                        d->s0 % 4 == 0 && d->s1 % 4 == 0;
+    if (sr != nullptr && (mx->order != MQC_ORDER_BA || !staged))
+        return fail(MQC_ERR_UNSUPPORTED,
+                    "quantize_mx_sr: needs order BA and an NCHW-like source (contiguous, 16-byte aligned planes)");
     DevInfo *dv;
     mqc_status st = dev_info(dv);
     if (st != MQC_OK) return st;
@@ -488,10 +529,7 @@ mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, 
     const int blk = mx->block == MQC_BLOCK_SQ32 ? kSquare : (along_i ? kAlongI : kAlongO);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool dual = codes_alt != nullptr;
-    // staged kernel: FP8, positions contiguous (element stride 1 along W,
-    // W along H), every plane 16-byte aligned
-    if (d->s3 == 1 && d->s2 == d->d3 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && d->s0 % 4 == 0 &&
-        d->s1 % 4 == 0) {
+    if (staged) {
         StagedParams sp{};
         sp.q = p;
         sp.IT = (!fp4 && p.I1 <= 16) ? 16 : 32;     // FP4 rows are 32 codes
@@ -502,15 +540,29 @@ mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, 
         sp.nIT = static_cast<int32_t>(ceil_div(p.I1, sp.IT));
         sp.blk = blk;
         sp.map_a = map_a ? 1 : 0;
+        if (sr != nullptr) {
+            sp.seed = sr->seed;
+            sp.offset = sr->offset;
+            sp.a16_blocks = static_cast<int32_t>(ceil_div(p.A, 16));
+        }
         const int64_t ntiles = int64_t(sp.nPT) * sp.nOT * sp.nIT;
         if (ntiles > (int64_t(1) << 31) - 1) return fail(MQC_ERR_INVALID, "quantize: tensor too large");
-        const int smem = kStagedTileBytes + 32 * 64 * 4 + 64 * 4;
-        // the shared-memory limit is raised once per (format, block, tile) kernel
-        const int ai = (p.fmt * 3 + blk) * 4 + (sp.OT == 32 ? 2 : 0) + (sp.IT == 32 ? 1 : 0);
+        // tile, block reciprocals, square maxima (+ the codes of the tile with SR)
+        const int smem = kStagedTileBytes + 32 * 64 * 4 + 64 * 4 + (sr ? kStagedTileBytes / 4 : 0);
+        // the shared-memory limit is raised once per (SR, format, block, tile) kernel
+        const int ai = (sr ? 36 : 0) + (p.fmt * 3 + blk) * 4 + (sp.OT == 32 ? 2 : 0) + (sp.IT == 32 ? 1 : 0);
         cudaError_t ae = cudaSuccess;
-        if (p.fmt == MQC_E4M3) launch_staged<0>(sp, static_cast<unsigned>(ntiles), smem, s, ae, !dv->quant_attr[ai]);
-        else if (p.fmt == MQC_E5M2) launch_staged<1>(sp, static_cast<unsigned>(ntiles), smem, s, ae, !dv->quant_attr[ai]);
-        else launch_staged<2>(sp, static_cast<unsigned>(ntiles), smem, s, ae, !dv->quant_attr[ai]);
+        const unsigned g = static_cast<unsigned>(ntiles);
+        const bool set = !dv->quant_attr[ai];
+        if (sr == nullptr) {
+            if (p.fmt == MQC_E4M3) launch_staged<0, false>(sp, g, smem, s, ae, set);
+            else if (p.fmt == MQC_E5M2) launch_staged<1, false>(sp, g, smem, s, ae, set);
+            else launch_staged<2, false>(sp, g, smem, s, ae, set);
+        } else {
+            if (p.fmt == MQC_E4M3) launch_staged<0, true>(sp, g, smem, s, ae, set);
+            else if (p.fmt == MQC_E5M2) launch_staged<1, true>(sp, g, smem, s, ae, set);
+            else launch_staged<2, true>(sp, g, smem, s, ae, set);
+        }
         if (ae != cudaSuccess) return cuda_fail(ae, "cudaFuncSetAttribute");
         dv->quant_attr[ai] = true;
         cudaError_t e = cudaGetLastError();
@@ -523,6 +575,8 @@ mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *d, const mqc_mx *mx, 
     if (e != cudaSuccess) return cuda_fail(e, "mx_quantize_kernel launch");
     return MQC_OK;
 }
+
+extern "C" {
 
 // ------------------------------------------------------------------ im2col
 static void im2col_geometry(const mqc_conv *c, const mqc_mx *mx, int64_t &Ap, int64_t &Bp, int64_t &chunk_codes,
@@ -609,15 +663,60 @@ size_t mqc_conv2d_fwd_workspace_bytes(const mqc_conv *c, const mqc_mx *xf, const
     return widened_bytes(xf, c->N, c->C, c->H, c->W) + widened_bytes(wf, c->K, c->C, c->R, c->S);
 }
 
+}  // extern "C"
+
+// Quantized output of the forward (the next layer's input, quantized in the
+// GEMM epilogue): format, block mode, activation and destination buffers.
+struct QoutArgs {
+    const mqc_mx *yf;
+    int act;
+    void *yq, *yq_alt;
+    uint8_t *ys;
+    float *y;      // optional fp32 copy of the activated output
+};
+
+static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx *xf, const void *wq,
+                                const uint8_t *ws, const mqc_mx *wf, const mqc_conv *c, float *y, void *workspace,
+                                size_t workspace_bytes, void *stream, const QoutArgs *qo);
+
+extern "C" {
+
 mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, const void *wq, const uint8_t *ws,
                           const mqc_mx *wf, const mqc_conv *c, float *y, void *workspace, size_t workspace_bytes,
                           void *stream) {
     if (!conv_ok(c) || y == nullptr) return fail(MQC_ERR_INVALID, "conv2d_fwd: bad conv descriptor or null output");
+    return conv_fwd_impl(xq, xs, xf, wq, ws, wf, c, y, workspace, workspace_bytes, stream, nullptr);
+}
+
+mqc_status mqc_conv2d_fwd_quant(const void *xq, const uint8_t *xs, const mqc_mx *xf, const void *wq,
+                                const uint8_t *ws, const mqc_mx *wf, const mqc_conv *c, int32_t act,
+                                const mqc_mx *yf, void *yq, uint8_t *ys, void *yq_alt, float *y, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    if (!conv_ok(c) || yq == nullptr || ys == nullptr || !mx_ok(yf))
+        return fail(MQC_ERR_INVALID, "conv2d_fwd_quant: bad conv descriptor, output or output format");
+    if (act < MQC_ACT_NONE || act > MQC_ACT_SILU) return fail(MQC_ERR_INVALID, "conv2d_fwd_quant: bad activation");
+    if (yf->order != MQC_ORDER_BA || yf->block == MQC_BLOCK_B32)
+        return fail(MQC_ERR_UNSUPPORTED, "conv2d_fwd_quant: the output is written in order BA, blocks A32 or SQ32");
+    if (!aligned16(yq) || (yq_alt != nullptr && !aligned16(yq_alt)))
+        return fail(MQC_ERR_ALIGNMENT, "conv2d_fwd_quant: output codes not 16-byte aligned");
+    if (y != nullptr && (reinterpret_cast<uintptr_t>(y) & 3u) != 0)
+        return fail(MQC_ERR_ALIGNMENT, "conv2d_fwd_quant: fp32 output not 4-byte aligned");
+    const QoutArgs qo{yf, act, yq, yq_alt, ys, y};
+    return conv_fwd_impl(xq, xs, xf, wq, ws, wf, c, y, workspace, workspace_bytes, stream, &qo);
+}
+
+}  // extern "C"
+
+static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx *xf, const void *wq,
+                                const uint8_t *ws, const mqc_mx *wf, const mqc_conv *c, float *y, void *workspace,
+                                size_t workspace_bytes, void *stream, const QoutArgs *qo) {
     mqc_status st = check_gemm_operand("X", xq, xs, xf, MQC_ORDER_BA, true);
     if (st != MQC_OK) return st;
     st = check_gemm_operand("W", wq, ws, wf, MQC_ORDER_BA, true);
     if (st != MQC_OK) return st;
     if (c->R * c->S > kMaxTaps) return fail(MQC_ERR_UNSUPPORTED, "conv2d_fwd: at most %d kernel taps", kMaxTaps);
+    // one activation tensor map per stride phase, four at most
+    if (c->stride_h * c->stride_w > 4) return fail(MQC_ERR_UNSUPPORTED, "conv2d_fwd: stride product above 4");
     DevInfo *dv;
     if ((st = dev_info(dv)) != MQC_OK) return st;
 
@@ -635,7 +734,25 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     memset(&G, 0, sizeof G);
     G.CB = static_cast<int32_t>(nb32(Cp));
     G.wkb = largest_wkb(G.CB);
-    choose_rows(Q, P, N, G.bq, G.bp, G.bn);
+    if (qo == nullptr) {
+        choose_rows(Q, P, N, G.bq, G.bp, G.bn);
+    } else {
+        // quantized output: rows n fastest, bn = 16 (a batch of at most 16)
+        // or 32, so that the rows of one pixel are lanes of one warp; the
+        // pixels of a tile: the fewest computed rows, then the longest run
+        // along q
+        G.bn = N <= 16 ? 16 : 32;
+        const int pix = 128 / G.bn;
+        G.bq = pix;
+        G.bp = 1;
+        for (int bq = pix / 2; bq >= 1; bq /= 2) {
+            const int bp = pix / bq;
+            if (ceil_div(Q, bq) * bq * ceil_div(P, bp) * bp < ceil_div(Q, G.bq) * G.bq * ceil_div(P, G.bp) * G.bp) {
+                G.bq = bq;
+                G.bp = bp;
+            }
+        }
+    }
     G.BN = choose_bn(K);
     G.nb_atoms = static_cast<int32_t>(ceil_div(G.BN, 128));
     G.Ne = N;
@@ -647,10 +764,9 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     G.a_st_h = sh;
     G.a_st_w = sw;
     G.idesc = make_idesc_mx(mma_fmt(ox.mma_fmt), mma_fmt(ow.mma_fmt), 128, G.BN);
-    if (sh * sw > 4) return fail(MQC_ERR_UNSUPPORTED, "conv2d_fwd: stride product above 4");
     // A: one map per stride phase; dims (C, W', H', N) so that rows run along q
     bool phase_ok[16] = {};
-    for (int attempt = 0; attempt < 2; ++attempt) {
+    for (int attempt = qo ? 1 : 0; attempt < 2; ++attempt) {
         G.rows_nfirst = attempt;
         st = MQC_OK;
         for (int a = 0; a < sh && st == MQC_OK; ++a)
@@ -738,9 +854,30 @@ mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf, c
     G.os_p = Q;
     G.os_n = int64_t(K) * P * Q;
     G.os_c = int64_t(P) * Q;
+    if (qo != nullptr) {
+        int64_t Kp, Np_ba, Kp_ab, Np;
+        padded(qo->yf->fmt, MQC_ORDER_BA, K, N, Kp, Np_ba);
+        padded(qo->yf->fmt, MQC_ORDER_AB, K, N, Kp_ab, Np);
+        G.q_codes = static_cast<uint8_t *>(qo->yq);
+        G.q_codes_alt = static_cast<uint8_t *>(qo->yq_alt);
+        G.q_scales = qo->ys;
+        G.q_y = qo->y;
+        G.q_fmt = qo->yf->fmt;
+        G.q_sq = qo->yf->block == MQC_BLOCK_SQ32 ? 1 : 0;
+        G.q_act = qo->act;
+        G.q_emax = emax_elem(qo->yf->fmt);
+        G.q_Kp = static_cast<int32_t>(Kp);
+        G.q_Np = static_cast<int32_t>(Np);
+        G.q_nbA = static_cast<int32_t>(nb32(Kp));
+        G.q_nbB = static_cast<int32_t>(nb32(N));
+        G.q_lanes = G.bn;
+        G.out = nullptr;
+    }
     G.num_units = G.TQ * G.TP * G.TN * G.NT;
     return launch_gemm<kConv>(G, *dv, static_cast<cudaStream_t>(stream));
 }
+
+extern "C" {
 
 // ------------------------------------------------------------------ input gradient
 // Input gradient of a strided convolution as one sub-pixel GEMM (see
@@ -1134,13 +1271,14 @@ mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx
     st = check_gemm_operand("X", xq, xs, xf, MQC_ORDER_AB, false);
     if (st != MQC_OK) return st;
     if (c->R * c->S > kMaxTaps) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_weight: at most %d kernel taps", kMaxTaps);
+    // one activation tensor map per stride phase, four at most
+    if (c->stride_h * c->stride_w > 4) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_weight: stride product above 4");
     DevInfo *dv;
     if ((st = dev_info(dv)) != MQC_OK) return st;
     const int N = c->N, C = c->C, H = c->H, W = c->W, K = c->K, R = c->R, S = c->S;
     const int sh = c->stride_h, sw = c->stride_w, P = conv_P(c), Q = conv_Q(c);
     GemmParams G;
     memset(&G, 0, sizeof G);
-    if (sh * sw > 4) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_weight: stride product above 4");
     const WgradPlan plan = wgrad_plan(c, *dv);
     const int64_t kiters = plan.kiters;
     G.BN = plan.BN;

@@ -343,7 +343,76 @@ struct StagedParams {
     int32_t nPT, nOT, nIT;       // tile counts
     int32_t blk;                 // kAlongI, kAlongO or kSquare
     int32_t map_a;               // the inner axis i is A (order BA)
+    // stochastic rounding (order BA only): Philox4x64-10 key (seed, 0),
+    // counter (element index / 16, offset, 0, 0); element index
+    // ((pix*B + b)*A16 + a) with A16 = A rounded up to 16
+    uint64_t seed, offset;
+    int32_t a16_blocks;          // A16 / 16
 };
+
+// Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
+// easy as 1, 2, 3", SC 2011) for the counter (c0, c1, 0, 0) and key (k0, 0):
+// ten rounds of two 64x64->128-bit products with the published multipliers,
+// the key bumped by the published Weyl increments between rounds.
+__device__ __forceinline__ void philox4x64_10(uint64_t c0, uint64_t c1, uint64_t k0, uint64_t (&out)[4]) {
+    uint64_t c2 = 0, c3 = 0, k1 = 0;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += 0x9E3779B97F4A7C15ull;
+            k1 += 0xBB67AE8584CAA73Bull;
+        }
+        const uint64_t h0 = __umul64hi(0xD2E7470EE14C6C93ull, c0), l0 = 0xD2E7470EE14C6C93ull * c0;
+        const uint64_t h1 = __umul64hi(0xCA5A826395121157ull, c2), l1 = 0xCA5A826395121157ull * c2;
+        const uint64_t n0 = h1 ^ c1 ^ k0, n2 = h0 ^ c3 ^ k1;
+        c0 = n0;
+        c1 = l1;
+        c2 = n2;
+        c3 = l0;
+    }
+    out[0] = c0;
+    out[1] = c1;
+    out[2] = c2;
+    out[3] = c3;
+}
+
+// Stochastic rounding of v (already divided by the block scale) to the
+// element format with 16 uniform random bits r (paper, section III-A, Eq. 6:
+// gradients are rounded stochastically).  |v| lies between neighbouring
+// magnitudes lo <= |v| < hi; with f = (|v| - lo) / (hi - lo) the magnitude
+// becomes hi when r < f * 2^16, else lo.  Above the largest finite magnitude
+// it saturates; the sign is kept.  In the format's normal range lo is |v|
+// with the fp32 mantissa cut to the format's MB bits, and f * 2^16 is the
+// cut-off remainder over 2^(7 - MB); below it |v| is a multiple of the
+// subnormal step 2^(EMIN - MB) plus f steps.  Returns the code (8 or 4 bits).
+template <int FMT>
+__device__ __forceinline__ uint32_t sr_code(float v, uint32_t r) {
+    constexpr int MB = FMT == 0 ? 3 : (FMT == 1 ? 2 : 1);
+    constexpr int BIAS = FMT == 0 ? 7 : (FMT == 1 ? 15 : 1);
+    constexpr int EMIN = 1 - BIAS;                                   // exponent of the smallest normal
+    constexpr float VMAX = FMT == 0 ? 448.0f : (FMT == 1 ? 57344.0f : 6.0f);
+    constexpr uint32_t CMAX = FMT == 0 ? 0x7Eu : (FMT == 1 ? 0x7Bu : 0x7u);
+    constexpr float SUB = FMT == 0 ? 512.0f : (FMT == 1 ? 65536.0f : 2.0f);   // 2^(MB - EMIN)
+    constexpr int SIGN = FMT == 2 ? 3 : 7;
+    const uint32_t bits = __float_as_uint(v);
+    const uint32_t ab = bits & 0x7FFFFFFFu;
+    const float a = __uint_as_float(ab);
+    uint32_t code;
+    if (!(a < VMAX)) {
+        code = CMAX;
+    } else if (static_cast<int>(ab >> 23) - 127 >= EMIN) {
+        const uint32_t rem = ab & ((1u << (23 - MB)) - 1u);
+        const uint32_t lo = (static_cast<uint32_t>(static_cast<int>(ab >> 23) - 127 + BIAS) << MB) |
+                            ((ab >> (23 - MB)) & ((1u << MB) - 1u));
+        code = lo + ((r << (7 - MB)) < rem ? 1u : 0u);
+    } else {
+        const float t = a * SUB;                                     // exact: a power-of-two scaling
+        const uint32_t lo = static_cast<uint32_t>(t);
+        const float f = t - static_cast<float>(lo);
+        code = lo + (static_cast<float>(r) < f * 65536.0f ? 1u : 0u);
+    }
+    return ((bits >> 31) << SIGN) | code;
+}
 
 __device__ __forceinline__ void cp_async_16(void *smem, const void *gmem, int src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(src_bytes)
@@ -378,8 +447,13 @@ __device__ __forceinline__ void store_row(uint8_t *dst, const uint32_t (&h)[NQ],
 // OT, IT: tile extents (16 or 32); PT = positions per tile; NS = threads per
 // position.  A thread owns o-rows {sub, sub + NS, ...} in the primary pass and
 // i-columns {sub, sub + NS, ...} in the second-order pass (64 values each).
-template <int FMT, int BLK, int OT, int IT>
-__global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid_constant__ StagedParams sp) {
+//
+// SR: stochastic rounding (order BA): pass 1 draws the random bits of its
+// rows (one Philox block per 16 codes of a row) and keeps the codes in
+// shared memory; pass 2 reorders those codes instead of converting again,
+// so both orders hold the same rounding decisions.
+template <int FMT, int BLK, int OT, int IT, bool SR>
+__global__ void __launch_bounds__(256, SR ? 2 : 3) mx_quantize_staged_kernel(const __grid_constant__ StagedParams sp) {
     constexpr int PT = kStagedTileBytes / (4 * OT * IT);
     constexpr int NS = 256 / PT;
     constexpr int RO = OT / NS, RI = IT / NS;       // owned rows / columns per thread
@@ -387,6 +461,7 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
     float *tile = reinterpret_cast<float *>(smem_q);                        // [o][i][pos]
     float *s_inv = reinterpret_cast<float *>(smem_q + kStagedTileBytes);    // [block][pos]
     int *s_amax = reinterpret_cast<int *>(s_inv + 32 * 64);                 // [pos] (square blocks)
+    uint8_t *s_codes = reinterpret_cast<uint8_t *>(s_amax + 64);            // SR: [o][i][pos], one code per byte
     const QuantParams &p = sp.q;
     const int tid = threadIdx.x;
     const int pos = tid % PT, sub = tid / PT;
@@ -479,10 +554,11 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
         }
     }
     __syncthreads();
-    if (!pix_ok) return;
+    // (SR: every thread stays for the barrier before pass 2)
+    if (!SR && !pix_ok) return;
 
     // ---- pass 1: primary rows [pix][o][i0 .. i0 + IT) (clipped to the padded I1)
-    {
+    if (pix_ok) {
         const bool full_row = IT == 16 || p.I1 - i0 >= 32;
         float inv_i[BLK == kAlongO ? IT : 1];
         if (BLK == kAlongO) {
@@ -496,6 +572,32 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
             if (o0 + o >= p.O) break;
             const float inv_row = BLK == kAlongI ? s_inv[o * PT + pos] : inv_sq;
             uint32_t h[IT / 4];
+            if constexpr (SR) {
+                // random words of this row: Philox blocks (pix*B + b)*A16/16 + i0/16 + k
+                uint64_t rw[IT / 4];
+                const uint64_t blk0 = (static_cast<uint64_t>(pix) * p.B + (o0 + o)) * sp.a16_blocks + i0 / 16;
+#pragma unroll
+                for (int k = 0; k < IT / 16; ++k) {
+                    uint64_t w4[4];
+                    philox4x64_10(blk0 + k, sp.offset, sp.seed, w4);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) rw[4 * k + j] = w4[j];
+                }
+#pragma unroll
+                for (int q = 0; q < IT / 4; ++q) {
+                    uint32_t c[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int i = 4 * q + k;
+                        const float v = tp[(o * IT + i) * PT] * (BLK == kAlongO ? inv_i[i % (BLK == kAlongO ? IT : 1)] : inv_row);
+                        const uint32_t r = static_cast<uint32_t>(rw[i >> 2] >> (16 * (i & 3))) & 0xFFFFu;
+                        c[k] = sr_code<FMT>(v, r);
+                        s_codes[(o * IT + i) * PT + pos] = static_cast<uint8_t>(c[k]);
+                    }
+                    h[q] = FMT == 2 ? (c[0] | (c[1] << 4) | (c[2] << 8) | (c[3] << 12))
+                                    : (c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24));
+                }
+            } else {
 #pragma unroll
             for (int q = 0; q < IT / 4; ++q) {
                 float v[4];
@@ -504,11 +606,17 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
                     v[k] = tp[(o * IT + 4 * q + k) * PT] * (BLK == kAlongO ? inv_i[(4 * q + k) % (BLK == kAlongO ? IT : 1)] : inv_row);
                 h[q] = pack4<FMT>(v);
             }
+            }
             const int64_t off = (static_cast<int64_t>(pix) * p.O + o0 + o) * p.I1 + i0;   // in codes
             store_row<FMT, IT / 4>(p.codes + (FMT == 2 ? off / 2 : off), h, full_row ? IT : 16);
         }
     }
     if (p.codes_alt == nullptr) return;
+    if constexpr (SR) {
+        // every row of the tile (all positions) has been converted in pass 1
+        __syncthreads();
+    }
+    if (!pix_ok) return;
 
     // ---- pass 2: second order rows [pix][i][o0 .. o0 + OT) (clipped to the padded O2)
     {
@@ -527,11 +635,21 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
             uint32_t h[OT / 4];
 #pragma unroll
             for (int q = 0; q < OT / 4; ++q) {
+                if constexpr (SR) {
+                    // rows past O were never converted: their codes are +0
+                    uint32_t c[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        c[k] = o0 + 4 * q + k < p.O ? s_codes[((4 * q + k) * IT + i) * PT + pos] : 0u;
+                    h[q] = FMT == 2 ? (c[0] | (c[1] << 4) | (c[2] << 8) | (c[3] << 12))
+                                    : (c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24));
+                } else {
                 float v[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     v[k] = tp[((4 * q + k) * IT + i) * PT] * (BLK == kAlongI ? inv_o[(4 * q + k) % (BLK == kAlongI ? OT : 1)] : inv_col);
                 h[q] = pack4<FMT>(v);
+                }
             }
             const int64_t off = (static_cast<int64_t>(pix) * p.I + i0 + i) * p.O2 + o0;   // in codes
             store_row<FMT, OT / 4>(p.codes_alt + (FMT == 2 ? off / 2 : off), h, full_row ? OT : 16);
@@ -539,7 +657,7 @@ __global__ void __launch_bounds__(256, 3) mx_quantize_staged_kernel(const __grid
     }
 }
 
-template <int FMT, int BLK>
+template <int FMT, int BLK, bool SR>
 inline void launch_staged_tiles(const StagedParams &sp, unsigned grid, int smem, cudaStream_t s, cudaError_t &attr_err,
                                 bool set_attr) {
     auto pick = [&](auto kernel) {
@@ -550,22 +668,22 @@ inline void launch_staged_tiles(const StagedParams &sp, unsigned grid, int smem,
         kernel<<<grid, 256, smem, s>>>(sp);
     };
     if constexpr (FMT == 2) {            // FP4 rows are 32 codes (16 bytes): IT = 32
-        if (sp.OT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 32>);
-        else pick(mx_quantize_staged_kernel<FMT, BLK, 32, 32>);
+        if (sp.OT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 32, SR>);
+        else pick(mx_quantize_staged_kernel<FMT, BLK, 32, 32, SR>);
     } else {
-        if (sp.OT == 16 && sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 16>);
-        else if (sp.OT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 32>);
-        else if (sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 32, 16>);
-        else pick(mx_quantize_staged_kernel<FMT, BLK, 32, 32>);
+        if (sp.OT == 16 && sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 16, SR>);
+        else if (sp.OT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 16, 32, SR>);
+        else if (sp.IT == 16) pick(mx_quantize_staged_kernel<FMT, BLK, 32, 16, SR>);
+        else pick(mx_quantize_staged_kernel<FMT, BLK, 32, 32, SR>);
     }
 }
 
-template <int FMT>
+template <int FMT, bool SR>
 inline void launch_staged(const StagedParams &sp, unsigned grid, int smem, cudaStream_t s, cudaError_t &attr_err,
                           bool set_attr) {
-    if (sp.blk == kAlongI) launch_staged_tiles<FMT, kAlongI>(sp, grid, smem, s, attr_err, set_attr);
-    else if (sp.blk == kAlongO) launch_staged_tiles<FMT, kAlongO>(sp, grid, smem, s, attr_err, set_attr);
-    else launch_staged_tiles<FMT, kSquare>(sp, grid, smem, s, attr_err, set_attr);
+    if (sp.blk == kAlongI) launch_staged_tiles<FMT, kAlongI, SR>(sp, grid, smem, s, attr_err, set_attr);
+    else if (sp.blk == kAlongO) launch_staged_tiles<FMT, kAlongO, SR>(sp, grid, smem, s, attr_err, set_attr);
+    else launch_staged_tiles<FMT, kSquare, SR>(sp, grid, smem, s, attr_err, set_attr);
 }
 
 }  // namespace mqc

@@ -129,6 +129,31 @@ MQC_API mqc_status mqc_tensor_dims(mqc_role role, const mqc_conv *conv, int32_t 
 MQC_API mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *src_desc, const mqc_mx *mx,
                            void *codes, uint8_t *scales, void *codes_alt, void *stream);
 
+/* MX quantization with stochastic rounding of the elements (paper, section
+ * III-A, Eq. 6 and the text after it: the gradients are rounded
+ * stochastically, activations and weights to nearest).  Same arguments,
+ * blocks, scales and layout as mqc_quantize_mx; only the element rounding
+ * differs.  Each element x*2^-e lies between neighbouring magnitudes
+ * lo <= |x*2^-e| < hi of the format; with f = (|x*2^-e| - lo) / (hi - lo)
+ * and 16 random bits r, the magnitude is hi when r < f * 2^16, else lo
+ * (hi with probability f to within 2^-16); values beyond the largest finite
+ * magnitude saturate; the sign is kept.
+ *   seed, offset  the random bits of element (b, a) at spatial position pix
+ *           are bits 16*(j%4) .. 16*(j%4)+15 of word j/4 of the Philox4x64-10
+ *           block (Salmon et al., "Parallel random numbers: as easy as 1, 2,
+ *           3", SC 2011) with key (seed, 0) and counter (i/16, offset, 0, 0),
+ *           where i = (pix*d0 + b)*A16 + a, A16 = d1 rounded up to 16 and
+ *           j = i % 16.  The same (seed, offset) gives the same codes;
+ *           callers draw a new offset (or seed) per step.
+ * Requires mx->order == MQC_ORDER_BA (codes_alt may add the AB copy, with the
+ * same rounding decisions) and an NCHW-like source: element stride 1 along
+ * d3, d3 along d2, 16-byte aligned planes; else MQC_ERR_UNSUPPORTED before
+ * any launch.
+ * Errors: as mqc_quantize_mx, and MQC_ERR_UNSUPPORTED. */
+MQC_API mqc_status mqc_quantize_mx_sr(const float *src, const mqc_t4 *src_desc, const mqc_mx *mx,
+                              void *codes, uint8_t *scales, void *codes_alt, uint64_t seed,
+                              uint64_t offset, void *stream);
+
 /* Channel-batch-first im2col on quantized X (paper, section IV-A): the
  * explicit expansion X'_{Cin,N} of shape (Kh Kw Cin) x (Hout Wout N).  The
  * output is the quantized layout above for a tensor with spatial P x Q,
@@ -162,6 +187,9 @@ MQC_API int64_t mqc_im2col_cbf_codes_bytes(const mqc_conv *conv, const mqc_mx *m
  *   wq, ws  W quantized with blocks along C: block A32 or SQ32, order BA.
  *   y       fp32 output [N][K][P][Q] (overwritten).
  *   workspace, workspace_bytes: at least mqc_conv2d_fwd_workspace_bytes().
+ * Limits: R*S <= 64 kernel taps and stride_h*stride_w <= 4 (one activation
+ * tensor map per stride phase); otherwise MQC_ERR_UNSUPPORTED before any
+ * launch.
  * Errors: MQC_ERR_INVALID, MQC_ERR_UNSUPPORTED, MQC_ERR_ALIGNMENT, MQC_ERR_CUDA,
  * MQC_ERR_WORKSPACE. */
 MQC_API mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_mx *xf,
@@ -169,6 +197,34 @@ MQC_API mqc_status mqc_conv2d_fwd(const void *xq, const uint8_t *xs, const mqc_m
                           const mqc_conv *conv, float *y,
                           void *workspace, size_t workspace_bytes, void *stream);
 MQC_API size_t mqc_conv2d_fwd_workspace_bytes(const mqc_conv *conv, const mqc_mx *xf, const mqc_mx *wf);
+
+/* Activations the quantized forward output can apply before quantizing. */
+typedef enum { MQC_ACT_NONE = 0, MQC_ACT_RELU = 1, MQC_ACT_SILU = 2 } mqc_act;
+
+/* Forward convolution whose output leaves the GEMM already quantized as the
+ * next layer's input (the paper's flow of section V and Fig. 4: the
+ * activation computed by a layer is on-chip, is quantized there and only the
+ * quantized tensor is stored).  Same GEMM and operand requirements as
+ * mqc_conv2d_fwd; the epilogue applies `act` to the fp32 accumulators
+ * (MQC_ACT_RELU: max(x, 0); MQC_ACT_SILU: x / (1 + exp(-x)) in fp32), then
+ * MX-quantizes the result Y [N][K][P][Q] as a tensor with B-axis N, A-axis
+ * K and spatial P x Q, exactly as mqc_quantize_mx would quantize that fp32
+ * tensor (round-to-nearest-even, same scale rule and layout).
+ *   yf      format (E4M3, E5M2 or E2M1), block (A32 or SQ32) and order (BA).
+ *   yq, ys  codes and scales: mqc_codes_bytes / mqc_scales_bytes of yf with
+ *           dims (N, K, P, Q).
+ *   yq_alt  optional (NULL): the same codes in order AB (the weight
+ *           gradient's operand order), as mqc_quantize_mx's codes_alt.
+ *   y       optional (NULL): an fp32 copy [N][K][P][Q] of the activated
+ *           output that was quantized (for checking; the point of this call
+ *           is not to write it).
+ *   act     an mqc_act value.
+ * Errors: as mqc_conv2d_fwd; MQC_ERR_UNSUPPORTED for order AB or B32. */
+MQC_API mqc_status mqc_conv2d_fwd_quant(const void *xq, const uint8_t *xs, const mqc_mx *xf,
+                                const void *wq, const uint8_t *ws, const mqc_mx *wf,
+                                const mqc_conv *conv, int32_t act, const mqc_mx *yf, void *yq,
+                                uint8_t *ys, void *yq_alt, float *y, void *workspace,
+                                size_t workspace_bytes, void *stream);
 
 /* Input gradient, Eq. 2: G_X = W^T * G_Y as the GEMM
  * G_X'{Cin,N} = W_f^T . G_Yf{Cout,N} of section IV-B, computed directly as a
@@ -182,7 +238,7 @@ MQC_API size_t mqc_conv2d_fwd_workspace_bytes(const mqc_conv *conv, const mqc_mx
  * first, and the results are stored depth-to-space.  Otherwise one implicit
  * GEMM per output stride phase, up to four phases per kernel launch, their
  * tiles interleaved so that the phases' outputs (which interleave in memory)
- * are written together.  stride_h * stride_w must be at most 64.
+ * are written together.  R*S <= 64; stride_h and stride_w at most 64.
  *   wq, ws  W quantized with blocks along K: block B32 or SQ32, order AB.
  *   gq, gs  G_Y quantized with blocks along K: block A32 or SQ32, order BA.
  *   gx      fp32 output [N][C][H][W] (overwritten).
@@ -205,6 +261,7 @@ MQC_API size_t mqc_conv2d_bwd_data_workspace_bytes(const mqc_conv *conv, const m
  *           mqc_conv2d_bwd_weight_workspace_bytes(); may be NULL when that
  *           size is 0.
  * The split-K reduction is deterministic (fixed order).
+ * Limits: R*S <= 64 and stride_h*stride_w <= 4, as mqc_conv2d_fwd.
  * Errors: as mqc_conv2d_fwd. */
 MQC_API mqc_status mqc_conv2d_bwd_weight(const void *gq, const uint8_t *gs, const mqc_mx *gf,
                                  const void *xq, const uint8_t *xs, const mqc_mx *xf,

@@ -94,6 +94,20 @@ def test_invalid_arguments_rejected_before_launch(mqc):
     # a convolution whose kernel is larger than the padded input
     assert mqc.mqc_conv2d_fwd(p, p, mx, p, p, mx, mqc.conv_desc(1, 32, 2, 2, 8, 5, 5, 1, 1), p, None, 0, None) == -1
     assert mqc.lib.mqc_debug_expire_wait(10, None) == -1
+    # stochastic rounding: primary order BA and an NCHW-like source only
+    assert mqc.mqc_quantize_mx_sr(ctypes.c_void_p(16), d, mqc.MX(0, 2, 1), ctypes.c_void_p(16), ctypes.c_void_p(16),
+                                  None, 1, 0, None) == -2
+    dt = mqc.T4(2, 32, 8, 8, 2048, 64, 1, 8)     # H and W swapped in memory
+    assert mqc.mqc_quantize_mx_sr(ctypes.c_void_p(16), dt, mx, ctypes.c_void_p(16), ctypes.c_void_p(16),
+                                  None, 1, 0, None) == -2
+    assert "quantize_mx_sr" in mqc.lib.mqc_last_error_message().decode()
+    # forward and weight gradient: at most four stride phases (stride_h * stride_w <= 4)
+    s3 = mqc.conv_desc(2, 32, 12, 12, 32, 3, 3, 3, 1)
+    assert mqc.mqc_conv2d_fwd(p, p, mx, p, p, mx, s3, p, None, 0, None) == -2
+    assert "stride product" in mqc.lib.mqc_last_error_message().decode()
+    sq_ab = mqc.MX(0, 2, 1)
+    assert mqc.mqc_conv2d_bwd_weight(p, p, sq_ab, p, p, sq_ab, s3, p, None, 0, None) == -2
+    assert mqc.mqc_conv2d_bwd_weight_noalloc(p, p, sq_ab, p, p, sq_ab, s3, p, None) == -2
 
 
 def test_gemm_workspace_sizes_cover_widened_fp4_operands(mqc):

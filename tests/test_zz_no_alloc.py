@@ -6,10 +6,14 @@ loops that cannot pay for an allocation per call.  This entry point keeps its
 split-K partial sums in a fixed array inside the library instead of a caller
 workspace.  Here it is called twice in a row through the C ABI (different
 problems, so the second call reuses the array the first one filled) and each
-result is compared with the workspace entry point's, within the tolerance the
-parity tests use: |diff| <= 1e-3 * sum|a*b| + 1e-6 per element, sum|a*b| from
-the oracle.  The file sorts last so that a failure here stops a run only
-after every other test has run.
+result is compared with the workspace entry point's.  Both run the same plan
+and the same fixed-order split-K reduction, so the results must be identical
+bit for bit (a partial sum left over from the previous call would show); they
+are also checked against the oracle's tolerance, |diff| <= 1e-3 * sum|a*b| +
+1e-6 per element.  A problem whose scratch exceeds the array is rejected with
+MQC_ERR_WORKSPACE before anything runs, leaving the output untouched.  The
+file sorts last so that a failure here stops a run only after every other
+test has run.
 """
 import ctypes
 
@@ -59,4 +63,34 @@ def test_noalloc_weight_gradient_matches_workspace_entry_point(mqc, orc):
         a = out.cpu().numpy().astype(np.float64)
         b = ref.cpu().numpy().astype(np.float64)
         assert np.isfinite(a).all()
+        assert torch.equal(out, ref), f"call {i}: no-alloc result is not bit-identical to the workspace call"
         assert (np.abs(a - b) <= 1e-3 * sabs + 1e-6).all(), f"call {i}: no-alloc result differs"
+
+
+def test_noalloc_rejects_problems_above_the_static_scratch(mqc):
+    """A weight gradient whose split-K partials need more than the static
+    array returns MQC_ERR_WORKSPACE and launches nothing: the NaN-filled
+    output is left as it was."""
+    import torch
+    # E2M1 output gradients: their widened copy alone (one byte per element,
+    # 64 x 128 x 56 x 56 = 25.7 MB) is larger than the array, whatever the
+    # split-K plan
+    N, C, H, W, K, R, S, st, pad = 64, 128, 56, 56, 128, 3, 3, 1, 1
+    cv = mqc.conv_desc(N, C, H, W, K, R, S, st, pad)
+    gmx, xmx = mqc.MX(mqc.E2M1, mqc.SQ32, mqc.ORDER_AB), mqc.MX(mqc.E4M3, mqc.SQ32, mqc.ORDER_AB)
+    need = mqc.conv2d_bwd_weight_workspace_bytes(cv, gmx, xmx)
+    assert need > mqc.NOALLOC_SCRATCH_BYTES
+    # operands of the right sizes (zeros), so that nothing could read out of bounds
+    gq = torch.zeros(mqc.mqc_codes_bytes(gmx, N, K, H, W), dtype=torch.uint8, device="cuda")
+    gs = torch.zeros(mqc.mqc_scales_bytes(gmx, N, K, H, W), dtype=torch.uint8, device="cuda")
+    xq = torch.zeros(mqc.mqc_codes_bytes(xmx, N, C, H, W), dtype=torch.uint8, device="cuda")
+    xs = torch.zeros(mqc.mqc_scales_bytes(xmx, N, C, H, W), dtype=torch.uint8, device="cuda")
+    out = torch.full((K, C, R, S), float("nan"), dtype=torch.float32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    P_ = lambda t: ctypes.c_void_p(t.data_ptr())
+    code = mqc.mqc_conv2d_bwd_weight_noalloc(P_(gq), P_(gs), gmx, P_(xq), P_(xs), xmx, cv, P_(out), stream)
+    assert code == -6, mqc.STATUS.get(code, code)
+    assert "static" in mqc.lib.mqc_last_error_message().decode()
+    torch.cuda.synchronize()
+    mqc.check(mqc.get_device_status())
+    assert torch.isnan(out).all()

@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="mqc", choices=["mqc", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-extras", action="store_true",
+                    help="skip the fused step, the tensor-bound layers and the stochastic-rounding quantizer")
     ap.add_argument("--profile", default=None, metavar="CALL[,CALL...]",
                     help="profiling mode: build one layer, then run the listed calls (quantize_x, quantize_w, quantize_g, fwd, "
                          "dgrad, wgrad) --reps times and exit")
@@ -116,12 +118,13 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = None
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix=f"mqc_clocks_gpu{self.idx}_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
@@ -151,6 +154,10 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
+        try:
+            os.unlink(self.path)
+        except OSError:
+            pass
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         load = [s for s in sm if s > 0.5 * max(sm)] or sm
@@ -253,8 +260,12 @@ class LayerBuffers:
     def gemm_flops(self):
         return self.L.gemm_flops()
 
-    def gemm_bytes(self, op):
+    def gemm_bytes(self, op, nxt=None):
         qx, qw, qg = self.q["x"], self.q["w"], self.q["g"]
+        if op == "fwd_quant":
+            ny = nxt.q["x"]
+            return (qx.codes.numel() + qx.scales.numel() + qw.codes.numel() + qw.scales.numel()
+                    + ny.codes.numel() + ny.codes_alt.numel() + ny.scales.numel())
         if op == "fwd":
             return qx.codes.numel() + qx.scales.numel() + qw.codes.numel() + qw.scales.numel() + 4 * self.y.numel()
         if op == "dgrad":
@@ -274,10 +285,14 @@ class LayerBuffers:
         return 3 + 1 + dgrad + (2 if self.split_k else 1) + self.n_widen
 
 
-def run_layer(mqc, lb: LayerBuffers, workspace, stream, events=None, only=None):
+def run_layer(mqc, lb: LayerBuffers, workspace, stream, events=None, only=None, nxt=None, with_x=True):
     """All calls of one layer through the C ABI; `events` (optional) collects
     (name, start, end) CUDA events around every call on `stream`; `only`
-    (a tuple of call names) restricts the run to those calls (profiling)."""
+    (a tuple of call names) restricts the run to those calls (profiling).
+    With `nxt` (the next layer's buffers) the forward is "fwd_quant": its
+    epilogue applies SiLU and writes the next layer's quantized input (both
+    code orders) instead of the fp32 output; `with_x` False skips this
+    layer's own quantize_x (its input came from the previous forward)."""
     c_void = ctypes.c_void_p
     P = lambda t: c_void(t.data_ptr())
 
@@ -295,14 +310,27 @@ def run_layer(mqc, lb: LayerBuffers, workspace, stream, events=None, only=None):
             mqc.check(fn())
 
     for name, t in (("x", lb.x), ("w", lb.w), ("g", lb.g)):
+        if name == "x" and not with_x:
+            continue
         q = lb.q[name]
         timed(f"quantize_{name}", lambda q=q, t=t, name=name: mqc.mqc_quantize_mx(
             P(t), lb.desc[name], q.mx, P(q.codes), P(q.scales), P(q.codes_alt), stream))
+    if only is not None and "quantize_g_sr" in only:
+        # the output gradient with stochastically rounded elements (timed alone)
+        q = lb.q["g"]
+        timed("quantize_g_sr", lambda: mqc.mqc_quantize_mx_sr(
+            P(lb.g), lb.desc["g"], q.mx, P(q.codes), P(q.scales), P(q.codes_alt), 1234, 0, stream))
     qx, qw, qg = lb.q["x"], lb.q["w"], lb.q["g"]
     wq_ab, gq_ab, xq_ab = qw.other_order(), qg.other_order(), qx.other_order()
     wsp = P(workspace) if lb.ws_bytes else None
-    timed("fwd", lambda: mqc.mqc_conv2d_fwd(P(qx.codes), P(qx.scales), qx.mx, P(qw.codes), P(qw.scales), qw.mx,
-                                            lb.cv, P(lb.y), wsp, lb.ws_fwd, stream))
+    if nxt is not None:
+        ny = nxt.q["x"]
+        timed("fwd_quant", lambda: mqc.mqc_conv2d_fwd_quant(
+            P(qx.codes), P(qx.scales), qx.mx, P(qw.codes), P(qw.scales), qw.mx, lb.cv, mqc.ACT_SILU, ny.mx,
+            P(ny.codes), P(ny.scales), P(ny.codes_alt), None, wsp, lb.ws_fwd, stream))
+    else:
+        timed("fwd", lambda: mqc.mqc_conv2d_fwd(P(qx.codes), P(qx.scales), qx.mx, P(qw.codes), P(qw.scales),
+                                                qw.mx, lb.cv, P(lb.y), wsp, lb.ws_fwd, stream))
     timed("dgrad", lambda: mqc.mqc_conv2d_bwd_data(P(wq_ab.codes), P(wq_ab.scales), wq_ab.mx, P(qg.codes),
                                                    P(qg.scales), qg.mx, lb.cv, P(lb.gx), wsp, lb.ws_dgrad, stream))
     timed("wgrad", lambda: mqc.mqc_conv2d_bwd_weight(P(gq_ab.codes), P(gq_ab.scales), gq_ab.mx, P(xq_ab.codes),
@@ -398,29 +426,88 @@ def capture_graph(torch, fn):
     return g
 
 
-def graph_call_times(mqc, torch, lb, workspace, reps, names=CALLS):
-    """Device time (ms) of each named call of one layer: the call captured as
-    a CUDA graph and replayed `reps` times, each replay between a pair of
-    events and preceded by an L2 flush (a 256 MiB write)."""
+def graph_call_times(mqc, torch, lb, workspace, reps, names=CALLS, k=8, nxt=None):
+    """Device time (ms) of each named call of one layer, launch cost
+    amortised: one CUDA graph holds k (L2 flush, call) pairs, another the k
+    flushes alone (a 256 MiB write each, larger than the 126 MB L2); each is
+    replayed `reps` times between a pair of events and the call's time is
+    (median with calls - median of flushes) / k.  Returns lists of per-call
+    estimates (one per replay pair)."""
     cur = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    out = {}
-    for name in names:
-        g = capture_graph(torch, lambda: run_layer(mqc, lb, workspace, cur(), only=(name,)))
-        g.replay()
-        ev = []
-        for _ in range(reps):
+
+    def body(name):
+        for _ in range(k):
             flush.fill_(1)
+            if name is not None:
+                run_layer(mqc, lb, workspace, cur(), only=(name,), nxt=nxt if name == "fwd_quant" else None)
+
+    def timed(g):
+        out = []
+        for _ in range(reps):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             g.replay()
             e1.record()
-            ev.append((e0, e1))
+            out.append((e0, e1))
         torch.cuda.synchronize()
-        out[name] = [a.elapsed_time(b) for a, b in ev]
+        return [a.elapsed_time(b) for a, b in out]
+
+    g_flush = capture_graph(torch, lambda: body(None))
+    g_flush.replay()
+    t_flush = statistics.median(timed(g_flush))
+    out = {}
+    for name in names:
+        g = capture_graph(torch, lambda: body(name))
+        g.replay()
+        out[name] = [max(1e-6, (t - t_flush) / k) for t in timed(g)]
         del g
+    del g_flush
     mqc.check(mqc.get_device_status())
     return out
+
+
+def graph_fn_times(mqc, torch, fn, reps, k=8):
+    """graph_call_times for any callable that issues C-ABI calls on the
+    current stream: (median of k (flush, fn) pairs - median of k flushes) / k."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def body(with_fn):
+        for _ in range(k):
+            flush.fill_(1)
+            if with_fn:
+                fn()
+
+    def timed(g):
+        out = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            out.append((e0, e1))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in out]
+
+    gf = capture_graph(torch, lambda: body(False))
+    gf.replay()
+    t_flush = statistics.median(timed(gf))
+    g = capture_graph(torch, lambda: body(True))
+    g.replay()
+    out = [max(1e-6, (t - t_flush) / k) for t in timed(g)]
+    del g, gf
+    mqc.check(mqc.get_device_status())
+    return out
+
+
+def quantize_weights(mqc, layers, stream):
+    """Every layer's weights in one launch (mqc_quantize_mx_batch): the
+    weights are quantized together once per weight update."""
+    P = lambda t: t.data_ptr()
+    qs = [lb.q["w"] for lb in layers]
+    mqc.check(mqc.mqc_quantize_mx_batch([P(lb.w) for lb in layers], [lb.desc["w"] for lb in layers], qs[0].mx,
+                                        [P(q.codes) for q in qs], [P(q.scales) for q in qs],
+                                        [P(q.codes_alt) for q in qs], stream))
 
 
 def sweep(mqc, torch, wl, args):
@@ -486,17 +573,93 @@ def profile_call(mqc, torch, wl, args):
     """Runs one layer's calls once (so every operand exists), then the chosen
     call `reps` more times; used as the small case of an ncu capture."""
     lb = LayerBuffers(mqc, torch, wl.layers[args.layer], wl, args.layer, False)
+    names = tuple(args.profile.split(","))
+    # fwd_quant writes the next layer's quantized input
+    nxt = (LayerBuffers(mqc, torch, wl.layers[args.layer + 1], wl, args.layer + 1, False)
+           if "fwd_quant" in names else None)
     workspace = torch.empty(max(lb.ws_bytes, 16), dtype=torch.uint8, device="cuda")
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     run_layer(mqc, lb, workspace, stream)
     events = []
     for _ in range(args.reps):
-        run_layer(mqc, lb, workspace, stream, events, only=tuple(args.profile.split(",")))
+        run_layer(mqc, lb, workspace, stream, events, only=names, nxt=nxt)
     torch.cuda.synchronize()
     mqc.check(mqc.get_device_status())
     ms = [e0.elapsed_time(e1) for _, e0, e1 in events]
     print(json.dumps({"profile": args.profile, "layer": args.layer, "ms": ms}), flush=True)
     return 0
+
+
+# --------------------------------------------------------------------------- extras
+def fused_step(mqc, torch, args, layers, workspace, layer_calls, allreduce_gw, step_flops, pk, world):
+    """The training step with quantize-in-epilogue (the paper's section V /
+    Fig. 4 flow): forwards 0-6 apply SiLU and write the next layer's SQ32
+    E4M3 codes (both orders) and scales, so layers 1-7 skip quantize_x and
+    no fp32 activation is written.  Same flops as the step; its own graph,
+    timed like the step, plus the per-call time of every fused forward."""
+    g = capture_graph(torch, lambda: layer_calls(fused=True))
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+        allreduce_gw()
+    torch.cuda.synchronize()
+    mqc.check(mqc.get_device_status())
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        g.replay()
+        allreduce_gw()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, torch.device("cuda"))
+    mqc.check(mqc.get_device_status())
+    del g
+    calls = []
+    for i in range(len(layers) - 1):
+        lb, nxt = layers[i], layers[i + 1]
+        t = statistics.median(graph_call_times(mqc, torch, lb, workspace, 5, names=("fwd_quant",), nxt=nxt)["fwd_quant"])
+        byt = lb.gemm_bytes("fwd_quant", nxt)
+        calls.append({"layer": i, "call": "fwd_quant", "ms": round(t, 5), "bytes": byt,
+                      "frac_of_hbm_roofline": round(byt / (pk["hbm_gbs"] * 1e9) * 1e3 / t, 4)})
+    # one batched weight launch; layers 1-7 have no quantize_x
+    launches = sum(lb.launches(mqc) for lb in layers) - 2 * (len(layers) - 1)
+    return {"value": world * step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "gpu_launches_per_step": launches,
+            "what": "forwards 0-6 quantize their SiLU output in the epilogue as the next layer's SQ32 E4M3 input "
+                    "(both orders); layers 1-7 skip quantize_x; no fp32 activation written",
+            "calls": calls}
+
+
+TENSOR_BOUND = ((4, "latent-replay N=128 C=K=256 14x14, X E2M1, W E4M3, G_Y E5M2"),
+                ((5, "fp8", 128), "large-batch N=128 C=K=128 80x80 MXFP8"),
+                ((5, "fp4", 128), "large-batch N=128 C=K=128 80x80 MXFP4"))
+
+
+def tensor_bound_layers(mqc, torch, pk):
+    """Per-call TFLOP/s of the three GEMMs on the tensor-bound configurations
+    (latent-replay block, large-batch layer at N=128 in MXFP8 and MXFP4) as
+    fractions of the dense MXFP8 peak (2 x the measured bf16 peak) and, for
+    all-FP4 operands, of the dense MXFP4 peak (2 x MXFP8, the nominal ratio)."""
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    out = []
+    for key, what in TENSOR_BOUND:
+        wl = synth.WORKLOADS[key]
+        lb = LayerBuffers(mqc, torch, wl.layers[0], wl, 0, False)
+        ws = torch.empty(max(lb.ws_bytes, 16), dtype=torch.uint8, device="cuda")
+        run_layer(mqc, lb, ws, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        per = graph_call_times(mqc, torch, lb, ws, 5, names=("fwd", "dgrad", "wgrad"), k=4)
+        all_fp4 = wl.fmt_x == wl.fmt_w == wl.fmt_g == synth.E2M1
+        for name, v in per.items():
+            ms = statistics.median(v)
+            tf = lb.gemm_flops() / (ms * 1e-3) / 1e12
+            out.append({"workload": wl.name, "what": what, "call": name, "ms": round(ms, 5), "tflops": round(tf, 1),
+                        "frac_of_mxfp8_peak": round(tf / fp8_peak, 4),
+                        "frac_of_mxfp4_peak": round(tf / (2 * fp8_peak), 4) if all_fp4 else None})
+        del lb, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 # --------------------------------------------------------------------------- main arm
@@ -523,7 +686,8 @@ def main(argv=None):
     workspace = torch.empty(max(ws_max, 16), dtype=torch.uint8, device="cuda")
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     step_flops = sum(3 * lb.gemm_flops() for lb in layers)
-    launches_per_step = sum(lb.launches(mqc) for lb in layers)
+    # one batched launch quantizes every layer's weights
+    launches_per_step = sum(lb.launches(mqc) for lb in layers) - (len(layers) - 1)
     gws = [lb.gw for lb in layers]
 
     def allreduce_gw():
@@ -533,26 +697,29 @@ def main(argv=None):
         return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
     wstream = torch.cuda.Stream()
-    rest = tuple(c for c in CALLS if c != "quantize_w")
+    rest = tuple(c for c in CALLS if c != "quantize_w") + ("fwd_quant",)
 
-    def layer_calls(events=None):
+    def layer_calls(events=None, fused=False):
         # the weights are known when the step starts (as right after a weight
         # update), so their quantizations run on a second stream, overlapping
-        # the activation work; each layer's GEMMs wait for its own weights
+        # the activation work; each layer's GEMMs wait for its own weights.
+        # fused: each forward but the last applies SiLU and writes the next
+        # layer's quantized input in its epilogue (section V / Fig. 4 of the
+        # paper), so layers 1-7 have no quantize_x and no fp32 activation
+        # is written or read again
         main = torch.cuda.current_stream()
         fork = torch.cuda.Event()
         fork.record(main)
         wstream.wait_event(fork)
-        ready = []
         with torch.cuda.stream(wstream):
-            for lb in layers:
-                run_layer(mqc, lb, workspace, cur_stream(), only=("quantize_w",))
-                ev = torch.cuda.Event()
-                ev.record(wstream)
-                ready.append(ev)
-        for lb, ev in zip(layers, ready):
-            main.wait_event(ev)
-            run_layer(mqc, lb, workspace, cur_stream(), events, only=rest)
+            quantize_weights(mqc, layers, cur_stream())
+            ready = torch.cuda.Event()
+            ready.record(wstream)
+        for i, lb in enumerate(layers):
+            if i == 0:
+                main.wait_event(ready)
+            nxt = layers[i + 1] if fused and i + 1 < len(layers) else None
+            run_layer(mqc, lb, workspace, cur_stream(), events, only=rest, nxt=nxt, with_x=not fused or i == 0)
 
     def step(events=None):
         layer_calls(events)
@@ -597,12 +764,20 @@ def main(argv=None):
     # per-call durations: each call as its own graph (cold L2, no host gaps)
     per = {}
     for li, lb in enumerate(layers):
-        for name, v in graph_call_times(mqc, torch, lb, workspace, max(3, min(args.steps, 10))).items():
+        for name, v in graph_call_times(mqc, torch, lb, workspace, max(3, min(args.steps, 10)),
+                                        names=tuple(c for c in CALLS if c != "quantize_w")).items():
             per[(li, name)] = v
+    cur = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    per[("all", "quantize_w")] = graph_fn_times(mqc, torch, lambda: quantize_weights(mqc, layers, cur()),
+                                                max(3, min(args.steps, 10)))
     calls = []
     for (li, name), v in per.items():
-        lb = layers[li]
         d = statistics.mean(v)
+        if li == "all":
+            byt = sum(lb.quant_bytes("w") for lb in layers)
+            calls.append({"layer": "all", "call": name, "ms": d, "bytes": byt, "flops": 0})
+            continue
+        lb = layers[li]
         if name.startswith("quantize"):
             byt = lb.quant_bytes(name[-1])
             calls.append({"layer": li, "call": name, "ms": d, "bytes": byt, "flops": 0})
@@ -645,8 +820,7 @@ def main(argv=None):
             for lb in layers:
                 for dst, src in zip((lb.x, lb.w, lb.g), lb.host_in):
                     dst.copy_(src, non_blocking=True)
-            step_graph.replay()
-            allreduce_gw()
+            step()      # the 48 C-ABI calls of the step, issued one by one from the host
             for lb in layers:
                 for dst, src in zip(lb.host_out, (lb.y, lb.gx, lb.gw)):
                     dst.copy_(src, non_blocking=True)
@@ -655,7 +829,27 @@ def main(argv=None):
         barrier()
         ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, torch.device("cuda"))
         e2e = {"value": world * step_flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems,
+               "how": "fp32 X, W, G_Y of every layer copied from pinned host memory, the step's C-ABI calls "
+                      "issued one by one (no graph), Y, G_X, G_W copied back, every step"}
+
+    # ---- extras: the fused step, the tensor-bound layers, the stochastic-rounding quantizer
+    fused = tensor_bound = sr_quant = None
+    if not args.skip_extras:
+        fused = fused_step(mqc, torch, args, layers, workspace, layer_calls, allreduce_gw, step_flops, pk, world)
+        for c in fused["calls"]:       # what the fused forward replaces: the fp32 forward + the next quantize_x
+            c["ms_unfused"] = round(statistics.mean(per[(c["layer"], "fwd")])
+                                    + statistics.mean(per[(c["layer"] + 1, "quantize_x")]), 5)
+        tensor_bound = tensor_bound_layers(mqc, torch, pk)
+        lb0 = layers[0]
+        t_sr = statistics.median(graph_call_times(mqc, torch, lb0, workspace, 5, names=("quantize_g_sr",))
+                                 ["quantize_g_sr"])
+        t_rn = statistics.median(graph_call_times(mqc, torch, lb0, workspace, 5, names=("quantize_g",))["quantize_g"])
+        byt = lb0.quant_bytes("g")
+        sr_quant = {"call": "quantize_g_sr layer 0", "ms": t_sr, "gbs": byt / (t_sr * 1e-3) / 1e9,
+                    "frac_of_hbm": byt / (t_sr * 1e-3) / 1e9 / pk["hbm_gbs"], "ms_round_to_nearest": t_rn,
+                    "what": "G_Y 16x32x320x320 fp32 -> E5M2 SQ32, both orders, elements rounded stochastically "
+                            "with Philox4x64-10 bits"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
@@ -672,6 +866,7 @@ def main(argv=None):
             "quantizer_gbs": quant_gbs, "quantizer_frac_of_hbm": quant_gbs / pk["hbm_gbs"],
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
+            "fused_step": fused, "tensor_bound": tensor_bound, "sr_quantizer": sr_quant,
             "calls": [{k: (round(v, 5) if isinstance(v, float) else v) for k, v in c.items()} for c in calls],
         }
         print(json.dumps(line), flush=True)

@@ -33,7 +33,7 @@ EXPORTS = ("mqc_codes_bytes", "mqc_scales_bytes", "mqc_tensor_dims", "mqc_quanti
            "mqc_conv2d_bwd_weight", "mqc_conv2d_bwd_weight_workspace_bytes", "mqc_get_device_status",
            "mqc_debug_expire_wait", "mqc_status_string", "mqc_last_error_message", "mqc_version",
            "mqc_conv2d_bwd_weight_noalloc", "mqc_conv2d_fwd_workspace_bytes", "mqc_conv2d_bwd_data_workspace_bytes",
-           "mqc_quantize_mx_sr", "mqc_conv2d_fwd_quant")
+           "mqc_quantize_mx_sr", "mqc_conv2d_fwd_quant", "mqc_quantize_mx_batch")
 ACT_NONE, ACT_RELU, ACT_SILU = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "mqc_tensor_dims": (i32, [i32, P(Conv), P(i32)]),
         "mqc_quantize_mx": (i32, [vp, P(T4), P(MX), vp, vp, vp, vp]),
         "mqc_quantize_mx_sr": (i32, [vp, P(T4), P(MX), vp, vp, vp, ctypes.c_uint64, ctypes.c_uint64, vp]),
+        "mqc_quantize_mx_batch": (i32, [i32, P(vp), P(T4), P(MX), P(vp), P(vp), P(vp), vp]),
         "mqc_im2col_cbf": (i32, [vp, vp, P(Conv), P(MX), vp, vp, vp]),
         "mqc_im2col_cbf_scales_bytes": (i64, [P(Conv), P(MX)]),
         "mqc_im2col_cbf_codes_bytes": (i64, [P(Conv), P(MX)]),
@@ -121,6 +122,16 @@ def mqc_quantize_mx(src_ptr, desc: T4, mx: MX, codes_ptr, scales_ptr, codes_alt_
 def mqc_quantize_mx_sr(src_ptr, desc: T4, mx: MX, codes_ptr, scales_ptr, codes_alt_ptr, seed, offset, stream) -> int:
     return lib.mqc_quantize_mx_sr(src_ptr, ctypes.byref(desc), ctypes.byref(mx), codes_ptr, scales_ptr,
                                   codes_alt_ptr, seed, offset, stream)
+
+
+def mqc_quantize_mx_batch(srcs, descs, mx: MX, codes, scales, codes_alt, stream) -> int:
+    """One launch for len(srcs) tensors; pointer lists (ints or c_void_p),
+    T4 descriptors, one shared MX; codes_alt a list or None."""
+    n = len(srcs)
+    arr = lambda xs: (ctypes.c_void_p * n)(*[x.value if isinstance(x, ctypes.c_void_p) else x for x in xs])
+    alt = arr(codes_alt) if codes_alt is not None else None
+    return lib.mqc_quantize_mx_batch(n, arr(srcs), (T4 * n)(*descs), ctypes.byref(mx), arr(codes), arr(scales),
+                                     alt, stream)
 
 
 def mqc_im2col_cbf(codes_ptr, scales_ptr, conv: Conv, mx: MX, codes_out_ptr, scales_out_ptr, stream) -> int:
@@ -248,6 +259,27 @@ def quantize_mx(src, fmt: int, block: int, order: int, both_orders: bool = False
         check(mqc_quantize_mx_sr(_ptr(src), desc, mx, _ptr(codes), _ptr(scales), _ptr(alt), sr_seed, sr_offset,
                                  _stream()))
     return Quantized(codes, scales, (d0, d1, d2, d3), mx, alt)
+
+
+def quantize_mx_batch(srcs, fmt: int, block: int, order: int, both_orders: bool = False) -> list:
+    """MX-quantize several 4-D fp32 CUDA tensors in one launch (same format,
+    block mode and order): one Quantized per tensor."""
+    torch = _torch()
+    mx = MX(fmt, block, order)
+    outs = []
+    for src in srcs:
+        assert src.is_cuda and src.dtype == torch.float32 and src.dim() == 4
+        d = tuple(src.shape)
+        codes = torch.empty(mqc_codes_bytes(mx, *d), dtype=torch.uint8, device=src.device)
+        scales = torch.empty(mqc_scales_bytes(mx, *d), dtype=torch.uint8, device=src.device)
+        alt = (torch.empty(mqc_codes_bytes(MX(fmt, block, 1 - order), *d), dtype=torch.uint8, device=src.device)
+               if both_orders else None)
+        outs.append(Quantized(codes, scales, d, mx, alt))
+    descs = [T4(*s.shape, *s.stride()) for s in srcs]
+    check(mqc_quantize_mx_batch([s.data_ptr() for s in srcs], descs, mx, [q.codes.data_ptr() for q in outs],
+                                [q.scales.data_ptr() for q in outs],
+                                [q.codes_alt.data_ptr() for q in outs] if both_orders else None, _stream()))
+    return outs
 
 
 def im2col_cbf(xq: Quantized, cv: Conv):

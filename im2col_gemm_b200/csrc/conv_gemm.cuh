@@ -319,11 +319,11 @@ struct KitWalker {
 // A template parameter as well, so that the one-tile kernel carries no
 // sub-tile loops.
 // Activations the quantized forward output can apply before quantizing:
-// 0 none, 1 ReLU, 2 SiLU (x * sigmoid(x), with CUDA's expf and an IEEE
-// division).
+// 0 none, 1 ReLU, 2 SiLU x / (1 + e^-x), with CUDA's fast exponential and
+// division intrinsics (a few ulp; the codes are decided on this fp32 value).
 __device__ __forceinline__ float activate(float x, int act) {
     if (act == 1) return fmaxf(x, 0.0f);
-    if (act == 2) return x / (1.0f + expf(-x));
+    if (act == 2) return __fdividef(x, 1.0f + __expf(-x));
     return x;
 }
 
@@ -389,12 +389,24 @@ __device__ __forceinline__ void qout_chunk(const GemmParams &p, const uint32_t (
     const int K = p.Ncols;
     float v[32];
     float m = 0.0f;
+    if (row_ok && k0 + 32 <= K) {
+        // whole chunk inside the output: no per-element masks
+        if (p.q_act == 2) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const float x = (row_ok && k0 + j < K) ? activate(__uint_as_float(r[j]), p.q_act) : 0.0f;
-        v[j] = x;
-        m = fmaxf(m, fabsf(x));
+            for (int j = 0; j < 32; ++j) v[j] = activate(__uint_as_float(r[j]), 2);
+        } else if (p.q_act == 1) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = fmaxf(__uint_as_float(r[j]), 0.0f);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = (row_ok && k0 + j < K) ? activate(__uint_as_float(r[j]), p.q_act) : 0.0f;
     }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
     if (p.q_y != nullptr && row_ok) {
         // optional fp32 copy, NCHW [N][K][P][Q]: p.os_* give the strides
         float *op = p.q_y + static_cast<int64_t>(n) * p.os_n + static_cast<int64_t>(pix) + static_cast<int64_t>(k0) * p.os_c;
@@ -440,13 +452,15 @@ __device__ __forceinline__ void qout_chunk(const GemmParams &p, const uint32_t (
 #pragma unroll
     for (int q = 0; q < 8; ++q) s_tr[lane * 9 + q] = w[q];
     __syncwarp();
-    const uint8_t *tb = reinterpret_cast<const uint8_t *>(s_tr);
+    // lane L: byte L % 4 of word L / 4 of every row, four rows per output word
     uint32_t t[8];
+    const uint32_t sel = static_cast<uint32_t>(lane & 3) | (static_cast<uint32_t>(4 + (lane & 3)) << 4);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-        t[q] = 0u;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) t[q] |= static_cast<uint32_t>(tb[(4 * q + b) * 36 + lane]) << (8 * b);
+        const uint32_t *col = s_tr + (lane >> 2);
+        const uint32_t lo = __byte_perm(col[(4 * q) * 9], col[(4 * q + 1) * 9], sel);
+        const uint32_t hi = __byte_perm(col[(4 * q + 2) * 9], col[(4 * q + 3) * 9], sel);
+        t[q] = __byte_perm(lo, hi, 0x5410u);
     }
     // pixels and row validity of the lanes' groups
     const int pix0 = __shfl_sync(0xFFFFFFFFu, pix, 0), pix1 = __shfl_sync(0xFFFFFFFFu, pix, 16);

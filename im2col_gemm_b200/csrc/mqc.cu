@@ -466,8 +466,9 @@ mqc_status mqc_quantize_mx_sr(const float *src, const mqc_t4 *d, const mqc_mx *m
 
 }  // extern "C"
 
-static mqc_status quantize_impl(const float *src, const mqc_t4 *d, const mqc_mx *mx, void *codes, uint8_t *scales,
-                                void *codes_alt, void *stream, const SrArgs *sr) {
+// Argument checks shared by the quantization entry points.
+static mqc_status check_quant_args(const float *src, const mqc_t4 *d, const mqc_mx *mx, const void *codes,
+                                   const uint8_t *scales, const void *codes_alt) {
     if (src == nullptr || d == nullptr || codes == nullptr || scales == nullptr || !mx_ok(mx))
         return fail(MQC_ERR_INVALID, "quantize: null pointer or bad mx descriptor");
     if (d->d0 <= 0 || d->d1 <= 0 || d->d2 <= 0 || d->d3 <= 0)
@@ -477,18 +478,14 @@ static mqc_status quantize_impl(const float *src, const mqc_t4 *d, const mqc_mx 
         return fail(MQC_ERR_ALIGNMENT, "quantize: codes not 16-byte aligned");
     if (static_cast<int64_t>(d->d2) * d->d3 > (int64_t(1) << 31) - 64)
         return fail(MQC_ERR_INVALID, "quantize: too many spatial positions");
-    // staged kernel: positions contiguous (element stride 1 along W, W along
-    // H), every plane 16-byte aligned
-    const bool staged = d->s3 == 1 && d->s2 == d->d3 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 &&
-                        d->s0 % 4 == 0 && d->s1 % 4 == 0;
-    if (sr != nullptr && (mx->order != MQC_ORDER_BA || !staged))
-        return fail(MQC_ERR_UNSUPPORTED,
-                    "quantize_mx_sr: needs order BA and an NCHW-like source (contiguous, 16-byte aligned planes)");
-    DevInfo *dv;
-    mqc_status st = dev_info(dv);
-    if (st != MQC_OK) return st;
+    return MQC_OK;
+}
 
-    QuantParams p{};
+// Parameters and tile count of the generic quantizer (mx_quantize_kernel)
+// for one tensor; `it` = 16 or 32 codes per tile row (0: choose).
+static void generic_quant_params(const float *src, const mqc_t4 *d, const mqc_mx *mx, void *codes, uint8_t *scales,
+                                 void *codes_alt, int it_req, QuantParams &p, int &it, int64_t &tiles) {
+    p = QuantParams{};
     p.src = src;
     p.sb = d->s0;
     p.sa = d->s1;
@@ -517,14 +514,36 @@ static mqc_status quantize_impl(const float *src, const mqc_t4 *d, const mqc_mx 
     p.emax = emax_elem(mx->fmt);
     // tile: IT = 16 when the innermost axis holds at most 16 FP8 codes, OT = 16
     // when the other axis (and its padded copy) has at most 16 elements
-    const int it = (!fp4 && p.I1 <= 16) ? 16 : 32;
+    it = it_req ? it_req : ((!fp4 && p.I1 <= 16) ? 16 : 32);
     p.OT = (!fp4 && p.O <= 16 && (codes_alt == nullptr || p.O2 <= 16)) ? 16 : 32;
     const int gsize = p.OT == 16 ? 2 : 1;
     p.nPT = static_cast<int32_t>(ceil_div(p.npix, 32 * gsize));
     p.nIT = static_cast<int32_t>(ceil_div(p.I1, it));
     p.nOT = static_cast<int32_t>(ceil_div(codes_alt ? std::max(p.O, p.O2) : p.O, p.OT));
-    const int64_t tiles = int64_t(p.nPT) * p.nOT * p.nIT;
+    tiles = int64_t(p.nPT) * p.nOT * p.nIT;
+}
+
+static mqc_status quantize_impl(const float *src, const mqc_t4 *d, const mqc_mx *mx, void *codes, uint8_t *scales,
+                                void *codes_alt, void *stream, const SrArgs *sr) {
+    mqc_status st = check_quant_args(src, d, mx, codes, scales, codes_alt);
+    if (st != MQC_OK) return st;
+    // staged kernel: positions contiguous (element stride 1 along W, W along
+    // H), every plane 16-byte aligned
+    const bool staged = d->s3 == 1 && d->s2 == d->d3 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 &&
+                        d->s0 % 4 == 0 && d->s1 % 4 == 0;
+    if (sr != nullptr && (mx->order != MQC_ORDER_BA || !staged))
+        return fail(MQC_ERR_UNSUPPORTED,
+                    "quantize_mx_sr: needs order BA and an NCHW-like source (contiguous, 16-byte aligned planes)");
+    DevInfo *dv;
+    if ((st = dev_info(dv)) != MQC_OK) return st;
+
+    QuantParams p;
+    int it;
+    int64_t tiles;
+    generic_quant_params(src, d, mx, codes, scales, codes_alt, 0, p, it, tiles);
     if (tiles > (int64_t(1) << 31) - 1) return fail(MQC_ERR_INVALID, "quantize: tensor too large");
+    const bool map_a = mx->order == MQC_ORDER_BA;
+    const bool fp4 = mx->fmt == MQC_E2M1;
     const bool along_i = (mx->block == MQC_BLOCK_A32) == map_a && mx->block != MQC_BLOCK_SQ32;
     const int blk = mx->block == MQC_BLOCK_SQ32 ? kSquare : (along_i ? kAlongI : kAlongO);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -575,6 +594,47 @@ static mqc_status quantize_impl(const float *src, const mqc_t4 *d, const mqc_mx 
     if (e != cudaSuccess) return cuda_fail(e, "mx_quantize_kernel launch");
     return MQC_OK;
 }
+
+extern "C" {
+
+mqc_status mqc_quantize_mx_batch(int32_t count, const float *const *srcs, const mqc_t4 *descs, const mqc_mx *mx,
+                                 void *const *codes, uint8_t *const *scales, void *const *codes_alt, void *stream) {
+    if (count < 1 || count > kMaxQuantBatch || srcs == nullptr || descs == nullptr || codes == nullptr ||
+        scales == nullptr || !mx_ok(mx))
+        return fail(MQC_ERR_INVALID, "quantize_mx_batch: count must be 1..%d, with non-null arrays", kMaxQuantBatch);
+    const bool dual = codes_alt != nullptr;
+    QuantBatch b{};
+    b.n = count;
+    int64_t total = 0;
+    for (int i = 0; i < count; ++i) {
+        void *alt = dual ? codes_alt[i] : nullptr;
+        if (dual && alt == nullptr)
+            return fail(MQC_ERR_INVALID, "quantize_mx_batch: codes_alt[%d] is null (all or none)", i);
+        mqc_status st = check_quant_args(srcs[i], &descs[i], mx, codes[i], scales[i], alt);
+        if (st != MQC_OK) return st;
+        int it;
+        int64_t tiles;
+        generic_quant_params(srcs[i], &descs[i], mx, codes[i], scales[i], alt, 32, b.q[i], it, tiles);
+        b.tile0[i] = static_cast<int32_t>(total);
+        total += tiles;
+        if (total > (int64_t(1) << 31) - 1) return fail(MQC_ERR_INVALID, "quantize_mx_batch: tensors too large");
+    }
+    b.tile0[count] = static_cast<int32_t>(total);
+    DevInfo *dv;
+    mqc_status st = dev_info(dv);
+    if (st != MQC_OK) return st;
+    const bool map_a = mx->order == MQC_ORDER_BA;
+    const bool along_i = (mx->block == MQC_BLOCK_A32) == map_a && mx->block != MQC_BLOCK_SQ32;
+    const int blk = mx->block == MQC_BLOCK_SQ32 ? kSquare : (along_i ? kAlongI : kAlongO);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (map_a) launch_quantize_batch<true>(b, blk, mx->fmt, dual, static_cast<unsigned>(total), s);
+    else launch_quantize_batch<false>(b, blk, mx->fmt, dual, static_cast<unsigned>(total), s);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "mx_quantize_batch_kernel launch");
+    return MQC_OK;
+}
+
+}  // extern "C"
 
 extern "C" {
 

@@ -90,8 +90,9 @@ enum QuantBlock : int { kAlongI = 0, kAlongO = 1, kSquare = 2 };
 
 // MAP_A: the i axis is A (primary order BA); otherwise it is B (order AB).
 // BLK: direction of the blocks relative to (i, o).  IT: 32 or 16 (FP8 only).
+// The work of one CTA (256 threads) on tile `t` of the tensor p.
 template <bool MAP_A, int BLK, int FMT, int IT, bool DUAL>
-__global__ void __launch_bounds__(256, 2) mx_quantize_kernel(const QuantParams p) {
+__device__ __forceinline__ void quantize_tile(const QuantParams &p, int t) {
     constexpr int OJ = 4;                             // o-rows per thread
     constexpr bool FP4 = FMT == 2;
     constexpr int RB = FP4 ? IT / 2 : IT;             // bytes of one 32- or 16-code row
@@ -105,7 +106,6 @@ __global__ void __launch_bounds__(256, 2) mx_quantize_kernel(const QuantParams p
     const int wo = warp % wpg;
     const int gsize = 8 / wpg;                        // position groups per CTA (2 or 1)
 
-    int t = blockIdx.x;
     const int pT = t % p.nPT;
     t /= p.nPT;
     const int oT = t % p.nOT;
@@ -287,6 +287,51 @@ __global__ void __launch_bounds__(256, 2) mx_quantize_kernel(const QuantParams p
         uint4 *dst = reinterpret_cast<uint4 *>(p.codes_alt + (FP4 ? off / 2 : off));
         dst[ch] = val;
     }
+}
+
+template <bool MAP_A, int BLK, int FMT, int IT, bool DUAL>
+__global__ void __launch_bounds__(256, 2) mx_quantize_kernel(const QuantParams p) {
+    quantize_tile<MAP_A, BLK, FMT, IT, DUAL>(p, blockIdx.x);
+}
+
+// Several tensors of the same format, block mode and code order in one
+// launch (e.g. the weights of every layer, quantized together after a weight
+// update): CTA b works on tile b - tile0[i] of tensor i, tile0[i] <= b <
+// tile0[i + 1].  Small tensors (a 3x3 kernel has 9 spatial positions, so 9
+// of a warp's 32 lanes work) then run side by side instead of one after the
+// other.
+constexpr int kMaxQuantBatch = 16;
+struct QuantBatch {
+    QuantParams q[kMaxQuantBatch];
+    int32_t tile0[kMaxQuantBatch + 1];
+    int32_t n;
+};
+
+template <bool MAP_A, int BLK, int FMT, bool DUAL>
+__global__ void __launch_bounds__(256, 2) mx_quantize_batch_kernel(const __grid_constant__ QuantBatch b) {
+    int i = 0;
+    while (i + 1 < b.n && static_cast<int>(blockIdx.x) >= b.tile0[i + 1]) ++i;
+    quantize_tile<MAP_A, BLK, FMT, 32, DUAL>(b.q[i], static_cast<int>(blockIdx.x) - b.tile0[i]);
+}
+
+template <bool MAP_A, int BLK, int FMT>
+inline void launch_quantize_batch_fmt(const QuantBatch &b, bool dual, unsigned grid, cudaStream_t s) {
+    if (dual) mx_quantize_batch_kernel<MAP_A, BLK, FMT, true><<<grid, 256, 0, s>>>(b);
+    else mx_quantize_batch_kernel<MAP_A, BLK, FMT, false><<<grid, 256, 0, s>>>(b);
+}
+
+template <bool MAP_A, int BLK>
+inline void launch_quantize_batch_blk(const QuantBatch &b, int fmt, bool dual, unsigned grid, cudaStream_t s) {
+    if (fmt == 0) launch_quantize_batch_fmt<MAP_A, BLK, 0>(b, dual, grid, s);
+    else if (fmt == 1) launch_quantize_batch_fmt<MAP_A, BLK, 1>(b, dual, grid, s);
+    else launch_quantize_batch_fmt<MAP_A, BLK, 2>(b, dual, grid, s);
+}
+
+template <bool MAP_A>
+inline void launch_quantize_batch(const QuantBatch &b, int blk, int fmt, bool dual, unsigned grid, cudaStream_t s) {
+    if (blk == kAlongI) launch_quantize_batch_blk<MAP_A, kAlongI>(b, fmt, dual, grid, s);
+    else if (blk == kAlongO) launch_quantize_batch_blk<MAP_A, kAlongO>(b, fmt, dual, grid, s);
+    else launch_quantize_batch_blk<MAP_A, kSquare>(b, fmt, dual, grid, s);
 }
 
 // Host-side dispatch over the compile-time variants.

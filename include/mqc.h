@@ -129,6 +129,19 @@ MQC_API mqc_status mqc_tensor_dims(mqc_role role, const mqc_conv *conv, int32_t 
 MQC_API mqc_status mqc_quantize_mx(const float *src, const mqc_t4 *src_desc, const mqc_mx *mx,
                            void *codes, uint8_t *scales, void *codes_alt, void *stream);
 
+/* Several tensors quantized in ONE kernel launch, e.g. the weights of every
+ * layer right after a weight update (the paper quantizes the weights once
+ * per update, section V).  Element i of each array describes one tensor
+ * exactly as the arguments of mqc_quantize_mx do; all tensors share the
+ * format, block mode and code order in `mx`; codes_alt is NULL or an array
+ * whose every entry is a buffer (a second code order for all tensors).
+ * The results are those of count separate mqc_quantize_mx calls.
+ *   count   1 .. 16.
+ * Errors: as mqc_quantize_mx, for the first tensor that fails its checks. */
+MQC_API mqc_status mqc_quantize_mx_batch(int32_t count, const float *const *srcs, const mqc_t4 *src_descs,
+                                 const mqc_mx *mx, void *const *codes, uint8_t *const *scales,
+                                 void *const *codes_alt, void *stream);
+
 /* MX quantization with stochastic rounding of the elements (paper, section
  * III-A, Eq. 6 and the text after it: the gradients are rounded
  * stochastically, activations and weights to nearest).  Same arguments,

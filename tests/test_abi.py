@@ -94,6 +94,13 @@ def test_invalid_arguments_rejected_before_launch(mqc):
     # a convolution whose kernel is larger than the padded input
     assert mqc.mqc_conv2d_fwd(p, p, mx, p, p, mx, mqc.conv_desc(1, 32, 2, 2, 8, 5, 5, 1, 1), p, None, 0, None) == -1
     assert mqc.lib.mqc_debug_expire_wait(10, None) == -1
+    # batched quantization: 1 .. 16 tensors, all codes_alt or none
+    one = [ctypes.c_void_p(16)]
+    assert mqc.mqc_quantize_mx_batch([], [], mx, [], [], None, None) == -1
+    assert mqc.mqc_quantize_mx_batch(one * 17, [d] * 17, mx, one * 17, one * 17, None, None) == -1
+    assert mqc.mqc_quantize_mx_batch(one * 2, [d, d], mx, one * 2, one * 2, [16, 0], None) == -1
+    assert mqc.mqc_quantize_mx_batch(one * 2, [d, bad], mx, one * 2, one * 2, None, None) == -1
+    assert mqc.mqc_quantize_mx_batch(one * 2, [d, d], mx, [16, 17], one * 2, None, None) == -5
     # stochastic rounding: primary order BA and an NCHW-like source only
     assert mqc.mqc_quantize_mx_sr(ctypes.c_void_p(16), d, mqc.MX(0, 2, 1), ctypes.c_void_p(16), ctypes.c_void_p(16),
                                   None, 1, 0, None) == -2

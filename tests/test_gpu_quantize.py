@@ -127,3 +127,28 @@ def test_im2col_cbf_parity(mqc, orc, fmt, block, order):
         eco, eso = orc.im2col_cbf(rc, rs, N, C, H, W, R, S, st, st, pad, pad, fmt, block, order)
         assert np.array_equal(_host(co), eco), (N, C, H, W, R, S, st, pad)
         assert np.array_equal(_host(so), eso), (N, C, H, W, R, S, st, pad)
+
+
+def test_quantize_batch_equals_single_calls(mqc, orc):
+    """mqc_quantize_mx_batch: the eight weight tensors of the YOLOv8n training
+    stack (3x3 and 1x1 kernels, E4M3, SQ32, both orders) in one launch, and a
+    set of small ragged tensors in A32 / B32 and E2M1, bit-identical to the
+    oracle's quantization of each tensor."""
+    wl = synth.WORKLOADS[3]
+    ws = [synth.layer_inputs(wl, i)[1] for i in range(len(wl.layers))]
+    qs = mqc.quantize_mx_batch([_dev(w) for w in ws], 0, 2, 0, both_orders=True)
+    for w, q in zip(ws, qs):
+        rc, rs = orc.quantize(w, 0, 2, 0)
+        assert np.array_equal(_host(q.codes), rc) and np.array_equal(_host(q.scales), rs)
+        assert np.array_equal(_host(q.codes_alt), orc.quantize(w, 0, 2, 1)[0])
+    small = [synth.random_tensor(s, seed=40 + i, dist="student_t")
+             for i, s in enumerate([(37, 45, 3, 3), (16, 40, 1, 1), (70, 33, 2, 5), (5, 16, 4, 4)])]
+    for fmt, blk, order in ((2, 0, 0), (0, 1, 1), (1, 1, 0)):
+        qs = mqc.quantize_mx_batch([_dev(x) for x in small], fmt, blk, order, both_orders=(fmt == 0))
+        for x, q in zip(small, qs):
+            rc, rs = orc.quantize(x, fmt, blk, order)
+            assert np.array_equal(_host(q.codes), rc), (fmt, blk, order, x.shape)
+            assert np.array_equal(_host(q.scales), rs), (fmt, blk, order, x.shape)
+            if fmt == 0:
+                assert np.array_equal(_host(q.codes_alt), orc.quantize(x, fmt, blk, 1 - order)[0])
+    mqc.check(mqc.get_device_status())

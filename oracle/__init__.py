@@ -79,6 +79,10 @@ def lib():
         L.oracle_encode_sr.argtypes = [i32, dbl, u32]
         L.oracle_encode_sr.restype = i32
         L.oracle_quantize_sr.argtypes = [vp, i64, i64, i64, i64, vp, i32, i32, i32, u64, u64, vp, vp]
+        L.oracle_nvfp4_scales_bytes.argtypes = [i32, i32, i64, i64, i64, i64]
+        L.oracle_nvfp4_scales_bytes.restype = i64
+        L.oracle_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i64, vp, i32, i32, vp, vp, vp]
+        L.oracle_dequantize_nvfp4.argtypes = [vp, vp, ctypes.c_float, i64, i64, i64, i64, i32, i32, vp]
         _lib = L
     return _lib
 
@@ -178,6 +182,31 @@ def quantize_sr(x: np.ndarray, fmt: int, block: int, order: int, seed: int, offs
     lib().oracle_quantize_sr(_p(x), d0, d1, d2, d3, _p(strides), fmt, block, order, seed, offset, _p(codes),
                              _p(scales))
     return codes, scales
+
+
+NV_A16, NV_B16, NV_SQ16 = 0, 1, 2
+
+
+def quantize_nvfp4(x: np.ndarray, block: int, order: int):
+    """NVFP4 quantization (paper, Eq. 4-6) of a 4-D fp32 tensor: (codes,
+    E4M3 block scales, per-tensor fp32 scale T)."""
+    assert x.dtype == np.float32 and x.ndim == 4
+    d0, d1, d2, d3 = x.shape
+    strides = np.array([s // 4 for s in x.strides], dtype=np.int64)
+    codes = np.zeros(codes_bytes(E2M1, order, d0, d1, d2, d3), dtype=np.uint8)
+    scales = np.zeros(int(lib().oracle_nvfp4_scales_bytes(block, order, d0, d1, d2, d3)), dtype=np.uint8)
+    t = np.zeros(1, dtype=np.float32)
+    lib().oracle_quantize_nvfp4(_p(x), d0, d1, d2, d3, _p(strides), block, order, _p(codes), _p(scales), _p(t))
+    return codes, scales, float(t[0])
+
+
+def dequantize_nvfp4(codes, scales, tscale, shape, block, order) -> np.ndarray:
+    d0, d1, d2, d3 = shape
+    out = np.empty((d0, d1, d2, d3), dtype=np.float64)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    lib().oracle_dequantize_nvfp4(_p(codes), _p(scales), float(tscale), d0, d1, d2, d3, block, order, _p(out))
+    return out
 
 
 ACT_NONE, ACT_RELU, ACT_SILU = 0, 1, 2

@@ -33,6 +33,8 @@
  *   - Stochastic rounding of the elements (section III-A, Eq. 6: the
  *     gradients are rounded stochastically), with random bits from the
  *     Philox4x64-10 counter-based generator (Salmon et al., SC 2011).
+ *   - NVFP4 (section III-A, Eq. 4-6): per-tensor FP32 scale, E4M3 scale per
+ *     block of 16, E2M1 elements, evaluated step by step in fp32.
  *   - The per-element quantization-count and stored-bytes model behind
  *     Table I (section IV-C).
  */
@@ -396,6 +398,114 @@ void oracle_quantize_sr(const float *src, int64_t d0, int64_t d1, int64_t d2, in
                     }
             }
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4: the format of the paper's own experiments (section III-A,        */
+/* Eq. 4-6): a per-tensor FP32 scale, an E4M3 scale per block of 16,        */
+/* E2M1 elements                                                             */
+/* ------------------------------------------------------------------------ */
+/* Blocks of 16: along the A-axis (NV_A16), along the B-axis (NV_B16), or a
+ * 16x16 square over (B, A) (NV_SQ16).  The pages give the steps as real
+ * formulas; they are evaluated here in IEEE fp32, one rounding per step in
+ * the order the equations write them (the precision the CUDA kernel decides
+ * the codes in):
+ *   Eq. 4  T  = max|X| / (448 * 6)
+ *   Eq. 5  Bs = CastE4M3( max|X_i| / (T * 6) )      round to nearest even
+ *   Eq. 6  q  = Round( x / (Bs * T) )               E2M1, nearest even, saturating
+ * A block whose scale is 0 (or a tensor whose maximum is 0) gets zero codes
+ * (x * 0, so the sign of zero is kept).  Layout: the E2M1 codes as in
+ * oracle_quantize; one E4M3 scale byte per block:
+ *   NV_A16 : scales[(pix*Bp + b)*nb16(Ap) + a/16]
+ *   NV_B16 : scales[(pix*nb16(Bp) + b/16)*Ap + a]
+ *   NV_SQ16: scales[(pix*nb16(Bp) + b/16)*nb16(Ap) + a/16] */
+enum { NV_A16 = 0, NV_B16 = 1, NV_SQ16 = 2 };
+static int64_t nb16(int64_t x) { return (x + 15) / 16; }
+
+int64_t oracle_nvfp4_scales_bytes(int block, int order, int64_t d0, int64_t d1, int64_t d2, int64_t d3)
+{
+    int64_t Ap, Bp;
+    oracle_padded_extents(OR_E2M1, order, d1, d0, &Ap, &Bp);
+    int64_t pix = d2 * d3;
+    if (block == NV_A16) return pix * Bp * nb16(Ap);
+    if (block == NV_B16) return pix * nb16(Bp) * Ap;
+    return pix * nb16(Bp) * nb16(Ap);
+}
+
+static int64_t nv_scale_index(int block, int64_t pix, int64_t b, int64_t a, int64_t Ap, int64_t Bp)
+{
+    if (block == NV_A16) return (pix * Bp + b) * nb16(Ap) + a / 16;
+    if (block == NV_B16) return (pix * nb16(Bp) + b / 16) * Ap + a;
+    return (pix * nb16(Bp) + b / 16) * nb16(Ap) + a / 16;
+}
+
+void oracle_quantize_nvfp4(const float *src, int64_t d0, int64_t d1, int64_t d2, int64_t d3,
+                           const int64_t *strides, int block, int order,
+                           uint8_t *codes, uint8_t *scales, float *tscale)
+{
+    int64_t Ap, Bp;
+    oracle_padded_extents(OR_E2M1, order, d1, d0, &Ap, &Bp);
+    memset(codes, 0, (size_t)oracle_codes_bytes(OR_E2M1, order, d0, d1, d2, d3));
+    float amax = 0.0f;
+    for (int64_t b = 0; b < d0; ++b)
+        for (int64_t a = 0; a < d1; ++a)
+            for (int64_t h = 0; h < d2; ++h)
+                for (int64_t w = 0; w < d3; ++w) {
+                    float x = fabsf(src[b * strides[0] + a * strides[1] + h * strides[2] + w * strides[3]]);
+                    if (x > amax) amax = x;
+                }
+    const float T = amax / 2688.0f;                       /* Eq. 4: 448 * 6 */
+    *tscale = T;
+    const float d = T * 6.0f;
+    int64_t eb = (block == NV_A16) ? 1 : 16;
+    int64_t ea = (block == NV_B16) ? 1 : 16;
+    int64_t npix = d2 * d3;
+#pragma omp parallel for schedule(static)
+    for (int64_t pix = 0; pix < npix; ++pix) {
+        int64_t h = pix / d3, w = pix % d3;
+        for (int64_t b0 = 0; b0 < Bp; b0 += eb)
+            for (int64_t a0 = 0; a0 < Ap; a0 += ea) {
+                int64_t b1 = b0 + eb < Bp ? b0 + eb : Bp, a1 = a0 + ea < Ap ? a0 + ea : Ap;
+                float bmax = 0.0f;
+                for (int64_t b = b0; b < b1; ++b)
+                    for (int64_t a = a0; a < a1; ++a) {
+                        float x = fabsf((float)src_at(src, d0, d1, strides, b, a, h, w));
+                        if (x > bmax) bmax = x;
+                    }
+                const float q = T > 0.0f ? bmax / d : 0.0f;                     /* Eq. 5 */
+                const int sc = oracle_encode(OR_E4M3, (double)q);
+                scales[nv_scale_index(block, pix, b0, a0, Ap, Bp)] = (uint8_t)sc;
+                int fin;
+                const float Bs = (float)oracle_decode(OR_E4M3, sc, &fin);
+                const float s = Bs * T;
+                for (int64_t b = b0; b < b1; ++b)
+                    for (int64_t a = a0; a < a1; ++a) {
+                        if (b >= d0 || a >= d1) continue;
+                        const float x = (float)src_at(src, d0, d1, strides, b, a, h, w);
+                        const float v = s > 0.0f ? x / s : x * 0.0f;              /* Eq. 6 */
+                        put_code(codes, OR_E2M1, code_index(order, pix, b, a, Ap, Bp), oracle_encode(OR_E2M1, (double)v));
+                    }
+            }
+    }
+}
+
+/* Dense double tensor of an NVFP4 quantization: element value * Bs * T. */
+void oracle_dequantize_nvfp4(const uint8_t *codes, const uint8_t *scales, float tscale, int64_t d0, int64_t d1,
+                             int64_t d2, int64_t d3, int block, int order, double *out)
+{
+    int64_t Ap, Bp;
+    oracle_padded_extents(OR_E2M1, order, d1, d0, &Ap, &Bp);
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < d0; ++b)
+        for (int64_t a = 0; a < d1; ++a)
+            for (int64_t h = 0; h < d2; ++h)
+                for (int64_t w = 0; w < d3; ++w) {
+                    int64_t pix = h * d3 + w;
+                    int fin;
+                    double v = oracle_decode(OR_E2M1, get_code(codes, OR_E2M1, code_index(order, pix, b, a, Ap, Bp)), &fin);
+                    double bs = oracle_decode(OR_E4M3, scales[nv_scale_index(block, pix, b, a, Ap, Bp)], &fin);
+                    out[((b * d1 + a) * d2 + h) * d3 + w] = v * bs * (double)tscale;
+                }
 }
 
 /* Dequantize back to a dense double tensor [d0][d1][d2][d3]:

@@ -33,7 +33,9 @@ EXPORTS = ("mqc_codes_bytes", "mqc_scales_bytes", "mqc_tensor_dims", "mqc_quanti
            "mqc_conv2d_bwd_weight", "mqc_conv2d_bwd_weight_workspace_bytes", "mqc_get_device_status",
            "mqc_debug_expire_wait", "mqc_status_string", "mqc_last_error_message", "mqc_version",
            "mqc_conv2d_bwd_weight_noalloc", "mqc_conv2d_fwd_workspace_bytes", "mqc_conv2d_bwd_data_workspace_bytes",
-           "mqc_quantize_mx_sr", "mqc_conv2d_fwd_quant", "mqc_quantize_mx_batch")
+           "mqc_quantize_mx_sr", "mqc_conv2d_fwd_quant", "mqc_quantize_mx_batch", "mqc_quantize_nvfp4",
+           "mqc_nvfp4_scales_bytes", "mqc_conv2d_fwd_nvfp4")
+NV_A16, NV_B16, NV_SQ16 = 0, 1, 2
 ACT_NONE, ACT_RELU, ACT_SILU = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -72,6 +74,9 @@ def _load() -> ctypes.CDLL:
         "mqc_quantize_mx": (i32, [vp, P(T4), P(MX), vp, vp, vp, vp]),
         "mqc_quantize_mx_sr": (i32, [vp, P(T4), P(MX), vp, vp, vp, ctypes.c_uint64, ctypes.c_uint64, vp]),
         "mqc_quantize_mx_batch": (i32, [i32, P(vp), P(T4), P(MX), P(vp), P(vp), P(vp), vp]),
+        "mqc_quantize_nvfp4": (i32, [vp, P(T4), i32, i32, vp, vp, vp, vp, vp]),
+        "mqc_nvfp4_scales_bytes": (i64, [i32, i32, i32, i32, i32, i32]),
+        "mqc_conv2d_fwd_nvfp4": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, P(Conv), vp, vp]),
         "mqc_im2col_cbf": (i32, [vp, vp, P(Conv), P(MX), vp, vp, vp]),
         "mqc_im2col_cbf_scales_bytes": (i64, [P(Conv), P(MX)]),
         "mqc_im2col_cbf_codes_bytes": (i64, [P(Conv), P(MX)]),
@@ -280,6 +285,47 @@ def quantize_mx_batch(srcs, fmt: int, block: int, order: int, both_orders: bool 
                                 [q.scales.data_ptr() for q in outs],
                                 [q.codes_alt.data_ptr() for q in outs] if both_orders else None, _stream()))
     return outs
+
+
+class QuantizedNV(Quantized):
+    """NVFP4 codes + E4M3 block scales + the per-tensor fp32 scale (a 2-float
+    device buffer: [0] T, [1] scratch)."""
+
+    def __init__(self, codes, scales, dims, block, order, tscale, codes_alt=None):
+        super().__init__(codes, scales, dims, MX(E2M1, block, order), codes_alt)
+        self.nv_block, self.tscale = block, tscale
+
+    def other_order(self) -> "QuantizedNV":
+        if self.codes_alt is None:
+            raise ValueError("quantized without the second code order")
+        return QuantizedNV(self.codes_alt, self.scales, self.dims, self.nv_block, 1 - self.mx.order, self.tscale,
+                           self.codes)
+
+
+def quantize_nvfp4(src, block: int, order: int, both_orders: bool = False) -> QuantizedNV:
+    """NVFP4-quantize a 4-D fp32 CUDA tensor [d0=B][d1=A][d2][d3] (NCHW-like)."""
+    torch = _torch()
+    assert src.is_cuda and src.dtype == torch.float32 and src.dim() == 4
+    d = tuple(src.shape)
+    codes = torch.empty(mqc_codes_bytes(MX(E2M1, 0, order), *d), dtype=torch.uint8, device=src.device)
+    scales = torch.empty(lib.mqc_nvfp4_scales_bytes(block, order, *d), dtype=torch.uint8, device=src.device)
+    alt = (torch.empty(mqc_codes_bytes(MX(E2M1, 0, 1 - order), *d), dtype=torch.uint8, device=src.device)
+           if both_orders else None)
+    ts = torch.zeros(2, dtype=torch.float32, device=src.device)
+    check(lib.mqc_quantize_nvfp4(_ptr(src), ctypes.byref(T4(*d, *src.stride())), block, order, _ptr(codes),
+                                 _ptr(scales), _ptr(alt), _ptr(ts), _stream()))
+    return QuantizedNV(codes, scales, d, block, order, ts, alt)
+
+
+def conv2d_fwd_nvfp4(xq: QuantizedNV, wq: QuantizedNV, cv: Conv, out=None):
+    """Forward convolution of NVFP4 operands on the tensor core (kind::mxf4nvf4)."""
+    torch = _torch()
+    P, Q = conv_out_hw(cv)
+    y = out if out is not None else torch.empty((cv.N, cv.K, P, Q), dtype=torch.float32, device=xq.codes.device)
+    check(lib.mqc_conv2d_fwd_nvfp4(_ptr(xq.codes), _ptr(xq.scales), _ptr(xq.tscale), xq.nv_block, _ptr(wq.codes),
+                                   _ptr(wq.scales), _ptr(wq.tscale), wq.nv_block, ctypes.byref(cv), _ptr(y),
+                                   _stream()))
+    return y
 
 
 def im2col_cbf(xq: Quantized, cv: Conv):

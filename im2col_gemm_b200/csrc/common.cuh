@@ -203,6 +203,20 @@ __device__ __forceinline__ void tc_mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc,
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] . B[smem]^T for packed E2M1 operands (K = 64 per
+// instruction, 32 bytes of each operand row) with four UE4M3 scale factors
+// per row per instruction, one per 16 elements of K (kind::mxf4nvf4,
+// scale_vec::4X): byte q of the row's 32-bit scale word in tensor memory
+// scales K elements 16q .. 16q + 15.
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // 32 lanes x 16 consecutive 32-bit columns: thread i of the warp receives
 // lane (base lane + i), columns col .. col+15.
 __device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -263,6 +277,13 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
 // factor ids (B at bits 4..5, A at 29..30) are OR-ed in per K-block.
 __host__ __device__ constexpr uint32_t make_idesc_mx(uint32_t afmt, uint32_t bfmt, uint32_t M, uint32_t N) {
     return (afmt << 7) | (bfmt << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
+}
+
+// Instruction descriptor of kind::mxf4nvf4 with UE4M3 scale factors: A and
+// B E2M1 (format 1), scale format bit 23 = 0 (UE4M3), dense K = 64 (bit 31
+// = 0), N>>3 at 17..22, M>>4 at 24..28.
+__host__ __device__ constexpr uint32_t make_idesc_nvf4(uint32_t M, uint32_t N) {
+    return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 }  // namespace mqc

@@ -73,6 +73,7 @@ struct ScaleSrc {
     int32_t kb_pitch;
     int32_t rows;
     int32_t H, W;
+    int32_t nblk;          // NV: scale blocks of 16 per row (bytes past them read as 0)
 };
 
 struct ConvTap {
@@ -171,6 +172,11 @@ struct alignas(64) GemmParams {
     uint8_t *q_codes, *q_codes_alt, *q_scales;
     float *q_y;                  // optional fp32 copy of the activated output (NCHW), else null
     int32_t q_fmt, q_sq, q_act, q_emax, q_Kp, q_Np, q_nbA, q_nbB, q_lanes;
+    // CONV NV (template flag): NVFP4 operands, packed E2M1 codes (a 32-byte
+    // K-block holds 64 elements), four UE4M3 scales per row and K-block (one
+    // atom per K-block), kind::mxf4nvf4; the epilogue multiplies by the
+    // per-tensor scales nv_tx[0] * nv_tw[0]
+    const float *nv_tx, *nv_tw;
     // output
     float *out;
     int64_t out_base, os_q, os_p, os_n, os_c, os_m, split_pitch;
@@ -498,8 +504,9 @@ __device__ __forceinline__ void qout_chunk(const GemmParams &p, const uint32_t (
     }
 }
 
-template <int KIND, bool SFV4, int UMT, bool QOUT = false>
+template <int KIND, bool SFV4, int UMT, bool QOUT = false, bool NV = false>
 __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
+    constexpr int SPK = NV ? 4 : 1;           // scale atoms per group of 4 K-blocks
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -515,8 +522,8 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
     const int a_sub_stage = 128 * kb_bytes * KS;   // one sub-tile's A rows of a stage
     const int a_stage = UM * a_sub_stage;
     const int b_stage = p.BN * kb_bytes * KS;
-    const int sfa_stage = 512 * GA * UM;       // A atoms [group][sub-tile]
-    const int sfb_stage = 512 * GA * p.nb_atoms;
+    const int sfa_stage = 512 * GA * UM * SPK;       // A atoms [group][sub-tile] (NV: [K-block])
+    const int sfb_stage = 512 * GA * p.nb_atoms * SPK;
     uint8_t *sA = smem;
     uint8_t *sB = sA + S * a_stage;
     uint8_t *sSFA = sB + S * b_stage;
@@ -599,7 +606,7 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const uint64_t lim = p.timeout_ns;
-    const int sf_cols = GA * (4 * UM + 4 * p.nb_atoms);   // TMEM scale columns per stage
+    const int sf_cols = GA * SPK * (4 * UM + 4 * p.nb_atoms);   // TMEM scale columns per stage
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -743,11 +750,32 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                     break;
                 }
                 const uint32_t sf_t = tmem + kSfTmemBase + s * sf_cols;     // SFA [group][sub-tile], then SFB
-                const uint32_t sfb_t = sf_t + 4 * GA * UM;
+                const uint32_t sfb_t = sf_t + 4 * GA * UM * SPK;
                 const int nkb = KIND == kConv ? min(KS, I.tkb - KS * ki) : 4 * min(GA, I.nkit - GA * ki);
                 const int ngr = (nkb + 3) >> 2;
                 const uint32_t a_s = static_cast<uint32_t>(s * a_stage) >> 4;
                 const uint32_t b_s = static_cast<uint32_t>(s * b_stage) >> 4;
+                if constexpr (NV) {
+                    // one A and one B scale atom per K-block (one MMA of K = 64)
+                    if (leader) {
+                        for (int kb = 0; kb < nkb; ++kb) {
+                            tc_cp_32x128b_warpx4(sf_t + 4 * kb, sfa_desc0 + static_cast<uint64_t>((s * sfa_stage + kb * 512) >> 4));
+                            tc_cp_32x128b_warpx4(sfb_t + 4 * kb, sfb_desc0 + static_cast<uint64_t>((s * sfb_stage + kb * 512) >> 4));
+                        }
+                        for (int kb = 0; kb < nkb; ++kb) {
+                            const uint32_t g = static_cast<uint32_t>(kb >> 2), k4 = static_cast<uint32_t>(kb & 3);
+                            const uint32_t j = k4 >> lg_wkb;
+                            const uint32_t within = k4 & static_cast<uint32_t>(p.wkb - 1);
+                            const uint32_t bo = b_s + g * b_grp + j * b_sub + within * 2;
+                            const uint32_t ao = a_s + g * a_grp + j * a_sub + within * 2;
+                            tc_mma_nvf4(d_tmem, adesc0 + ao, bdesc0 + bo, p.idesc, sf_t + 4 * kb, sfb_t + 4 * kb,
+                                        (ki > 0 || kb > 0) ? 1u : 0u);
+                        }
+                        tc_commit(&empty[s]);
+                    }
+                    __syncwarp();
+                    continue;
+                }
                 if (leader) {
                     for (int g = 0; g < ngr; ++g) {
                         for (int i = 0; i < UM; ++i)
@@ -901,6 +929,59 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                 for (int g = 0; g < GA && ok; ++g) {
                   const KbWalker kg = k2;                 // start of the group (each sub-tile walks it)
                   for (int i = 0; i < UM; ++i) {
+                    if constexpr (KIND == kConv && NV) {
+                        // four UE4M3 scales (blocks of 16 along C) per row and
+                        // K-block: one atom per K-block; blocks past the row's
+                        // last read as 0 (their codes are TMA zero fill)
+                        uint32_t na[4][4] = {}, nb[4][4] = {};   // [K-block][row j]
+                        if (g < ngr) {
+#pragma unroll
+                            for (int kb = 0; kb < 4; ++kb) {
+                                if (4 * g + kb >= nkb) break;
+                                const ConvTap T = p.taps[k2.tap];
+                                const int cb = k2.cb;
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
+                                    if (ra_ok[j] && ra_aw[j] == T.aw && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W) {
+                                        const uint8_t *src = p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
+                                                             ra_off[j] + cb * p.sfa.kb_pitch;
+                                        uint32_t w = 0u;
+#pragma unroll
+                                        for (int q = 0; q < 4; ++q)
+                                            if (4 * cb + q < p.sfa.nblk) w |= static_cast<uint32_t>(__ldg(src + q)) << (8 * q);
+                                        na[kb][j] = w;
+                                    }
+                                }
+                                const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    if (!rb_ok[0][j]) continue;
+                                    uint32_t w = 0u;
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q)
+                                        if (4 * cb + q < p.sfb.nblk) w |= static_cast<uint32_t>(__ldg(bsrc + rb_off[0][j] + q)) << (8 * q);
+                                    nb[kb][j] = w;
+                                }
+                                k2.advance(1, p.CB);
+                            }
+                        }
+                        if (!slot) {
+                            if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            slot = true;
+                        }
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb) {
+                            *reinterpret_cast<uint4 *>(sSFA + s * sfa_stage + (g * 4 + kb) * 512 + lane * 16) =
+                                make_uint4(na[kb][0], na[kb][1], na[kb][2], na[kb][3]);
+                            *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + (g * 4 + kb) * 512 + lane * 16) =
+                                make_uint4(nb[kb][0], nb[kb][1], nb[kb][2], nb[kb][3]);
+                        }
+                        continue;
+                    }
                     if (UM > 1) {
                         set_rows(i);
                         k2 = kg;
@@ -1228,6 +1309,13 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                     const int cb = I.col0 + c0;
                     const int nv = row_ok ? min(32, p.Ncols - cb) : 0;
                     float *op = orow + static_cast<int64_t>(cb) * p.os_c;
+                    if constexpr (NV) {
+                        const float ts = __ldg(p.nv_tx) * __ldg(p.nv_tw);   // T_x * T_w (Eq. 6 applied to both operands)
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            if (jj < nv) op[jj * p.os_c] = __uint_as_float(r[jj]) * ts;
+                        continue;
+                    }
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj)
                         if (jj < nv) op[jj * p.os_c] = __uint_as_float(r[jj]);

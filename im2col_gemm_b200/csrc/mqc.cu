@@ -19,6 +19,7 @@
 #include "quantize.cuh"
 #include "widen.cuh"
 #include "subpixel.cuh"
+#include "nvfp4.cuh"
 
 using namespace mqc;
 
@@ -89,7 +90,8 @@ struct DevInfo {
     int sms = 0;
     int max_smem = 0;
     bool gemm_attr[16] = {};  // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind, [7] SFV4 weight
-                              // gradient, [8 + 1 + 3 * SFV4 + log2(um)] forward with a quantized output
+                              // gradient, [8 + 1 + 3 * SFV4 + log2(um)] forward with a quantized output,
+                              // [15] NVFP4 forward
     bool quant_attr[72] = {};    // staged quantizer, [36*sr + (fmt*3 + blk)*4 + tile]
 };
 std::mutex g_dev_mu;
@@ -232,8 +234,10 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     } else {
         P.groups = (P.total_kb + 3) / 4;
     }
+    const bool nv = KIND == kConv && P.nv_tx != nullptr;   // NVFP4 operands (kind::mxf4nvf4)
+    const int spk = nv ? 4 : 1;                              // scale atoms per group of 4 K-blocks
     const int cache = KIND == kConv ? P.NT * P.groups * P.nb_atoms * 512 : 0;
-    P.sfb_cached = KIND == kConv && cache <= 16384 && !P.sfb_vec4;
+    P.sfb_cached = KIND == kConv && cache <= 16384 && !P.sfb_vec4 && !nv;
     // the 32-bit scale path reads B four bytes at a time unless B is cached
     if (!P.sfb_cached && !P.sfb_vec4) P.sf_vec4 = 0;
     // k16: the zero block (4 KB) 1 KB past the barriers; quantized output:
@@ -251,7 +255,7 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     P.um = 1;
     if (KIND == kConv) {
         P.MTILES = P.TQ * P.TP * P.TN;
-        if (P.total_kb <= 9 && P.BN <= 32) {
+        if (P.total_kb <= 9 && P.BN <= 32 && !nv) {
             for (int um = 4; um >= 2; um /= 2) {
                 const int64_t units = ceil_div(P.MTILES, um) * int64_t(P.nph) * P.NT;
                 if (2 * um * P.BN <= 256 && units >= 2 * d.sms) {
@@ -265,9 +269,9 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     auto stages_for = [&](int kbs, int &S) {
         const int ga = kbs / 4;
         const int kb_bytes = P.k16 ? 16 : 32;
-        const int per_stage =
-            P.um * 128 * kb_bytes * kbs + P.BN * kb_bytes * kbs + 512 * ga * P.um + 512 * ga * P.nb_atoms;
-        const int sf_cols = ga * (4 * P.um + 4 * P.nb_atoms);
+        const int per_stage = P.um * 128 * kb_bytes * kbs + P.BN * kb_bytes * kbs + 512 * ga * P.um * spk +
+                              512 * ga * P.nb_atoms * spk;
+        const int sf_cols = ga * spk * (4 * P.um + 4 * P.nb_atoms);
         S = std::min(8, (d.max_smem - fixed) / per_stage);
         S = std::min(S, (kTmemCols - kSfTmemBase) / sf_cols);
         return per_stage;
@@ -306,7 +310,9 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     const int smem = fixed + S * per_stage;
     const bool v4 = KIND == kConv && P.sf_vec4;
     auto kernel = P.sq_gather ? conv_gemm_kernel<kWgrad, true, 1> : conv_gemm_kernel<kWgrad, false, 1>;
-    if (KIND == kConv && !qout) {
+    if (nv) {
+        kernel = conv_gemm_kernel<kConv, false, 1, false, true>;
+    } else if (KIND == kConv && !qout) {
         if (P.um == 4) kernel = v4 ? conv_gemm_kernel<kConv, true, 4> : conv_gemm_kernel<kConv, false, 4>;
         else if (P.um == 2) kernel = v4 ? conv_gemm_kernel<kConv, true, 2> : conv_gemm_kernel<kConv, false, 2>;
         else kernel = v4 ? conv_gemm_kernel<kConv, true, 1> : conv_gemm_kernel<kConv, false, 1>;
@@ -315,8 +321,9 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
         else if (P.um == 2) kernel = v4 ? conv_gemm_kernel<kConv, true, 2, true> : conv_gemm_kernel<kConv, false, 2, true>;
         else kernel = v4 ? conv_gemm_kernel<kConv, true, 1, true> : conv_gemm_kernel<kConv, false, 1, true>;
     }
-    const int ai = KIND == kConv ? (qout ? 8 : 0) + 1 + (v4 ? 3 : 0) + (P.um == 4 ? 2 : P.um - 1)
-                                 : (P.sq_gather ? 7 : 0);
+    const int ai = nv ? 15
+                      : KIND == kConv ? (qout ? 8 : 0) + 1 + (v4 ? 3 : 0) + (P.um == 4 ? 2 : P.um - 1)
+                                      : (P.sq_gather ? 7 : 0);
     if (!d.gemm_attr[ai]) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.max_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -597,6 +604,73 @@ static mqc_status quantize_impl(const float *src, const mqc_t4 *d, const mqc_mx 
 
 extern "C" {
 
+int64_t mqc_nvfp4_scales_bytes(int32_t block, int32_t order, int32_t d0, int32_t d1, int32_t d2, int32_t d3) {
+    if (block < 0 || block > 2 || (order != 0 && order != 1) || d0 <= 0 || d1 <= 0 || d2 <= 0 || d3 <= 0) return -1;
+    int64_t Ap, Bp;
+    padded(MQC_E2M1, order, d1, d0, Ap, Bp);
+    const int64_t pix = int64_t(d2) * d3;
+    if (block == MQC_NV_A16) return pix * Bp * ceil_div(Ap, 16);
+    if (block == MQC_NV_B16) return pix * ceil_div(Bp, 16) * Ap;
+    return pix * ceil_div(Bp, 16) * ceil_div(Ap, 16);
+}
+
+mqc_status mqc_quantize_nvfp4(const float *src, const mqc_t4 *d, int32_t block, int32_t order, void *codes,
+                              uint8_t *scales, void *codes_alt, float *tscale, void *stream) {
+    if (src == nullptr || d == nullptr || codes == nullptr || scales == nullptr || tscale == nullptr ||
+        block < 0 || block > 2 || (order != 0 && order != 1))
+        return fail(MQC_ERR_INVALID, "quantize_nvfp4: null pointer or bad block / order");
+    if (d->d0 <= 0 || d->d1 <= 0 || d->d2 <= 0 || d->d3 <= 0)
+        return fail(MQC_ERR_INVALID, "quantize_nvfp4: extents must be positive");
+    if ((reinterpret_cast<uintptr_t>(src) & 3u) != 0 || (reinterpret_cast<uintptr_t>(tscale) & 3u) != 0)
+        return fail(MQC_ERR_ALIGNMENT, "quantize_nvfp4: src / tscale not 4-byte aligned");
+    if (!aligned16(codes) || (codes_alt != nullptr && !aligned16(codes_alt)))
+        return fail(MQC_ERR_ALIGNMENT, "quantize_nvfp4: codes not 16-byte aligned");
+    if (d->s3 != 1 || d->s2 != d->d3)
+        return fail(MQC_ERR_UNSUPPORTED, "quantize_nvfp4: spatial positions must be contiguous (NCHW-like)");
+    if (int64_t(d->d2) * d->d3 > (int64_t(1) << 31) - 64)
+        return fail(MQC_ERR_INVALID, "quantize_nvfp4: too many spatial positions");
+    DevInfo *dv;
+    mqc_status st = dev_info(dv);
+    if (st != MQC_OK) return st;
+    NvParams p{};
+    p.src = src;
+    p.sb = d->s0;
+    p.sa = d->s1;
+    p.B = d->d0;
+    p.A = d->d1;
+    p.npix = d->d2 * d->d3;
+    int64_t Ap, Bp, Ap2, Bp2;
+    padded(MQC_E2M1, order, p.A, p.B, Ap, Bp);
+    padded(MQC_E2M1, 1 - order, p.A, p.B, Ap2, Bp2);
+    p.Ap = static_cast<int32_t>(Ap);
+    p.Bp = static_cast<int32_t>(Bp);
+    p.Ap_alt = static_cast<int32_t>(Ap2);
+    p.Bp_alt = static_cast<int32_t>(Bp2);
+    p.order = order;
+    p.block = block;
+    const int64_t Acov = codes_alt ? std::max(Ap, Ap2) : Ap, Bcov = codes_alt ? std::max(Bp, Bp2) : Bp;
+    p.ntb = static_cast<int32_t>(ceil_div(Bcov, 16));
+    p.nta = static_cast<int32_t>(ceil_div(Acov, 16));
+    p.codes = static_cast<uint8_t *>(codes);
+    p.codes_alt = static_cast<uint8_t *>(codes_alt);
+    p.scales = scales;
+    p.tscale = tscale;
+    const int64_t ntiles = int64_t(p.npix) * p.ntb * p.nta;
+    if (ntiles > (int64_t(1) << 40)) return fail(MQC_ERR_INVALID, "quantize_nvfp4: tensor too large");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(tscale + 1, 0, sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(max|X|)");
+    const int64_t total = int64_t(p.B) * p.A * p.npix;
+    const int ga = static_cast<int>(std::min<int64_t>(ceil_div(total, 256), int64_t(dv->sms) * 8));
+    nv_amax_kernel<<<std::max(1, ga), 256, 0, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "nv_amax_kernel launch");
+    nv_quantize_kernel<<<static_cast<unsigned>(ceil_div(ntiles, 128)), 128, 0, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "nv_quantize_kernel launch");
+    return MQC_OK;
+}
+
 mqc_status mqc_quantize_mx_batch(int32_t count, const float *const *srcs, const mqc_t4 *descs, const mqc_mx *mx,
                                  void *const *codes, uint8_t *const *scales, void *const *codes_alt, void *stream) {
     if (count < 1 || count > kMaxQuantBatch || srcs == nullptr || descs == nullptr || codes == nullptr ||
@@ -735,9 +809,15 @@ struct QoutArgs {
     float *y;      // optional fp32 copy of the activated output
 };
 
+// NVFP4 operands of the forward: per-tensor scales and block modes.
+struct NvArgs {
+    const float *x_tscale, *w_tscale;
+    int x_block, w_block;
+};
+
 static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx *xf, const void *wq,
                                 const uint8_t *ws, const mqc_mx *wf, const mqc_conv *c, float *y, void *workspace,
-                                size_t workspace_bytes, void *stream, const QoutArgs *qo);
+                                size_t workspace_bytes, void *stream, const QoutArgs *qo, const NvArgs *nva = nullptr);
 
 extern "C" {
 
@@ -765,11 +845,25 @@ mqc_status mqc_conv2d_fwd_quant(const void *xq, const uint8_t *xs, const mqc_mx 
     return conv_fwd_impl(xq, xs, xf, wq, ws, wf, c, y, workspace, workspace_bytes, stream, &qo);
 }
 
+mqc_status mqc_conv2d_fwd_nvfp4(const void *xq, const uint8_t *xs, const float *x_tscale, int32_t x_block,
+                                const void *wq, const uint8_t *ws, const float *w_tscale, int32_t w_block,
+                                const mqc_conv *c, float *y, void *stream) {
+    if (!conv_ok(c) || y == nullptr || xq == nullptr || xs == nullptr || wq == nullptr || ws == nullptr ||
+        x_tscale == nullptr || w_tscale == nullptr)
+        return fail(MQC_ERR_INVALID, "conv2d_fwd_nvfp4: bad conv descriptor or null pointer");
+    if ((x_block != MQC_NV_A16 && x_block != MQC_NV_SQ16) || (w_block != MQC_NV_A16 && w_block != MQC_NV_SQ16))
+        return fail(MQC_ERR_UNSUPPORTED, "conv2d_fwd_nvfp4: operands need blocks along C (A16 or SQ16), order BA");
+    if (!aligned16(xq) || !aligned16(wq)) return fail(MQC_ERR_ALIGNMENT, "conv2d_fwd_nvfp4: codes not 16-byte aligned");
+    const NvArgs nva{x_tscale, w_tscale, x_block, w_block};
+    const mqc_mx fx{MQC_E2M1, MQC_BLOCK_A32, MQC_ORDER_BA};   // the code layout of E2M1 (the blocks are nva's)
+    return conv_fwd_impl(xq, xs, &fx, wq, ws, &fx, c, y, nullptr, 0, stream, nullptr, &nva);
+}
+
 }  // extern "C"
 
 static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx *xf, const void *wq,
                                 const uint8_t *ws, const mqc_mx *wf, const mqc_conv *c, float *y, void *workspace,
-                                size_t workspace_bytes, void *stream, const QoutArgs *qo) {
+                                size_t workspace_bytes, void *stream, const QoutArgs *qo, const NvArgs *nva) {
     mqc_status st = check_gemm_operand("X", xq, xs, xf, MQC_ORDER_BA, true);
     if (st != MQC_OK) return st;
     st = check_gemm_operand("W", wq, ws, wf, MQC_ORDER_BA, true);
@@ -782,14 +876,23 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
 
     const int N = c->N, C = c->C, H = c->H, W = c->W, K = c->K, R = c->R, S = c->S;
     const int sh = c->stride_h, sw = c->stride_w, P = conv_P(c), Q = conv_Q(c);
-    if ((st = check_workspace("conv2d_fwd", workspace, workspace_bytes, mqc_conv2d_fwd_workspace_bytes(c, xf, wf))) !=
-        MQC_OK)
-        return st;
-    uint8_t *wsp = static_cast<uint8_t *>(workspace);
     GemmOperand ox, ow;
-    if ((st = gemm_operand(xq, xf, N, C, H, W, wsp, static_cast<cudaStream_t>(stream), ox)) != MQC_OK) return st;
-    if ((st = gemm_operand(wq, wf, K, C, R, S, wsp, static_cast<cudaStream_t>(stream), ow)) != MQC_OK) return st;
-    const int64_t Cp = ox.inner, Cpw = ow.inner;   // padded channel extents of X and W rows
+    if (nva == nullptr) {
+        if ((st = check_workspace("conv2d_fwd", workspace, workspace_bytes,
+                                  mqc_conv2d_fwd_workspace_bytes(c, xf, wf))) != MQC_OK)
+            return st;
+        uint8_t *wsp = static_cast<uint8_t *>(workspace);
+        if ((st = gemm_operand(xq, xf, N, C, H, W, wsp, static_cast<cudaStream_t>(stream), ox)) != MQC_OK) return st;
+        if ((st = gemm_operand(wq, wf, K, C, R, S, wsp, static_cast<cudaStream_t>(stream), ow)) != MQC_OK) return st;
+    } else {
+        // NVFP4: the packed codes themselves; a row of C padded to 32 codes is
+        // round32(C) / 2 bytes, and the K-blocks below are 32 bytes (64 codes)
+        ox.codes = static_cast<const uint8_t *>(xq);
+        ow.codes = static_cast<const uint8_t *>(wq);
+        ox.mma_fmt = ow.mma_fmt = MQC_E2M1;
+        ox.inner = ow.inner = round_up(C, 32) / 2;
+    }
+    const int64_t Cp = ox.inner, Cpw = ow.inner;   // padded channel extents of X and W rows (bytes)
     GemmParams G;
     memset(&G, 0, sizeof G);
     G.CB = static_cast<int32_t>(nb32(Cp));
@@ -823,7 +926,7 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
     G.Ncols = K;
     G.a_st_h = sh;
     G.a_st_w = sw;
-    G.idesc = make_idesc_mx(mma_fmt(ox.mma_fmt), mma_fmt(ow.mma_fmt), 128, G.BN);
+    G.idesc = nva ? make_idesc_nvf4(128, G.BN) : make_idesc_mx(mma_fmt(ox.mma_fmt), mma_fmt(ow.mma_fmt), 128, G.BN);
     // A: one map per stride phase; dims (C, W', H', N) so that rows run along q
     bool phase_ok[16] = {};
     for (int attempt = qo ? 1 : 0; attempt < 2; ++attempt) {
@@ -909,6 +1012,25 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
                 (reinterpret_cast<uintptr_t>(xs) & 3u) == 0;
     G.sfb_vec4 = G.CB % 4 == 0 && G.sfb.tap_pitch % 4 == 0 && G.sfb.row_pitch % 4 == 0 &&
                  (reinterpret_cast<uintptr_t>(ws) & 3u) == 0;
+    if (nva != nullptr) {
+        // E4M3 scales per 16 channels: A16 [pix][n][nb16], SQ16 [pix][n/16][nb16]
+        // (W: [tap][k or k/16][nb16]); a 32-byte K-block has 4 of them
+        const int64_t nb = round_up(C, 32) / 16;
+        const bool sqx16 = nva->x_block == MQC_NV_SQ16, sqw16 = nva->w_block == MQC_NV_SQ16;
+        G.sfa.pix_pitch = (sqx16 ? ceil_div(N, 16) : N) * nb;
+        G.sfa.row_shift = sqx16 ? 4 : 0;
+        G.sfa.row_pitch = static_cast<int32_t>(nb);
+        G.sfa.kb_pitch = 4;
+        G.sfa.nblk = static_cast<int32_t>(nb);
+        G.sfb.tap_pitch = (sqw16 ? ceil_div(K, 16) : K) * nb;
+        G.sfb.row_shift = sqw16 ? 4 : 0;
+        G.sfb.row_pitch = static_cast<int32_t>(nb);
+        G.sfb.kb_pitch = 4;
+        G.sfb.nblk = static_cast<int32_t>(nb);
+        G.sf_vec4 = G.sfb_vec4 = 0;
+        G.nv_tx = nva->x_tscale;
+        G.nv_tw = nva->w_tscale;
+    }
     G.out = y;
     G.os_q = 1;
     G.os_p = Q;

@@ -167,6 +167,36 @@ MQC_API mqc_status mqc_quantize_mx_sr(const float *src, const mqc_t4 *src_desc, 
                               void *codes, uint8_t *scales, void *codes_alt, uint64_t seed,
                               uint64_t offset, void *stream);
 
+/* NVFP4 block modes: blocks of 16 along the A-axis, along the B-axis, or a
+ * 16 x 16 square over (B, A). */
+typedef enum { MQC_NV_A16 = 0, MQC_NV_B16 = 1, MQC_NV_SQ16 = 2 } mqc_nv_block;
+
+/* NVFP4 quantization, the format of the paper's own experiments (section
+ * III-A, Eq. 4-6):
+ *   Eq. 4  T  = max|X| / (448 * 6)                      per tensor, fp32
+ *   Eq. 5  Bs = CastE4M3( max|X_i| / (T * 6) )          per block of 16, round to nearest even
+ *   Eq. 6  q  = Round( x / (Bs * T) )                   E2M1, nearest even, saturating
+ * each step one IEEE fp32 operation in that order; a block (or tensor) whose
+ * scale is 0 gets zero codes.  Two launches: max|X| over the tensor, then
+ * the blocks.
+ *   block   an mqc_nv_block value; order BA or AB (as mqc_mx.order).
+ *   codes   E2M1 codes in the layout of mqc_codes_bytes with fmt MQC_E2M1.
+ *   scales  one E4M3 byte per block, mqc_nvfp4_scales_bytes() bytes:
+ *             A16 : scales[(pix*Bp + b)*nb16(Ap) + a/16]
+ *             B16 : scales[(pix*nb16(Bp) + b/16)*Ap + a]
+ *             SQ16: scales[(pix*nb16(Bp) + b/16)*nb16(Ap) + a/16]
+ *           (Ap, Bp the padded extents of `order`, nb16(x) = ceil(x/16)).
+ *   codes_alt  optional second code order (shares the scales).
+ *   tscale  device buffer of 2 floats: tscale[0] receives T; tscale[1] is
+ *           scratch (the tensor maximum).
+ * The source's spatial positions must be contiguous (element stride 1 along
+ * d3, d3 along d2), else MQC_ERR_UNSUPPORTED.
+ * Errors: MQC_ERR_INVALID, MQC_ERR_ALIGNMENT, MQC_ERR_UNSUPPORTED, MQC_ERR_CUDA. */
+MQC_API mqc_status mqc_quantize_nvfp4(const float *src, const mqc_t4 *src_desc, int32_t block, int32_t order,
+                              void *codes, uint8_t *scales, void *codes_alt, float *tscale, void *stream);
+MQC_API int64_t mqc_nvfp4_scales_bytes(int32_t block, int32_t order, int32_t d0, int32_t d1, int32_t d2,
+                               int32_t d3);
+
 /* Channel-batch-first im2col on quantized X (paper, section IV-A): the
  * explicit expansion X'_{Cin,N} of shape (Kh Kw Cin) x (Hout Wout N).  The
  * output is the quantized layout above for a tensor with spatial P x Q,
@@ -238,6 +268,22 @@ MQC_API mqc_status mqc_conv2d_fwd_quant(const void *xq, const uint8_t *xs, const
                                 const mqc_conv *conv, int32_t act, const mqc_mx *yf, void *yq,
                                 uint8_t *ys, void *yq_alt, float *y, void *workspace,
                                 size_t workspace_bytes, void *stream);
+
+/* Forward convolution (Eq. 1) with NVFP4 operands (the format of the paper's
+ * experiments, section III-A, Eq. 4-7): the packed E2M1 codes go to the
+ * tensor core as they are (tcgen05.mma kind::mxf4nvf4, K = 64 per
+ * instruction, one UE4M3 scale per 16 elements of K, scale_vec::4X), and the
+ * fp32 accumulators are multiplied by the two per-tensor scales T_x * T_w
+ * (read on the device).
+ *   xq, xs, x_tscale, x_block  X from mqc_quantize_nvfp4: order BA, block
+ *           MQC_NV_A16 or MQC_NV_SQ16 (blocks along C), tscale[0] = T_x.
+ *   wq, ws, w_tscale, w_block  W likewise (order BA, blocks along C).
+ *   y       fp32 output [N][K][P][Q] (overwritten).
+ * No workspace.  Limits as mqc_conv2d_fwd.
+ * Errors: MQC_ERR_INVALID, MQC_ERR_UNSUPPORTED, MQC_ERR_ALIGNMENT, MQC_ERR_CUDA. */
+MQC_API mqc_status mqc_conv2d_fwd_nvfp4(const void *xq, const uint8_t *xs, const float *x_tscale, int32_t x_block,
+                                const void *wq, const uint8_t *ws, const float *w_tscale, int32_t w_block,
+                                const mqc_conv *conv, float *y, void *stream);
 
 /* Input gradient, Eq. 2: G_X = W^T * G_Y as the GEMM
  * G_X'{Cin,N} = W_f^T . G_Yf{Cout,N} of section IV-B, computed directly as a

@@ -139,3 +139,12 @@ def test_gemm_workspace_sizes_cover_widened_fp4_operands(mqc):
     assert mqc.mqc_conv2d_bwd_data_workspace_bytes(sub, fp8_b, fp8_a) == 4 * 128 * 48 + (4 * 2 * 128 + 255) // 256 * 256
     assert mqc.mqc_conv2d_bwd_data_workspace_bytes(cv, fp4_b, fp4_a) == (r(mqc.mqc_codes_bytes(fp4_b, 24, 40, 3, 3))
                                                                           + r(mqc.mqc_codes_bytes(fp4_a, 4, 24, P, Q)))
+
+
+@pytest.mark.parametrize("block", [0, 1, 2])
+@pytest.mark.parametrize("order", [0, 1])
+def test_nvfp4_scale_sizes_match_oracle(mqc, orc, block, order):
+    for dims in [(2, 32, 8, 8), (37, 45, 3, 2), (1, 1, 1, 1), (128, 128, 80, 80)]:
+        assert mqc.lib.mqc_nvfp4_scales_bytes(block, order, *dims) == \
+            int(orc.lib().oracle_nvfp4_scales_bytes(block, order, *dims))
+    assert mqc.lib.mqc_nvfp4_scales_bytes(3, order, 2, 32, 8, 8) == -1

@@ -217,6 +217,19 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
         : "memory");
 }
 
+// As above for OCP MXFP4 (kind::mxf4, scale_vec::2X): two E8M0 scale
+// factors per row per instruction, one per 32 elements of K, bytes sf_id and
+// sf_id + 1 (sf_id 0 or 2, in bits 30..31 of the scale addresses) of the
+// row's 32-bit scale word.
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // 32 lanes x 16 consecutive 32-bit columns: thread i of the warp receives
 // lane (base lane + i), columns col .. col+15.
 __device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -284,6 +297,11 @@ __host__ __device__ constexpr uint32_t make_idesc_mx(uint32_t afmt, uint32_t bfm
 // = 0), N>>3 at 17..22, M>>4 at 24..28.
 __host__ __device__ constexpr uint32_t make_idesc_nvf4(uint32_t M, uint32_t N) {
     return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// kind::mxf4: A and B E2M1 (format 1), E8M0 scale factors (bit 23 = 1), K = 64.
+__host__ __device__ constexpr uint32_t make_idesc_mxf4(uint32_t M, uint32_t N) {
+    return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
 }
 
 }  // namespace mqc

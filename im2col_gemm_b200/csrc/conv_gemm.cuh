@@ -73,7 +73,7 @@ struct ScaleSrc {
     int32_t kb_pitch;
     int32_t rows;
     int32_t H, W;
-    int32_t nblk;          // NV: scale blocks of 16 per row (bytes past them read as 0)
+    int32_t nblk;          // packed FP4: scale blocks per row (bytes past them read as 0)
 };
 
 struct ConvTap {
@@ -172,11 +172,15 @@ struct alignas(64) GemmParams {
     uint8_t *q_codes, *q_codes_alt, *q_scales;
     float *q_y;                  // optional fp32 copy of the activated output (NCHW), else null
     int32_t q_fmt, q_sq, q_act, q_emax, q_Kp, q_Np, q_nbA, q_nbB, q_lanes;
-    // CONV NV (template flag): NVFP4 operands, packed E2M1 codes (a 32-byte
-    // K-block holds 64 elements), four UE4M3 scales per row and K-block (one
-    // atom per K-block), kind::mxf4nvf4; the epilogue multiplies by the
-    // per-tensor scales nv_tx[0] * nv_tw[0]
+    // CONV PK (template parameter, packed FP4 operands: the E2M1 codes as
+    // stored, a 32-byte K-block holds 64 elements):
+    //   PK = 1  OCP MXFP4, two E8M0 scales per row and K-block (blocks of 32
+    //           along C), two K-blocks per scale atom, kind::mxf4 scale_vec::2X
+    //   PK = 2  NVFP4, four UE4M3 scales per row and K-block (blocks of 16),
+    //           one atom per K-block, kind::mxf4nvf4 scale_vec::4X; the
+    //           epilogue multiplies by the per-tensor scales nv_tx[0] * nv_tw[0]
     const float *nv_tx, *nv_tw;
+    int32_t pk;
     // output
     float *out;
     int64_t out_base, os_q, os_p, os_n, os_c, os_m, split_pitch;
@@ -504,9 +508,9 @@ __device__ __forceinline__ void qout_chunk(const GemmParams &p, const uint32_t (
     }
 }
 
-template <int KIND, bool SFV4, int UMT, bool QOUT = false, bool NV = false>
+template <int KIND, bool SFV4, int UMT, bool QOUT = false, int PK = 0>
 __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
-    constexpr int SPK = NV ? 4 : 1;           // scale atoms per group of 4 K-blocks
+    constexpr int SPK = PK == 2 ? 4 : (PK == 1 ? 2 : 1);   // scale bytes per row and K-block = atoms per group
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -755,12 +759,14 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                 const int ngr = (nkb + 3) >> 2;
                 const uint32_t a_s = static_cast<uint32_t>(s * a_stage) >> 4;
                 const uint32_t b_s = static_cast<uint32_t>(s * b_stage) >> 4;
-                if constexpr (NV) {
-                    // one A and one B scale atom per K-block (one MMA of K = 64)
+                if constexpr (PK != 0) {
+                    // K-block kb (one MMA of K = 64) takes its SPK scale bytes
+                    // per row from atom kb*SPK/4 at byte (kb*SPK) % 4
                     if (leader) {
-                        for (int kb = 0; kb < nkb; ++kb) {
-                            tc_cp_32x128b_warpx4(sf_t + 4 * kb, sfa_desc0 + static_cast<uint64_t>((s * sfa_stage + kb * 512) >> 4));
-                            tc_cp_32x128b_warpx4(sfb_t + 4 * kb, sfb_desc0 + static_cast<uint64_t>((s * sfb_stage + kb * 512) >> 4));
+                        const int natoms = (nkb * SPK + 3) >> 2;
+                        for (int a = 0; a < natoms; ++a) {
+                            tc_cp_32x128b_warpx4(sf_t + 4 * a, sfa_desc0 + static_cast<uint64_t>((s * sfa_stage + a * 512) >> 4));
+                            tc_cp_32x128b_warpx4(sfb_t + 4 * a, sfb_desc0 + static_cast<uint64_t>((s * sfb_stage + a * 512) >> 4));
                         }
                         for (int kb = 0; kb < nkb; ++kb) {
                             const uint32_t g = static_cast<uint32_t>(kb >> 2), k4 = static_cast<uint32_t>(kb & 3);
@@ -768,8 +774,14 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                             const uint32_t within = k4 & static_cast<uint32_t>(p.wkb - 1);
                             const uint32_t bo = b_s + g * b_grp + j * b_sub + within * 2;
                             const uint32_t ao = a_s + g * a_grp + j * a_sub + within * 2;
-                            tc_mma_nvf4(d_tmem, adesc0 + ao, bdesc0 + bo, p.idesc, sf_t + 4 * kb, sfb_t + 4 * kb,
-                                        (ki > 0 || kb > 0) ? 1u : 0u);
+                            const uint32_t at = static_cast<uint32_t>(kb * SPK) >> 2, sid = static_cast<uint32_t>(kb * SPK) & 3u;
+                            if (PK == 2)
+                                tc_mma_nvf4(d_tmem, adesc0 + ao, bdesc0 + bo, p.idesc, sf_t + 4 * at, sfb_t + 4 * at,
+                                            (ki > 0 || kb > 0) ? 1u : 0u);
+                            else
+                                tc_mma_mxf4(d_tmem, adesc0 + ao, bdesc0 + bo, p.idesc | (sid << 29) | (sid << 4),
+                                            (sf_t + 4 * at) | (sid << 30), (sfb_t + 4 * at) | (sid << 30),
+                                            (ki > 0 || kb > 0) ? 1u : 0u);
                         }
                         tc_commit(&empty[s]);
                     }
@@ -929,11 +941,12 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                 for (int g = 0; g < GA && ok; ++g) {
                   const KbWalker kg = k2;                 // start of the group (each sub-tile walks it)
                   for (int i = 0; i < UM; ++i) {
-                    if constexpr (KIND == kConv && NV) {
-                        // four UE4M3 scales (blocks of 16 along C) per row and
-                        // K-block: one atom per K-block; blocks past the row's
-                        // last read as 0 (their codes are TMA zero fill)
-                        uint32_t na[4][4] = {}, nb[4][4] = {};   // [K-block][row j]
+                    if constexpr (KIND == kConv && PK != 0) {
+                        // SPK scales per row and K-block (2 E8M0 for MXFP4, 4
+                        // UE4M3 for NVFP4): K-block kb fills bytes (kb*SPK) % 4
+                        // .. of atom kb*SPK/4; blocks past the row's last read
+                        // as 0 (their codes are TMA zero fill)
+                        uint32_t na[4][4] = {}, nb[4][4] = {};   // [atom][row j]
                         if (g < ngr) {
 #pragma unroll
                             for (int kb = 0; kb < 4; ++kb) {
@@ -948,9 +961,9 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                                                              ra_off[j] + cb * p.sfa.kb_pitch;
                                         uint32_t w = 0u;
 #pragma unroll
-                                        for (int q = 0; q < 4; ++q)
-                                            if (4 * cb + q < p.sfa.nblk) w |= static_cast<uint32_t>(__ldg(src + q)) << (8 * q);
-                                        na[kb][j] = w;
+                                        for (int q = 0; q < SPK; ++q)
+                                            if (SPK * cb + q < p.sfa.nblk) w |= static_cast<uint32_t>(__ldg(src + q)) << (8 * q);
+                                        na[(kb * SPK) >> 2][j] |= w << (8 * ((kb * SPK) & 3));
                                     }
                                 }
                                 const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
@@ -959,9 +972,9 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                                     if (!rb_ok[0][j]) continue;
                                     uint32_t w = 0u;
 #pragma unroll
-                                    for (int q = 0; q < 4; ++q)
-                                        if (4 * cb + q < p.sfb.nblk) w |= static_cast<uint32_t>(__ldg(bsrc + rb_off[0][j] + q)) << (8 * q);
-                                    nb[kb][j] = w;
+                                    for (int q = 0; q < SPK; ++q)
+                                        if (SPK * cb + q < p.sfb.nblk) w |= static_cast<uint32_t>(__ldg(bsrc + rb_off[0][j] + q)) << (8 * q);
+                                    nb[(kb * SPK) >> 2][j] |= w << (8 * ((kb * SPK) & 3));
                                 }
                                 k2.advance(1, p.CB);
                             }
@@ -974,11 +987,11 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                             slot = true;
                         }
 #pragma unroll
-                        for (int kb = 0; kb < 4; ++kb) {
-                            *reinterpret_cast<uint4 *>(sSFA + s * sfa_stage + (g * 4 + kb) * 512 + lane * 16) =
-                                make_uint4(na[kb][0], na[kb][1], na[kb][2], na[kb][3]);
-                            *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + (g * 4 + kb) * 512 + lane * 16) =
-                                make_uint4(nb[kb][0], nb[kb][1], nb[kb][2], nb[kb][3]);
+                        for (int a = 0; a < SPK; ++a) {
+                            *reinterpret_cast<uint4 *>(sSFA + s * sfa_stage + (g * SPK + a) * 512 + lane * 16) =
+                                make_uint4(na[a][0], na[a][1], na[a][2], na[a][3]);
+                            *reinterpret_cast<uint4 *>(sSFB + s * sfb_stage + (g * SPK + a) * 512 + lane * 16) =
+                                make_uint4(nb[a][0], nb[a][1], nb[a][2], nb[a][3]);
                         }
                         continue;
                     }
@@ -1309,7 +1322,7 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                     const int cb = I.col0 + c0;
                     const int nv = row_ok ? min(32, p.Ncols - cb) : 0;
                     float *op = orow + static_cast<int64_t>(cb) * p.os_c;
-                    if constexpr (NV) {
+                    if constexpr (PK == 2) {
                         const float ts = __ldg(p.nv_tx) * __ldg(p.nv_tw);   // T_x * T_w (Eq. 6 applied to both operands)
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)

@@ -91,7 +91,7 @@ struct DevInfo {
     int max_smem = 0;
     bool gemm_attr[16] = {};  // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind, [7] SFV4 weight
                               // gradient, [8 + 1 + 3 * SFV4 + log2(um)] forward with a quantized output,
-                              // [15] NVFP4 forward
+                              // [8] MXFP4 and [15] NVFP4 forward on packed codes
     bool quant_attr[72] = {};    // staged quantizer, [36*sr + (fmt*3 + blk)*4 + tile]
 };
 std::mutex g_dev_mu;
@@ -234,8 +234,9 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     } else {
         P.groups = (P.total_kb + 3) / 4;
     }
-    const bool nv = KIND == kConv && P.nv_tx != nullptr;   // NVFP4 operands (kind::mxf4nvf4)
-    const int spk = nv ? 4 : 1;                              // scale atoms per group of 4 K-blocks
+    const int pk = KIND == kConv ? P.pk : 0;                 // packed FP4 operands: 1 MXFP4, 2 NVFP4
+    const bool nv = pk != 0;
+    const int spk = pk == 2 ? 4 : (pk == 1 ? 2 : 1);         // scale atoms per group of 4 K-blocks
     const int cache = KIND == kConv ? P.NT * P.groups * P.nb_atoms * 512 : 0;
     P.sfb_cached = KIND == kConv && cache <= 16384 && !P.sfb_vec4 && !nv;
     // the 32-bit scale path reads B four bytes at a time unless B is cached
@@ -310,8 +311,10 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     const int smem = fixed + S * per_stage;
     const bool v4 = KIND == kConv && P.sf_vec4;
     auto kernel = P.sq_gather ? conv_gemm_kernel<kWgrad, true, 1> : conv_gemm_kernel<kWgrad, false, 1>;
-    if (nv) {
-        kernel = conv_gemm_kernel<kConv, false, 1, false, true>;
+    if (pk == 2) {
+        kernel = conv_gemm_kernel<kConv, false, 1, false, 2>;
+    } else if (pk == 1) {
+        kernel = conv_gemm_kernel<kConv, false, 1, false, 1>;
     } else if (KIND == kConv && !qout) {
         if (P.um == 4) kernel = v4 ? conv_gemm_kernel<kConv, true, 4> : conv_gemm_kernel<kConv, false, 4>;
         else if (P.um == 2) kernel = v4 ? conv_gemm_kernel<kConv, true, 2> : conv_gemm_kernel<kConv, false, 2>;
@@ -321,7 +324,7 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
         else if (P.um == 2) kernel = v4 ? conv_gemm_kernel<kConv, true, 2, true> : conv_gemm_kernel<kConv, false, 2, true>;
         else kernel = v4 ? conv_gemm_kernel<kConv, true, 1, true> : conv_gemm_kernel<kConv, false, 1, true>;
     }
-    const int ai = nv ? 15
+    const int ai = pk == 2 ? 15 : pk == 1 ? 8
                       : KIND == kConv ? (qout ? 8 : 0) + 1 + (v4 ? 3 : 0) + (P.um == 4 ? 2 : P.um - 1)
                                       : (P.sq_gather ? 7 : 0);
     if (!d.gemm_attr[ai]) {
@@ -877,7 +880,10 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
     const int N = c->N, C = c->C, H = c->H, W = c->W, K = c->K, R = c->R, S = c->S;
     const int sh = c->stride_h, sw = c->stride_w, P = conv_P(c), Q = conv_Q(c);
     GemmOperand ox, ow;
-    if (nva == nullptr) {
+    // both operands OCP MXFP4 (plain forward): the packed codes go to the
+    // tensor core as they are (kind::mxf4), no widening
+    const bool mxf4 = nva == nullptr && qo == nullptr && xf->fmt == MQC_E2M1 && wf->fmt == MQC_E2M1;
+    if (nva == nullptr && !mxf4) {
         if ((st = check_workspace("conv2d_fwd", workspace, workspace_bytes,
                                   mqc_conv2d_fwd_workspace_bytes(c, xf, wf))) != MQC_OK)
             return st;
@@ -926,7 +932,9 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
     G.Ncols = K;
     G.a_st_h = sh;
     G.a_st_w = sw;
-    G.idesc = nva ? make_idesc_nvf4(128, G.BN) : make_idesc_mx(mma_fmt(ox.mma_fmt), mma_fmt(ow.mma_fmt), 128, G.BN);
+    G.idesc = nva    ? make_idesc_nvf4(128, G.BN)
+              : mxf4 ? make_idesc_mxf4(128, G.BN)
+                     : make_idesc_mx(mma_fmt(ox.mma_fmt), mma_fmt(ow.mma_fmt), 128, G.BN);
     // A: one map per stride phase; dims (C, W', H', N) so that rows run along q
     bool phase_ok[16] = {};
     for (int attempt = qo ? 1 : 0; attempt < 2; ++attempt) {
@@ -1030,6 +1038,21 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
         G.sf_vec4 = G.sfb_vec4 = 0;
         G.nv_tx = nva->x_tscale;
         G.nv_tw = nva->w_tscale;
+        G.pk = 2;
+    } else if (mxf4) {
+        // E8M0 scales per 32 channels (the MX layout above); a 32-byte K-block
+        // (64 codes) has 2 of them
+        const int64_t nb = round_up(C, 32) / 32;     // (Cp above counts bytes here)
+        G.sfa.pix_pitch = (sqx ? nb32(N) : N) * nb;
+        G.sfa.row_pitch = static_cast<int32_t>(nb);
+        G.sfa.kb_pitch = 2;
+        G.sfa.nblk = static_cast<int32_t>(nb);
+        G.sfb.tap_pitch = (sqw ? nb32(K) : K) * nb;
+        G.sfb.row_pitch = static_cast<int32_t>(nb);
+        G.sfb.kb_pitch = 2;
+        G.sfb.nblk = static_cast<int32_t>(nb);
+        G.sf_vec4 = G.sfb_vec4 = 0;
+        G.pk = 1;
     }
     G.out = y;
     G.os_q = 1;

@@ -659,6 +659,28 @@ def tensor_bound_layers(mqc, torch, pk):
                         "frac_of_mxfp4_peak": round(tf / (2 * fp8_peak), 4) if all_fp4 else None})
         del lb, ws
         torch.cuda.empty_cache()
+    # NVFP4 (the paper's own format) forward on the large-batch layer: X and W
+    # quantized with 16 x 16 squares, tcgen05 kind::mxf4nvf4 on packed codes
+    wl = synth.WORKLOADS[(5, "fp4", 128)]
+    L = wl.layers[0]
+    x, w, _ = synth.layer_inputs(wl, 0)
+    xq = mqc.quantize_nvfp4(torch.from_numpy(x).cuda(), mqc.NV_SQ16, 0)
+    wq = mqc.quantize_nvfp4(torch.from_numpy(w).cuda(), mqc.NV_SQ16, 0)
+    cv = mqc.conv_desc(L.N, L.C, L.H, L.W, L.K, L.R, L.S, L.stride, L.pad)
+    y = torch.empty((L.N, L.K, L.P, L.Q), dtype=torch.float32, device="cuda")
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    fwd = lambda: mqc.check(mqc.lib.mqc_conv2d_fwd_nvfp4(
+        ptr(xq.codes), ptr(xq.scales), ptr(xq.tscale), mqc.NV_SQ16, ptr(wq.codes), ptr(wq.scales), ptr(wq.tscale),
+        mqc.NV_SQ16, ctypes.byref(cv), ptr(y), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
+    fwd()
+    ms = statistics.median(graph_fn_times(mqc, torch, fwd, 5, k=4))
+    tf = L.gemm_flops() / (ms * 1e-3) / 1e12
+    out.append({"workload": "large-batch-nvfp4-n128-c128-80x80",
+                "what": "large-batch N=128 C=K=128 80x80, X and W NVFP4 (E2M1, E4M3 scales per 16x16, fp32 tensor scale)",
+                "call": "fwd", "ms": round(ms, 5), "tflops": round(tf, 1), "frac_of_mxfp8_peak": round(tf / fp8_peak, 4),
+                "frac_of_mxfp4_peak": round(tf / (2 * fp8_peak), 4)})
+    del xq, wq, y
+    torch.cuda.empty_cache()
     return out
 
 

@@ -73,7 +73,8 @@ struct ScaleSrc {
     int32_t kb_pitch;
     int32_t rows;
     int32_t H, W;
-    int32_t nblk;          // packed FP4: scale blocks per row (bytes past them read as 0)
+    int32_t nblk;          // packed FP4: scale blocks along K per row (bytes past them read as 0);
+                           // kb_pitch is then the distance between consecutive blocks
 };
 
 struct ConvTap {
@@ -947,7 +948,40 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                         // .. of atom kb*SPK/4; blocks past the row's last read
                         // as 0 (their codes are TMA zero fill)
                         uint32_t na[4][4] = {}, nb[4][4] = {};   // [atom][row j]
-                        if (g < ngr) {
+                        if (g < ngr && p.sf_vec4) {
+                            // whole atoms with one aligned 32-bit load per row:
+                            // atom a = K-blocks a*4/SPK .. of one tap, scale
+                            // blocks SPK*cb .. SPK*cb + 3 adjacent (host check)
+#pragma unroll
+                            for (int a = 0; a < SPK; ++a) {
+                                if (4 * g + a * (4 / SPK) >= nkb) break;
+                                const ConvTap T = p.taps[k2.tap];
+                                const int cb = k2.cb;
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
+                                    if (ra_ok[j] && ra_aw[j] == T.aw && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W)
+                                        na[a][j] = __ldg(reinterpret_cast<const uint32_t *>(
+                                            p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch + ra_off[j] +
+                                            SPK * cb));
+                                }
+                                const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch;
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    if (!rb_ok[0][j]) continue;
+                                    if (p.sfb.kb_pitch == 1) {
+                                        nb[a][j] = __ldg(reinterpret_cast<const uint32_t *>(bsrc + rb_off[0][j] + SPK * cb));
+                                    } else {   // the B scales of consecutive blocks are kb_pitch apart
+                                        uint32_t w = 0u;
+#pragma unroll
+                                        for (int q = 0; q < 4; ++q)
+                                            w |= static_cast<uint32_t>(__ldg(bsrc + rb_off[0][j] + (SPK * cb + q) * p.sfb.kb_pitch)) << (8 * q);
+                                        nb[a][j] = w;
+                                    }
+                                }
+                                k2.advance(4 / SPK, p.CB);
+                            }
+                        } else if (g < ngr) {
 #pragma unroll
                             for (int kb = 0; kb < 4; ++kb) {
                                 if (4 * g + kb >= nkb) break;
@@ -957,23 +991,26 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                                 for (int j = 0; j < 4; ++j) {
                                     const int hh = ra_h[j] + T.sf_dh, ww = ra_w[j] + T.sf_dw;
                                     if (ra_ok[j] && ra_aw[j] == T.aw && hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W) {
+                                        // scale block SPK*cb + q along K, kb_pitch bytes apart
                                         const uint8_t *src = p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
-                                                             ra_off[j] + cb * p.sfa.kb_pitch;
+                                                             ra_off[j];
                                         uint32_t w = 0u;
 #pragma unroll
                                         for (int q = 0; q < SPK; ++q)
-                                            if (SPK * cb + q < p.sfa.nblk) w |= static_cast<uint32_t>(__ldg(src + q)) << (8 * q);
+                                            if (SPK * cb + q < p.sfa.nblk)
+                                                w |= static_cast<uint32_t>(__ldg(src + (SPK * cb + q) * p.sfa.kb_pitch)) << (8 * q);
                                         na[(kb * SPK) >> 2][j] |= w << (8 * ((kb * SPK) & 3));
                                     }
                                 }
-                                const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch + cb * p.sfb.kb_pitch;
+                                const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch;
 #pragma unroll
                                 for (int j = 0; j < 4; ++j) {
                                     if (!rb_ok[0][j]) continue;
                                     uint32_t w = 0u;
 #pragma unroll
                                     for (int q = 0; q < SPK; ++q)
-                                        if (SPK * cb + q < p.sfb.nblk) w |= static_cast<uint32_t>(__ldg(bsrc + rb_off[0][j] + q)) << (8 * q);
+                                        if (SPK * cb + q < p.sfb.nblk)
+                                            w |= static_cast<uint32_t>(__ldg(bsrc + rb_off[0][j] + (SPK * cb + q) * p.sfb.kb_pitch)) << (8 * q);
                                     nb[(kb * SPK) >> 2][j] |= w << (8 * ((kb * SPK) & 3));
                                 }
                                 k2.advance(1, p.CB);

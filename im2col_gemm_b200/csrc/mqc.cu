@@ -240,7 +240,8 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     const int cache = KIND == kConv ? P.NT * P.groups * P.nb_atoms * 512 : 0;
     P.sfb_cached = KIND == kConv && cache <= 16384 && !P.sfb_vec4 && !nv;
     // the 32-bit scale path reads B four bytes at a time unless B is cached
-    if (!P.sfb_cached && !P.sfb_vec4) P.sf_vec4 = 0;
+    // (the packed-FP4 path has its own vector loads for both operands)
+    if (!P.sfb_cached && !P.sfb_vec4 && !nv) P.sf_vec4 = 0;
     // k16: the zero block (4 KB) 1 KB past the barriers; quantized output:
     // eight 32 x 36-byte transposition buffers there
     const bool qout = KIND == kConv && P.q_codes != nullptr;
@@ -1028,14 +1029,18 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
         G.sfa.pix_pitch = (sqx16 ? ceil_div(N, 16) : N) * nb;
         G.sfa.row_shift = sqx16 ? 4 : 0;
         G.sfa.row_pitch = static_cast<int32_t>(nb);
-        G.sfa.kb_pitch = 4;
+        G.sfa.kb_pitch = 1;
         G.sfa.nblk = static_cast<int32_t>(nb);
         G.sfb.tap_pitch = (sqw16 ? ceil_div(K, 16) : K) * nb;
         G.sfb.row_shift = sqw16 ? 4 : 0;
         G.sfb.row_pitch = static_cast<int32_t>(nb);
-        G.sfb.kb_pitch = 4;
+        G.sfb.kb_pitch = 1;
         G.sfb.nblk = static_cast<int32_t>(nb);
-        G.sf_vec4 = G.sfb_vec4 = 0;
+        // whole 4-byte atoms per load: every pitch and the block count
+        // multiples of 4 (then no block is past the row), aligned bases
+        G.sf_vec4 = nb % 4 == 0 && G.sfa.pix_pitch % 4 == 0 && G.sfb.tap_pitch % 4 == 0 &&
+                    (reinterpret_cast<uintptr_t>(xs) & 3u) == 0 && (reinterpret_cast<uintptr_t>(ws) & 3u) == 0;
+        G.sfb_vec4 = 0;
         G.nv_tx = nva->x_tscale;
         G.nv_tw = nva->w_tscale;
         G.pk = 2;
@@ -1045,13 +1050,17 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
         const int64_t nb = round_up(C, 32) / 32;     // (Cp above counts bytes here)
         G.sfa.pix_pitch = (sqx ? nb32(N) : N) * nb;
         G.sfa.row_pitch = static_cast<int32_t>(nb);
-        G.sfa.kb_pitch = 2;
+        G.sfa.kb_pitch = 1;
         G.sfa.nblk = static_cast<int32_t>(nb);
         G.sfb.tap_pitch = (sqw ? nb32(K) : K) * nb;
         G.sfb.row_pitch = static_cast<int32_t>(nb);
-        G.sfb.kb_pitch = 2;
+        G.sfb.kb_pitch = 1;
         G.sfb.nblk = static_cast<int32_t>(nb);
-        G.sf_vec4 = G.sfb_vec4 = 0;
+        // two K-blocks (4 scale bytes) per aligned load: an even number of
+        // K-blocks per tap, pitches and the block count multiples of 4
+        G.sf_vec4 = G.CB % 2 == 0 && nb % 4 == 0 && G.sfa.pix_pitch % 4 == 0 && G.sfb.tap_pitch % 4 == 0 &&
+                    (reinterpret_cast<uintptr_t>(xs) & 3u) == 0 && (reinterpret_cast<uintptr_t>(ws) & 3u) == 0;
+        G.sfb_vec4 = 0;
         G.pk = 1;
     }
     G.out = y;
@@ -1169,13 +1178,23 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
                               mqc_conv2d_bwd_data_workspace_bytes(c, wf, gf))) != MQC_OK)
         return st;
     uint8_t *wsp = static_cast<uint8_t *>(workspace);
+    const SubpixPlan sp = subpix_plan(c, wf);
+    // both operands OCP MXFP4 and the per-phase plan: the packed codes go to
+    // the tensor core as they are (kind::mxf4), no widening
+    const bool mxf4 = !sp.on && wf->fmt == MQC_E2M1 && gf->fmt == MQC_E2M1;
     GemmOperand ow, og;
-    if ((st = gemm_operand(wq, wf, K, C, R, S, wsp, static_cast<cudaStream_t>(stream), ow)) != MQC_OK) return st;
-    if ((st = gemm_operand(gq, gf, N, K, P, Q, wsp, static_cast<cudaStream_t>(stream), og)) != MQC_OK) return st;
+    if (!mxf4) {
+        if ((st = gemm_operand(wq, wf, K, C, R, S, wsp, static_cast<cudaStream_t>(stream), ow)) != MQC_OK) return st;
+        if ((st = gemm_operand(gq, gf, N, K, P, Q, wsp, static_cast<cudaStream_t>(stream), og)) != MQC_OK) return st;
+    } else {
+        ow.codes = static_cast<const uint8_t *>(wq);
+        og.codes = static_cast<const uint8_t *>(gq);
+        ow.mma_fmt = og.mma_fmt = MQC_E2M1;
+        ow.inner = og.inner = round_up(K, 32) / 2;     // bytes of a row of K codes padded to 32
+    }
     const int64_t Kp = og.inner, Kpw = ow.inner;   // padded output-channel extents of G_Y and W rows
     const bool sqg = gf->block == MQC_BLOCK_SQ32, sqw = wf->block == MQC_BLOCK_SQ32;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
-    const SubpixPlan sp = subpix_plan(c, wf);
     if (sp.on) {
         if (ow.inner != sp.g.kpw) return fail(MQC_ERR_UNSUPPORTED, "conv2d_bwd_data: weight row padding mismatch");
         uint8_t *scodes = wsp, *sscales = wsp + sp.codes_bytes;
@@ -1386,6 +1405,24 @@ mqc_status mqc_conv2d_bwd_data(const void *wq, const uint8_t *ws, const mqc_mx *
         G.sf_vec4 = G.CB % 4 == 0 && G.sfa.pix_pitch % 4 == 0 && G.sfa.row_pitch % 4 == 0 &&
                     (reinterpret_cast<uintptr_t>(gs) & 3u) == 0;
         G.sfb_vec4 = false;   // the weights' scales run along K with a stride of C per block
+        if (mxf4) {
+            // scales per 32 output channels: G_Y [pix][n or n/32][nbK] (blocks
+            // adjacent), W [tap][nbK][C or C/32] (blocks C or C/32 apart)
+            const int64_t nbK = round_up(K, 32) / 32;
+            G.idesc = make_idesc_mxf4(128, G.BN);
+            G.sfa.pix_pitch = (sqg ? nb32(N) : N) * nbK;
+            G.sfa.row_pitch = static_cast<int32_t>(nbK);
+            G.sfa.kb_pitch = 1;
+            G.sfa.nblk = static_cast<int32_t>(nbK);
+            G.sfb.tap_pitch = nbK * (sqw ? nb32(C) : C);
+            G.sfb.kb_pitch = static_cast<int32_t>(sqw ? nb32(C) : C);
+            G.sfb.nblk = static_cast<int32_t>(nbK);
+            // aligned 4-byte loads of the A scales (two K-blocks) when every
+            // tap has an even number of K-blocks and the pitches allow
+            G.sf_vec4 = G.CB % 2 == 0 && nbK % 4 == 0 && G.sfa.pix_pitch % 4 == 0 &&
+                        (reinterpret_cast<uintptr_t>(gs) & 3u) == 0;
+            G.pk = 1;
+        }
         G.out = gx;
         G.os_q = 1;
         G.os_p = int64_t(sh) * W;

@@ -150,7 +150,10 @@ def test_conv_bwd_weight_parity(mqc, orc, case, sq):
 # FP4 (E2M1) operands, alone or mixed with FP8: (case, format of the first
 # operand, format of the second) for each GEMM
 FP4_CASES = [((4, 48, 9, 11, 40, 3, 3, 2, 1), 2, 0), ((16, 16, 12, 12, 32, 3, 3, 2, 1), 2, 2),
-             ((3, 128, 10, 9, 160, 3, 3, 1, 1), 0, 2), ((40, 96, 5, 6, 130, 1, 1, 1, 0), 2, 1)]
+             ((3, 128, 10, 9, 160, 3, 3, 1, 1), 0, 2), ((40, 96, 5, 6, 130, 1, 1, 1, 0), 2, 1),
+             # both operands MXFP4: native kind::mxf4 forward and per-phase input
+             # gradient (odd H: the stride phases do not tile; C, K ragged)
+             ((6, 40, 9, 7, 24, 3, 3, 2, 1), 2, 2), ((5, 70, 8, 8, 100, 3, 3, 1, 1), 2, 2)]
 
 
 @pytest.mark.parametrize("case,fa,fb", FP4_CASES)

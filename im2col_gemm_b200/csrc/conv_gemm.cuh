@@ -153,6 +153,16 @@ struct alignas(64) GemmParams {
     // other 16 from a zero block) and the TMA views take 16 rows of 16 bytes
     // as one 256-byte row: (256, rows / 16, ...) boxes, row coordinates / 16
     int32_t k16;
+    // CONV k16 (narrow forward: 16-byte code rows and a batch of 16): a
+    // pixel's codes of the whole batch are one 256-byte run, the A maps are
+    // (256, W', H') and a box of 8 runs is a tile (rows n fastest, bn = 16,
+    // bq = 8 or bq x bp = 8 with a quantized output); the MMA reads the upper
+    // 16 bytes of every K-block row from the zero block, as for WGRAD
+    // sf_pix: square X blocks, so one scale byte per pixel serves all 16
+    // rows of the pixel (8 bytes per tap and tile, shared by shuffles)
+    // ep_stage: the fp32 tile goes through shared memory as [n][column][q]
+    // so that each (n, channel) gets its 8 consecutive q as 16-byte stores
+    int32_t sf_pix, ep_stage;
     // CONV d2s (input gradient as one sub-pixel GEMM): GEMM column n is
     // (phase n / cpad, channel n % cpad) and lands at channel offset
     // (n % cpad) * os_c + d2s_off[phase]; cpad is a multiple of 16.
@@ -509,8 +519,10 @@ __device__ __forceinline__ void qout_chunk(const GemmParams &p, const uint32_t (
     }
 }
 
-template <int KIND, bool SFV4, int UMT, bool QOUT = false, int PK = 0>
+template <int KIND, bool SFV4, int UMT, bool QOUT = false, int PK = 0, bool NAR = false>
 __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
+    // NAR: the narrow forward (k16 CONV: whole-batch pixel runs, per-pixel
+    // scale gather, staged epilogue); its code is only in these instances
     constexpr int SPK = PK == 2 ? 4 : (PK == 1 ? 2 : 1);   // scale bytes per row and K-block = atoms per group
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
@@ -541,13 +553,17 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
     uint64_t *empty = full + S;
     uint64_t *acc_full = empty + S;
     uint64_t *acc_empty = acc_full + kMaxAcc;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + kMaxAcc);
+    uint64_t *ep_bar = acc_empty + kMaxAcc;       // ep_stage: one per epilogue team (4 warps)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(ep_bar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
     // k16: the upper 16 bytes of every operand row (batch 16..31 of a K-block)
     // are read by the MMA from this zero block (256 rows x 16 bytes)
     uint8_t *sZ = reinterpret_cast<uint8_t *>(full) + 1024;
-    // QOUT: eight 32 x 36-byte transposition buffers (one per epilogue warp)
-    uint32_t *sTr = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(full) + 1024);
+    // QOUT: eight 32 x 36-byte transposition buffers (one per epilogue warp);
+    // ep_stage: two buffers per team of 16 planes (n) x 260 floats ([column][q]
+    // padded by 4, so that the 16 rows n of a store hit 8 banks pairwise)
+    uint32_t *sTr = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(full) + 1024 + (p.k16 ? 4096 : 0));
+    float *sEp = reinterpret_cast<float *>(sTr);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -561,6 +577,8 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
             mbar_init(&acc_full[a], 1);
             mbar_init(&acc_empty[a], 4);
         }
+        mbar_init(&ep_bar[0], 4);
+        mbar_init(&ep_bar[1], 4);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -656,8 +674,10 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
                                 if (i >= UM) break;
-                                uint8_t *dst = a_dst + i * a_sub_stage + j * 128 * row_bytes;
-                                if (p.sub > 1)   // slot dimension of extent 1: only slot T.aw is in range
+                                uint8_t *dst = a_dst + i * a_sub_stage + j * 128 * srow;
+                                if (NAR)           // 8 pixels x the whole batch (256-byte runs)
+                                    tma_load_3d(dst, &p.amap[T.map], &full[s], 0, oq[i] + T.dw, op[i] + T.dh);
+                                else if (p.sub > 1)   // slot dimension of extent 1: only slot T.aw is in range
                                     tma_load_5d(dst, &p.amap[T.map], &full[s], cx, -T.aw, oq[i] + T.dw, op[i] + T.dh,
                                                 on[i]);
                                 else if (p.rows_nfirst)
@@ -665,7 +685,7 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                                 else
                                     tma_load_4d(dst, &p.amap[T.map], &full[s], cx, oq[i] + T.dw, op[i] + T.dh, on[i]);
                             }
-                            tma_load_3d(b_dst + j * p.BN * row_bytes, &p.bmap[0], &full[s], cx, I.col0, T.btap);
+                            tma_load_3d(b_dst + j * p.BN * srow, &p.bmap[0], &full[s], cx, I.col0, T.btap);
                         }
                         kw.advance(p.wkb, p.CB);
                     }
@@ -1062,6 +1082,45 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                                             wb[at][j] = __ldg(reinterpret_cast<const uint32_t *>(bsrc + rb_off[at][j]));
                             }
                             k2.advance(4, p.CB);
+                        } else if (KIND == kConv && NAR && p.sf_pix) {
+                            // 8 pixels x 16 batch rows, one scale byte per pixel
+                            // and tap: lane l loads pixel l % 8 of K-block l / 8
+                            // (one tap each, CB = 1); row m takes pixel m / 16
+                            int q0 = I.q0, p0 = I.p0, n0 = I.n0;
+                            if (i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
+                            const int pi = lane & 7, kbl = lane >> 3;
+                            uint32_t v = 0u;
+                            if (4 * g + kbl < nkb) {
+                                const ConvTap T = p.taps[k2.tap + kbl];
+                                const int ip = static_cast<int>(p.fd_bq.div(static_cast<uint32_t>(pi)));
+                                const int q = q0 + pi - ip * p.bq, pr = p0 + ip;
+                                const int hh = p.a_st_h * pr + T.sf_dh, ww = p.a_st_w * q + T.sf_dw;
+                                if (q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n0 < p.Ne && hh >= 0 && hh < p.sfa.H &&
+                                    ww >= 0 && ww < p.sfa.W)
+                                    v = __ldg(p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
+                                              (n0 >> 5) * p.sfa.row_pitch);
+                            }
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int pix = (lane >> 4) + 2 * j;
+                                uint32_t w = 0u;
+#pragma unroll
+                                for (int kb = 0; kb < 4; ++kb) w |= __shfl_sync(0xFFFFFFFFu, v, pix + 8 * kb) << (8 * kb);
+                                wa[j] = w;
+                            }
+                            for (int kb = 0; kb < 4 && 4 * g + kb < nkb; ++kb) {
+                                if (gb) {
+                                    const ConvTap T = p.taps[k2.tap];
+                                    const uint8_t *bsrc = p.sfb.base + static_cast<int64_t>(T.btap) * p.sfb.tap_pitch;
+#pragma unroll
+                                    for (int at = 0; at < 2; ++at)
+#pragma unroll
+                                        for (int j = 0; j < 4; ++j)
+                                            if (rb_ok[at][j])
+                                                wb[at][j] |= static_cast<uint32_t>(__ldg(bsrc + rb_off[at][j])) << (8 * kb);
+                                }
+                                k2.advance(1, p.CB);
+                            }
                         } else if (KIND == kConv) {
                             for (int kb = 0; kb < 4 && 4 * g + kb < nkb; ++kb) {
                                 const ConvTap T = p.taps[k2.tap];
@@ -1216,7 +1275,9 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
         // measured slower with twice as many in flight)
         const int nteams = KIND == kConv && p.nacc >= 2 && !p.d2s ? 2 : 1;
         uint32_t tcount = 0;
-        for (int u = blockIdx.x; u < p.num_units && team < nteams; u += gridDim.x) {
+        uint32_t ep_round = 0;                 // ep_stage: staging rounds of this team (buffer, barrier phase)
+        bool ep_fail = false;
+        for (int u = blockIdx.x; u < p.num_units && team < nteams && !ep_fail; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
             // output row of this thread in sub-tile i
             bool row_ok;
@@ -1292,6 +1353,50 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                         if (I.col0 + c0 < p.Ncols)
                             qout_chunk(p, r, row_ok, qpix, n0 + in, I.col0 + c0, sTr + (team * 4 + qd) * (32 * 9), lane);
                     }
+                    continue;
+                }
+                if (KIND == kConv && NAR && !QOUT && p.ep_stage) {
+                    // batch-first rows: row m is batch m % 16 at pixel m / 16
+                    // (q0 + m / 16); the team writes the tile as [n][column][q]
+                    // and warp qd stores batch rows 4 qd .. 4 qd + 3, each
+                    // (n, channel) as two 16-byte runs of 4 q
+                    int q0 = I.q0, p0 = I.p0, n0 = I.n0;
+                    if (i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
+                    for (int c0 = 0; c0 < p.BN; c0 += 32) {
+                        uint32_t r[32];
+                        tc_ld_32x32b_x32(t_row + c0, r);
+                        tc_wait_ld();
+                        if (i + 1 == UM && c0 + 32 >= p.BN) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                        }
+                        float *stg = sEp + (team * 2 + (ep_round & 1u)) * (16 * 260);
+                        float *w = stg + (m & 15) * 260 + (m >> 4);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) w[jj * 8] = __uint_as_float(r[jj]);
+                        // the four warps of the team have written the tile (a
+                        // buffer is rewritten two rounds later, after every
+                        // warp has passed the next round's barrier, i.e. has
+                        // finished reading it)
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ep_bar[team]);
+                        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ep_bar[team], ep_round & 1u, lim, abort_flag))) {
+                            ep_fail = true;
+                            break;
+                        }
+                        ++ep_round;
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            const int idx = t * 32 + lane;
+                            const int nn = qd * 4 + (idx >> 6), k = (idx >> 1) & 31, half = idx & 1;
+                            const float4 v = *reinterpret_cast<const float4 *>(stg + nn * 260 + k * 8 + half * 4);
+                            const int n = n0 + nn, col = I.col0 + c0 + k, q = q0 + half * 4;
+                            if (n < p.Ne && col < p.Ncols && q < p.ph_Qe[0] && p0 < p.ph_Pe[0])
+                                *reinterpret_cast<float4 *>(p.out + n * p.os_n + col * p.os_c + p0 * p.os_p + q) = v;
+                        }
+                    }
+                    if (ep_fail) break;
                     continue;
                 }
                 float *orow = p.out + row_off;

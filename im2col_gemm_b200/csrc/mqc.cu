@@ -89,9 +89,10 @@ int conv_Q(const mqc_conv *c) { return (c->W + 2 * c->pad_w - c->S) / c->stride_
 struct DevInfo {
     int sms = 0;
     int max_smem = 0;
-    bool gemm_attr[16] = {};  // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind, [7] SFV4 weight
+    bool gemm_attr[20] = {};  // [0] weight gradient, [1 + 3 * SFV4 + log2(um)] forward kind, [7] SFV4 weight
                               // gradient, [8 + 1 + 3 * SFV4 + log2(um)] forward with a quantized output,
-                              // [8] MXFP4 and [15] NVFP4 forward on packed codes
+                              // [8] MXFP4 and [15] NVFP4 forward on packed codes, [16 + 2 * quantized
+                              // output + (um == 4)] narrow forward
     bool quant_attr[72] = {};    // staged quantizer, [36*sr + (fmt*3 + blk)*4 + tile]
 };
 std::mutex g_dev_mu;
@@ -243,10 +244,13 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     // (the packed-FP4 path has its own vector loads for both operands)
     if (!P.sfb_cached && !P.sfb_vec4 && !nv) P.sf_vec4 = 0;
     // k16: the zero block (4 KB) 1 KB past the barriers; quantized output:
-    // eight 32 x 36-byte transposition buffers there
+    // eight 32 x 36-byte transposition buffers there (after the zero block)
     const bool qout = KIND == kConv && P.q_codes != nullptr;
-    const int fixed = 1024 + (P.k16 ? 1024 + 4096 : (qout ? 1024 + 8 * 32 * 36 : 64 * 8 + 64)) +
-                      (P.sfb_cached ? cache : 0);
+    // ep_stage: two 16 x 260-float buffers per epilogue team after them
+    const int extra = (P.k16 || qout) ? 1024 + (P.k16 ? 4096 : 0) + (qout ? 8 * 32 * 36 : 0) +
+                                            (P.ep_stage ? 2 * 2 * 16 * 260 * 4 : 0)
+                                      : 64 * 8 + 64;
+    const int fixed = 1024 + extra + (P.sfb_cached ? cache : 0);
     // CONV with few K-blocks per tile and narrow column tiles: units of
     // um = 2 or 4 row tiles, so that the per-unit work of every role (decode,
     // barrier round trips, B loads, scale atoms of B) is shared by um MMAs;
@@ -259,6 +263,7 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
         P.MTILES = P.TQ * P.TP * P.TN;
         if (P.total_kb <= 9 && P.BN <= 32 && !nv) {
             for (int um = 4; um >= 2; um /= 2) {
+                if (P.k16 && um == 2) continue;    // the narrow kernels come with units of 1 or 4
                 const int64_t units = ceil_div(P.MTILES, um) * int64_t(P.nph) * P.NT;
                 if (2 * um * P.BN <= 256 && units >= 2 * d.sms) {
                     P.um = um;
@@ -312,7 +317,10 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     const int smem = fixed + S * per_stage;
     const bool v4 = KIND == kConv && P.sf_vec4;
     auto kernel = P.sq_gather ? conv_gemm_kernel<kWgrad, true, 1> : conv_gemm_kernel<kWgrad, false, 1>;
-    if (pk == 2) {
+    if (KIND == kConv && P.k16) {
+        if (qout) kernel = P.um == 4 ? conv_gemm_kernel<kConv, false, 4, true, 0, true> : conv_gemm_kernel<kConv, false, 1, true, 0, true>;
+        else kernel = P.um == 4 ? conv_gemm_kernel<kConv, false, 4, false, 0, true> : conv_gemm_kernel<kConv, false, 1, false, 0, true>;
+    } else if (pk == 2) {
         kernel = conv_gemm_kernel<kConv, false, 1, false, 2>;
     } else if (pk == 1) {
         kernel = conv_gemm_kernel<kConv, false, 1, false, 1>;
@@ -325,7 +333,8 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
         else if (P.um == 2) kernel = v4 ? conv_gemm_kernel<kConv, true, 2, true> : conv_gemm_kernel<kConv, false, 2, true>;
         else kernel = v4 ? conv_gemm_kernel<kConv, true, 1, true> : conv_gemm_kernel<kConv, false, 1, true>;
     }
-    const int ai = pk == 2 ? 15 : pk == 1 ? 8
+    const int ai = KIND == kConv && P.k16 ? 16 + (qout ? 2 : 0) + (P.um == 4 ? 1 : 0)
+                   : pk == 2 ? 15 : pk == 1 ? 8
                       : KIND == kConv ? (qout ? 8 : 0) + 1 + (v4 ? 3 : 0) + (P.um == 4 ? 2 : P.um - 1)
                                       : (P.sq_gather ? 7 : 0);
     if (!d.gemm_attr[ai]) {
@@ -900,11 +909,21 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
         ox.inner = ow.inner = round_up(C, 32) / 2;
     }
     const int64_t Cp = ox.inner, Cpw = ow.inner;   // padded channel extents of X and W rows (bytes)
+    // narrow channels (one 16-byte code row: C <= 16 of an 8-bit format) and
+    // a batch of 16: a pixel's codes of the whole batch are one contiguous
+    // 256-byte run, and an A box of 8 such runs is a whole tile (rows n
+    // fastest), instead of 128 separate 16-byte rows
+    const bool narrow = nva == nullptr && !mxf4 && Cp == 16 && Cpw == 16 && N == 16;
     GemmParams G;
     memset(&G, 0, sizeof G);
     G.CB = static_cast<int32_t>(nb32(Cp));
     G.wkb = largest_wkb(G.CB);
-    if (qo == nullptr) {
+    G.k16 = narrow ? 1 : 0;
+    if (narrow && qo == nullptr) {
+        G.bn = 16;
+        G.bq = 8;
+        G.bp = 1;
+    } else if (qo == nullptr) {
         choose_rows(Q, P, N, G.bq, G.bp, G.bn);
     } else {
         // quantized output: rows n fastest, bn = 16 (a batch of at most 16)
@@ -938,7 +957,7 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
                      : make_idesc_mx(mma_fmt(ox.mma_fmt), mma_fmt(ow.mma_fmt), 128, G.BN);
     // A: one map per stride phase; dims (C, W', H', N) so that rows run along q
     bool phase_ok[16] = {};
-    for (int attempt = qo ? 1 : 0; attempt < 2; ++attempt) {
+    for (int attempt = (qo || narrow) ? 1 : 0; attempt < 2; ++attempt) {
         G.rows_nfirst = attempt;
         st = MQC_OK;
         for (int a = 0; a < sh && st == MQC_OK; ++a)
@@ -947,7 +966,13 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
                 phase_ok[a * sw + b] = Hh > 0 && Ww > 0;
                 if (!phase_ok[a * sw + b]) continue;
                 const uint8_t *base = ox.codes + (int64_t(a) * W + b) * N * Cp;
-                if (!G.rows_nfirst) {
+                if (narrow) {
+                    // (n and c as one 256-byte dimension, W', H') of phase (a, b)
+                    const uint64_t dims[3] = {uint64_t(N) * Cp, uint64_t(Ww), uint64_t(Hh)};
+                    const uint64_t strd[2] = {uint64_t(sw) * N * Cp, uint64_t(sh) * W * N * Cp};
+                    const uint32_t box[3] = {uint32_t(N * Cp), uint32_t(G.bq), uint32_t(G.bp)};
+                    st = encode_codes_map(&G.amap[a * sw + b], base, 3, dims, strd, box, 0);
+                } else if (!G.rows_nfirst) {
                     const uint64_t dims[4] = {uint64_t(Cp), uint64_t(Ww), uint64_t(Hh), uint64_t(N)};
                     const uint64_t strd[3] = {uint64_t(sw) * N * Cp, uint64_t(sh) * W * N * Cp, uint64_t(Cp)};
                     const uint32_t box[4] = {uint32_t(32 * G.wkb), uint32_t(G.bq), uint32_t(G.bp), uint32_t(G.bn)};
@@ -965,8 +990,9 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
     {
         const uint64_t dims[3] = {uint64_t(Cpw), uint64_t(K), uint64_t(R) * S};
         const uint64_t strd[2] = {uint64_t(Cpw), uint64_t(K) * Cpw};
-        const uint32_t box[3] = {uint32_t(32 * G.wkb), uint32_t(box_rows(K, G.BN)), 1u};
-        if ((st = encode_codes_map(&G.bmap[0], ow.codes, 3, dims, strd, box, G.wkb)) != MQC_OK) return st;
+        const uint32_t box[3] = {uint32_t(narrow ? 16 : 32 * G.wkb), uint32_t(box_rows(K, G.BN)), 1u};
+        if ((st = encode_codes_map(&G.bmap[0], ow.codes, 3, dims, strd, box, narrow ? 0 : G.wkb)) != MQC_OK)
+            return st;
     }
     G.ntaps = 0;
     for (int r = 0; r < R; ++r)
@@ -998,11 +1024,16 @@ static mqc_status conv_fwd_impl(const void *xq, const uint8_t *xs, const mqc_mx 
         if (!phase_ok[i]) G.amap[i] = G.amap[0];
     G.n_amaps = sh * sw;
     G.n_bmaps = 1;
-    G.a_box_bytes = 32 * G.wkb * G.bq * G.bp * G.bn;
-    G.b_box_bytes = 32 * G.wkb * box_rows(K, G.BN);
+    const int rowb = narrow ? 16 : 32 * G.wkb;     // shared-memory bytes of a row of a box
+    G.a_box_bytes = rowb * G.bq * G.bp * G.bn;
+    G.b_box_bytes = rowb * box_rows(K, G.BN);
     G.a_slab = 128;
     G.b_slab = G.BN;
     const bool sqx = xf->block == MQC_BLOCK_SQ32, sqw = wf->block == MQC_BLOCK_SQ32;
+    // square X blocks: the 16 rows of a pixel share its scale byte
+    G.sf_pix = narrow && sqx ? 1 : 0;
+    // the staged fp32 epilogue stores 16-byte runs of q: 16-byte aligned rows
+    G.ep_stage = narrow && qo == nullptr && Q % 4 == 0 && (reinterpret_cast<uintptr_t>(y) & 15u) == 0 ? 1 : 0;
     G.sfa.base = xs;
     G.sfa.pix_pitch = (sqx ? nb32(N) : N) * nb32(Cp);
     G.sfa.row_shift = sqx ? 5 : 0;

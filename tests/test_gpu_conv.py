@@ -55,6 +55,12 @@ FWD_CASES = [
     (3, 128, 10, 9, 160, 3, 3, 1, 1),     # two column tiles, 4-block boxes
     (8, 96, 7, 6, 256, 1, 1, 1, 0),       # C with 3 blocks
     (5, 32, 12, 12, 24, 2, 3, 1, 0),      # non-square kernel, K < 32
+    # batch 16 with 16-byte code rows (C <= 16): whole-batch pixel runs,
+    # batch-first rows; Q a multiple of 4 takes the staged epilogue
+    (16, 16, 24, 24, 32, 3, 3, 2, 1),     # Q = 12: the last 8-wide tile half empty
+    (16, 3, 17, 33, 40, 3, 3, 1, 1),      # C = 3, odd Q (plain stores), K = 40 (48-column tile)
+    (16, 8, 16, 16, 96, 1, 1, 1, 0),      # 1x1, three 32-column chunks
+    (16, 16, 10, 17, 20, 2, 3, 2, 0),     # non-square kernel, Q = 8, K = 20
 ]
 
 

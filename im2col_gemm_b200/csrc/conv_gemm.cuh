@@ -900,7 +900,29 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                     }
                 }
             };
-            set_rows(0);
+            // NAR, sf_pix: per sub-tile i, this lane's pixel (lane % 8) as a
+            // scale row and column before the tap offset (a row far out of
+            // range for pixels past the output) and its batch block offset
+            int np_h[4] = {0, 0, 0, 0}, np_w[4] = {0, 0, 0, 0}, np_o[4] = {0, 0, 0, 0};
+            const bool nar_pix = KIND == kConv && NAR && p.sf_pix;
+            if (nar_pix) {
+                const int pi = lane & 7;
+                const int ip = static_cast<int>(p.fd_bq.div(static_cast<uint32_t>(pi)));
+                const int iq = pi - ip * p.bq;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (i >= UM) break;
+                    int q0 = I.q0, p0 = I.p0, n0 = I.n0;
+                    if (i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
+                    const int q = q0 + iq, pr = p0 + ip;
+                    const bool okp = q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n0 < p.Ne;
+                    np_h[i] = okp ? p.a_st_h * pr : -(1 << 20);
+                    np_w[i] = p.a_st_w * q;
+                    np_o[i] = (n0 >> 5) * p.sfa.row_pitch;
+                }
+            } else {
+                set_rows(0);
+            }
             // B rows of this lane: col0 + 128 at + 32 j + lane
             // (WGRAD: with tap groups a B row is (tap, channel) and carries
             // its tap's pixel offset; otherwise every row has the unit's tap)
@@ -961,6 +983,21 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                 bool slot = false;
                 for (int g = 0; g < GA && ok; ++g) {
                   const KbWalker kg = k2;                 // start of the group (each sub-tile walks it)
+                  // NAR, sf_pix: scale offsets of this lane's K-block (lane / 8,
+                  // one tap each) of the group, read uniformly (out of range
+                  // past the stage's K-blocks)
+                  int tdh = -(1 << 20), tdw = 0;
+                  if (nar_pix) {
+#pragma unroll
+                      for (int kb = 0; kb < 4; ++kb)
+                          if (4 * g + kb < nkb) {
+                              const ConvTap T = p.taps[kg.tap + kb];
+                              if (kb == (lane >> 3)) {
+                                  tdh = T.sf_dh;
+                                  tdw = T.sf_dw;
+                              }
+                          }
+                  }
                   for (int i = 0; i < UM; ++i) {
                     if constexpr (KIND == kConv && PK != 0) {
                         // SPK scales per row and K-block (2 E8M0 for MXFP4, 4
@@ -1053,7 +1090,7 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                         continue;
                     }
                     if (UM > 1) {
-                        set_rows(i);
+                        if (!nar_pix) set_rows(i);
                         k2 = kg;
                     }
                     const bool gb = i == 0 && !skip_b;      // B atoms: once per group
@@ -1086,20 +1123,18 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                             // 8 pixels x 16 batch rows, one scale byte per pixel
                             // and tap: lane l loads pixel l % 8 of K-block l / 8
                             // (one tap each, CB = 1); row m takes pixel m / 16
-                            int q0 = I.q0, p0 = I.p0, n0 = I.n0;
-                            if (i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
-                            const int pi = lane & 7, kbl = lane >> 3;
+                            int bh = np_h[0], bw = np_w[0], bo = np_o[0];
+#pragma unroll
+                            for (int t = 1; t < 4; ++t)
+                                if (t == i) {
+                                    bh = np_h[t];
+                                    bw = np_w[t];
+                                    bo = np_o[t];
+                                }
+                            const int hh = bh + tdh, ww = bw + tdw;
                             uint32_t v = 0u;
-                            if (4 * g + kbl < nkb) {
-                                const ConvTap T = p.taps[k2.tap + kbl];
-                                const int ip = static_cast<int>(p.fd_bq.div(static_cast<uint32_t>(pi)));
-                                const int q = q0 + pi - ip * p.bq, pr = p0 + ip;
-                                const int hh = p.a_st_h * pr + T.sf_dh, ww = p.a_st_w * q + T.sf_dw;
-                                if (q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n0 < p.Ne && hh >= 0 && hh < p.sfa.H &&
-                                    ww >= 0 && ww < p.sfa.W)
-                                    v = __ldg(p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch +
-                                              (n0 >> 5) * p.sfa.row_pitch);
-                            }
+                            if (hh >= 0 && hh < p.sfa.H && ww >= 0 && ww < p.sfa.W)
+                                v = __ldg(p.sfa.base + (static_cast<int64_t>(hh) * p.sfa.W + ww) * p.sfa.pix_pitch + bo);
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 const int pix = (lane >> 4) + 2 * j;

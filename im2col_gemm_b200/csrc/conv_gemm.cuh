@@ -117,6 +117,11 @@ struct alignas(64) GemmParams {
     int32_t sq_gather;           // WGRAD: square blocks on both operands, 16-row groups of an atom aligned
     int32_t sq16;                // WGRAD, sq_gather: a 32-row group of B may hold two taps (cpad = 16 mod 32)
     int32_t groups;              // CONV: groups of 4 K-blocks per tile
+    // scale-gather warps in use (at most 5 and at most the stages; 0: that
+    // maximum).  Warp w takes the stages w, w + nsf, ...: with every unit
+    // having the same stages, the host picks nsf so that no warp keeps
+    // drawing the largest stage of each unit
+    int32_t nsf;
     // CONV: a unit is um consecutive 128-row tiles (sub-tiles) sharing the
     // B operand, the pipeline stages and the per-unit bookkeeping; each
     // sub-tile has its own accumulator (um x BN TMEM columns per unit)
@@ -163,6 +168,13 @@ struct alignas(64) GemmParams {
     // ep_stage: the fp32 tile goes through shared memory as [n][column][q]
     // so that each (n, channel) gets its 8 consecutive q as 16-byte stores
     int32_t sf_pix, ep_stage;
+    // CONV ep_vec: the 4 rows of each lane quad are 4 consecutive q of one
+    // (p, n) and every output row start is 16-byte aligned: the epilogue
+    // transposes 4 x 4 blocks across the quad and stores 16-byte runs (in the
+    // instances with the 32-bit scale gather or units of several tiles only:
+    // in the others the extra code measured slower on the sub-pixel input
+    // gradient and gained nothing)
+    int32_t ep_vec;
     // CONV d2s (input gradient as one sub-pixel GEMM): GEMM column n is
     // (phase n / cpad, channel n % cpad) and lands at channel offset
     // (n % cpad) * os_c + d2s_off[phase]; cpad is a multiple of 16.
@@ -254,6 +266,35 @@ __device__ __forceinline__ UnitInfo decode_unit(const GemmParams &p, int u) {
         I.nk = (I.nkit + ga - 1) / ga;
     }
     return I;
+}
+
+// 4 x 4 transpose across the lanes of a quad: lane e of the quad holds row e
+// (x0..x3 = columns 0..3) on entry and column e (x0..x3 = rows 0..3) on exit.
+// Two exchange steps, each swapping the off-diagonal halves of 2 x 2 blocks
+// (of single entries with lane e ^ 1, then of 2 x 2 blocks with lane e ^ 2).
+__device__ __forceinline__ void quad_transpose(uint32_t &x0, uint32_t &x1, uint32_t &x2, uint32_t &x3, int e) {
+    const bool odd = (e & 1) != 0, hi = (e & 2) != 0;
+    uint32_t a = odd ? x0 : x1, b = odd ? x2 : x3;
+    a = __shfl_xor_sync(0xFFFFFFFFu, a, 1);
+    b = __shfl_xor_sync(0xFFFFFFFFu, b, 1);
+    if (odd) {
+        x0 = a;
+        x2 = b;
+    } else {
+        x1 = a;
+        x3 = b;
+    }
+    a = hi ? x0 : x2;
+    b = hi ? x1 : x3;
+    a = __shfl_xor_sync(0xFFFFFFFFu, a, 2);
+    b = __shfl_xor_sync(0xFFFFFFFFu, b, 2);
+    if (hi) {
+        x0 = a;
+        x1 = b;
+    } else {
+        x2 = a;
+        x3 = b;
+    }
 }
 
 // Row m (0..127) of a CONV tile -> interleave slot and output coordinates
@@ -844,13 +885,13 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
             __syncwarp();
             ++tcount;
         }
-    } else if (sf_warp_index(warp) >= 0 && sf_warp_index(warp) < min(kNumSfWarps, S)) {
+    } else if (sf_warp_index(warp) >= 0 && sf_warp_index(warp) < (p.nsf > 0 ? p.nsf : min(kNumSfWarps, S))) {
         // ------------------------------------------------------------ scale-factor gather
         // scale warp w handles the stages whose global index is w modulo nsf.
         // nsf <= S: a warp's consecutive stages are at most S apart, so when
         // it waits for slot s it is never two phases ahead of the consumer
         // (a parity wait cannot tell phase r from phase r - 2)
-        const int nsf = min(kNumSfWarps, S);
+        const int nsf = p.nsf > 0 ? p.nsf : min(kNumSfWarps, S);
         const int sfw = sf_warp_index(warp);
         uint32_t it = 0;             // global index of the first stage of the unit
         uint32_t gnext = static_cast<uint32_t>(sfw);   // global index of this warp's next stage
@@ -1497,6 +1538,24 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                         continue;
                     }
                     const int cb = I.col0 + c0;
+                    if (KIND == kConv && PK != 2 && (SFV4 || UM > 1) && p.ep_vec) {
+                        // lane quad = 4 consecutive q (row_ok is the same for
+                        // the 4): per block of 4 columns, lane e stores column
+                        // 4 b + e of the quad's 4 rows as one 16-byte run
+                        const int e = lane & 3;
+                        float *qrow = orow - e;
+#pragma unroll
+                        for (int b = 0; b < 8; ++b) {
+                            uint32_t x0 = r[4 * b], x1 = r[4 * b + 1], x2 = r[4 * b + 2], x3 = r[4 * b + 3];
+                            quad_transpose(x0, x1, x2, x3, e);
+                            const int col = cb + 4 * b + e;
+                            if (row_ok && col < p.Ncols)
+                                *reinterpret_cast<float4 *>(qrow + static_cast<int64_t>(col) * p.os_c) =
+                                    make_float4(__uint_as_float(x0), __uint_as_float(x1), __uint_as_float(x2),
+                                                __uint_as_float(x3));
+                        }
+                        continue;
+                    }
                     const int nv = row_ok ? min(32, p.Ncols - cb) : 0;
                     float *op = orow + static_cast<int64_t>(cb) * p.os_c;
                     if constexpr (PK == 2) {

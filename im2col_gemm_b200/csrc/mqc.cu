@@ -293,6 +293,31 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
     const int per_stage = P.kbs == 8 ? ps8 : ps4;
     if (S < 3) return fail(MQC_ERR_UNSUPPORTED, "tile does not fit in shared memory");
     P.stages = S;
+    P.nsf = 0;
+    if (KIND == kConv && P.nph == 1) {
+        // every unit has the same stages (kbs K-blocks, the last one the
+        // rest): over one period of the round robin (lcm of the stages per
+        // unit and the warp count), the busiest warp's K-blocks per unit,
+        // each stage counted one more for its fixed cost; the fewest wins,
+        // ties to more warps
+        const int nk = (P.ph_tkb[0] + P.kbs - 1) / P.kbs;
+        const int nmax = std::min(kNumSfWarps, S);
+        double best = 1e300;
+        for (int nsf = nmax; nsf >= 1 && nk > 0; --nsf) {
+            int L = nk;
+            while (L % nsf != 0) L += nk;
+            double worst = 0.0;
+            for (int w = 0; w < nsf; ++w) {
+                int load = 0;
+                for (int g = w; g < L; g += nsf) load += std::min(P.kbs, P.ph_tkb[0] - P.kbs * (g % nk)) + 1;
+                worst = std::max(worst, double(load) * nk / L);
+            }
+            if (worst < best - 1e-9) {
+                best = worst;
+                P.nsf = nsf;
+            }
+        }
+    }
     if (P.sub < 1) P.sub = 1;
     P.fd_NT = make_fastdiv(P.NT);
     P.fd_nph = make_fastdiv(P.nph);
@@ -341,6 +366,18 @@ mqc_status launch_gemm(GemmParams &P, const DevInfo &d, cudaStream_t stream) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.max_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         const_cast<DevInfo &>(d).gemm_attr[ai] = true;
+    }
+    // vector stores of the plain fp32 epilogue: rows q-consecutive in lane
+    // quads (no slots, q fastest, whole quads per p row), every row start and
+    // stride a multiple of 4 floats, the output 16-byte aligned
+    P.ep_vec = 0;
+    if (KIND == kConv && !P.k16 && !qout && pk == 0 && (P.sf_vec4 || P.um > 1) && P.d2s == 0 && P.sub == 1 &&
+        !P.rows_nfirst && P.bq % 4 == 0 &&
+        P.os_q == 1 && P.os_p % 4 == 0 && P.os_c % 4 == 0 && P.os_n % 4 == 0 &&
+        (reinterpret_cast<uintptr_t>(P.out) & 15u) == 0) {
+        bool ok4 = true;
+        for (int ph = 0; ph < P.nph; ++ph) ok4 = ok4 && P.ph_out_base[ph] % 4 == 0 && P.ph_Qe[ph] % 4 == 0;
+        P.ep_vec = ok4 ? 1 : 0;
     }
     const int grid = std::max(1, std::min(P.num_units, d.sms));
     kernel<<<grid, gemm_threads<KIND>(), smem, stream>>>(P);

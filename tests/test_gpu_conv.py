@@ -61,6 +61,11 @@ FWD_CASES = [
     (16, 3, 17, 33, 40, 3, 3, 1, 1),      # C = 3, odd Q (plain stores), K = 40 (48-column tile)
     (16, 8, 16, 16, 96, 1, 1, 1, 0),      # 1x1, three 32-column chunks
     (16, 16, 10, 17, 20, 2, 3, 2, 0),     # non-square kernel, Q = 8, K = 20
+    (6, 40, 12, 20, 30, 3, 3, 1, 1),      # Q = 20, K = 30 (ragged columns)
+    # 16-byte runs of 4 q per lane quad: the 32-bit scale gather (C = 128),
+    # and units of several 128-row tiles (many tiles, one K-block)
+    (4, 128, 8, 12, 30, 1, 1, 1, 0),
+    (16, 32, 80, 80, 30, 1, 1, 1, 0),
 ]
 
 
@@ -99,6 +104,7 @@ DGRAD_CASES = BWD_CASES + [
     (2, 32, 11, 10, 48, 3, 3, 3, 1),
     (3, 16, 13, 12, 32, 5, 5, 2, 2),
     (2, 64, 7, 9, 160, 3, 3, 2, 1),
+    (6, 30, 12, 20, 40, 3, 3, 1, 1),      # stride 1, W = 20: 16-byte runs of 4 w, C = 30 (ragged columns)
 ]
 # the sub-pixel GEMM (stride 2, even H and W, C in 16s): phases no tap reaches
 # (1x1), a 3x3 window of offsets (5x5), column tiles that split the phases

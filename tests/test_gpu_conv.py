@@ -114,6 +114,7 @@ DGRAD_CASES += [
     (3, 16, 12, 10, 32, 5, 5, 2, 2),
     (2, 48, 6, 8, 40, 3, 3, 2, 1),
     (2, 16, 8, 8, 32, 4, 4, 2, 1),
+    (4, 32, 14, 24, 48, 3, 3, 2, 1),      # W = 24: 16-byte runs of 4 column pairs per lane quad
 ]
 
 

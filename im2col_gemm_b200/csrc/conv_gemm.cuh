@@ -318,6 +318,17 @@ __device__ __forceinline__ void conv_row(const GemmParams &p, int m, int &aw, in
     }
 }
 
+// conv_row of row m packed into one word, decoded once per kernel: the slot
+// and the (q, p, n) offsets in bytes 0-3 (each below 128, the slot below
+// 256), bit 31 set when m is past the tile's rows.
+__device__ __forceinline__ uint32_t conv_row_packed(const GemmParams &p, int m) {
+    int aw, iq, ip, in;
+    conv_row(p, m, aw, iq, ip, in);
+    const bool past = m >= p.sub * p.bq * p.bp * p.bn;
+    return static_cast<uint32_t>(aw) | (static_cast<uint32_t>(iq) << 8) | (static_cast<uint32_t>(ip) << 16) |
+           (static_cast<uint32_t>(in) << 24) | (past ? 0x80000000u : 0u);
+}
+
 // Origin (q, p, n) of the 128-row tile mt of a CONV launch (tiles run q
 // fastest, then p, then n; mt past the last tile gives n >= N: all rows out
 // of range, its boxes read zeros).
@@ -564,6 +575,10 @@ template <int KIND, bool SFV4, int UMT, bool QOUT = false, int PK = 0, bool NAR 
 __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(const __grid_constant__ GemmParams p) {
     // NAR: the narrow forward (k16 CONV: whole-batch pixel runs, per-pixel
     // scale gather, staged epilogue); its code is only in these instances
+    // ROWDEC: the tile rows of the gather and epilogue lanes decoded once per
+    // kernel (in the one-tile byte-gather instance the longer-lived registers
+    // measured slower on the sub-pixel input gradient, so it decodes per tile)
+    constexpr bool ROWDEC = KIND == kConv && (SFV4 || UMT > 1);
     constexpr int SPK = PK == 2 ? 4 : (PK == 1 ? 2 : 1);   // scale bytes per row and K-block = atoms per group
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // swizzled operand tiles need 1024-byte alignment
@@ -899,6 +914,12 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
         uint32_t ph = static_cast<uint32_t>(sfw / S) & 1u;
         bool ok = true;
         const bool skip_b = KIND == kConv && p.sfb_cached;
+        // CONV: this lane's rows lane + 32 j, decoded once
+        uint32_t rdec[4] = {0u, 0u, 0u, 0u};
+        if (ROWDEC) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) rdec[j] = conv_row_packed(p, lane + 32 * j);
+        }
         for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
             const uint32_t it_unit = it;
@@ -922,11 +943,10 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                 for (int j = 0; j < 4; ++j) {
                     const int m = lane + 32 * j;
                     if (KIND == kConv) {
-                        int aw, iq, ip, in;
-                        conv_row(p, m, aw, iq, ip, in);
+                        const uint32_t d = ROWDEC ? rdec[j] : conv_row_packed(p, m);
+                        const int aw = d & 0xFF, iq = (d >> 8) & 0xFF, ip = (d >> 16) & 0xFF, in = (d >> 24) & 0x7F;
                         const int q = q0 + iq, pr = p0 + ip, n = n0 + in;
-                        ra_ok[j] = m < p.sub * p.bq * p.bp * p.bn && p.sub * q + aw < p.ph_Qe[I.ph] &&
-                                   pr < p.ph_Pe[I.ph] && n < p.Ne;
+                        ra_ok[j] = !(d >> 31) && p.sub * q + aw < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
                         ra_h[j] = p.a_st_h * pr;
                         ra_w[j] = p.a_st_w * q;
                         ra_aw[j] = aw;
@@ -1353,6 +1373,8 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
         uint32_t tcount = 0;
         uint32_t ep_round = 0;                 // ep_stage: staging rounds of this team (buffer, barrier phase)
         bool ep_fail = false;
+        const uint32_t edec0 = ROWDEC ? conv_row_packed(p, m) : 0u;   // this thread's row, decoded once
+
         for (int u = blockIdx.x; u < p.num_units && team < nteams && !ep_fail; u += gridDim.x) {
             const UnitInfo I = decode_unit<KIND>(p, u);
             // output row of this thread in sub-tile i
@@ -1362,10 +1384,11 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                 if (KIND == kConv) {
                     int q0 = I.q0, p0 = I.p0, n0 = I.n0;
                     if (i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
-                    int aw, iq, ip, in;
-                    conv_row(p, m, aw, iq, ip, in);
-                    const int q = p.sub * (q0 + iq) + aw, pr = p0 + ip, n = n0 + in;
-                    row_ok = m < p.sub * p.bq * p.bp * p.bn && q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
+                    const uint32_t edec = ROWDEC ? edec0 : conv_row_packed(p, m);
+                    const int e_aw = edec & 0xFF, e_iq = (edec >> 8) & 0xFF, e_ip = (edec >> 16) & 0xFF;
+                    const int e_in = (edec >> 24) & 0x7F;
+                    const int q = p.sub * (q0 + e_iq) + e_aw, pr = p0 + e_ip, n = n0 + e_in;
+                    row_ok = !(edec >> 31) && q < p.ph_Qe[I.ph] && pr < p.ph_Pe[I.ph] && n < p.Ne;
                     row_off = p.ph_out_base[I.ph] + n * p.os_n + pr * p.os_p + q * p.os_q;
                 } else {
                     const int k = I.m0 + m;
@@ -1414,9 +1437,9 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                     // next-layer pixel and batch index of this row
                     int q0 = I.q0, p0 = I.p0, n0 = I.n0;
                     if (i > 0) tile_origin(p, I.mt0 + i, q0, p0, n0);
-                    int aw, iq, ip, in;
-                    conv_row(p, m, aw, iq, ip, in);
-                    const int qpix = (p0 + ip) * p.ph_Qe[0] + (q0 + iq);
+                    const uint32_t edec = ROWDEC ? edec0 : conv_row_packed(p, m);
+                    const int e_iq = (edec >> 8) & 0xFF, e_ip = (edec >> 16) & 0xFF, e_in = (edec >> 24) & 0x7F;
+                    const int qpix = (p0 + e_ip) * p.ph_Qe[0] + (q0 + e_iq);
                     for (int c0 = 0; c0 < p.BN; c0 += 32) {
                         uint32_t r[32];
                         tc_ld_32x32b_x32(t_row + c0, r);
@@ -1427,7 +1450,7 @@ __global__ void __launch_bounds__(gemm_threads<KIND>(), 1) conv_gemm_kernel(cons
                             if (lane == 0) mbar_arrive(&acc_empty[acc]);
                         }
                         if (I.col0 + c0 < p.Ncols)
-                            qout_chunk(p, r, row_ok, qpix, n0 + in, I.col0 + c0, sTr + (team * 4 + qd) * (32 * 9), lane);
+                            qout_chunk(p, r, row_ok, qpix, n0 + e_in, I.col0 + c0, sTr + (team * 4 + qd) * (32 * 9), lane);
                     }
                     continue;
                 }

@@ -135,6 +135,34 @@ mqc_status get_encoder() {
     return g_encode ? MQC_OK : fail(MQC_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
 }
 
+// Encoded maps, reused across calls: the key is every input of the encoder
+// (address, rank, extents, strides, box, swizzle), so a hit returns exactly
+// what encoding would (also after a buffer is freed and another lands at the
+// same address).  Direct-mapped, 256 entries, one lock.
+struct MapKey {
+    uint64_t base, dims[5], strides[4];
+    uint32_t box[5];
+    int32_t rank, wkb;
+    int32_t zero;                 // keeps the key free of padding bytes (compared with memcmp)
+};
+static_assert(sizeof(MapKey) == 112, "MapKey must have no padding");
+struct MapSlot {
+    MapKey key;
+    CUtensorMap map;
+    bool used;
+};
+constexpr int kMapCacheSlots = 256;
+MapSlot g_map_cache[kMapCacheSlots];
+std::mutex g_map_mutex;
+
+uint32_t map_key_hash(const MapKey &k) {
+    // FNV-1a over the key's bytes
+    const unsigned char *b = reinterpret_cast<const unsigned char *>(&k);
+    uint32_t h = 2166136261u;
+    for (size_t i = 0; i < sizeof k; ++i) h = (h ^ b[i]) * 16777619u;
+    return h;
+}
+
 // Encode a tiled map over 1-byte codes.  dims[0] is contiguous; strides are
 // the byte strides of dims[1..rank-1]; the inner box is 32*wkb bytes with the
 // matching shared-memory swizzle.
@@ -142,6 +170,25 @@ mqc_status encode_codes_map(CUtensorMap *map, const void *base, int rank, const 
                             const uint64_t *strides, const uint32_t *box, int wkb) {
     mqc_status st = get_encoder();
     if (st != MQC_OK) return st;
+    MapKey key;
+    memset(&key, 0, sizeof key);
+    key.base = reinterpret_cast<uint64_t>(base);
+    key.rank = rank;
+    key.wkb = wkb;
+    for (int i = 0; i < rank && i < 5; ++i) {
+        key.dims[i] = dims[i];
+        key.box[i] = box[i];
+    }
+    for (int i = 0; i + 1 < rank && i < 4; ++i) key.strides[i] = strides[i];
+    const uint32_t slot = map_key_hash(key) % kMapCacheSlots;
+    {
+        std::lock_guard<std::mutex> lock(g_map_mutex);
+        const MapSlot &c = g_map_cache[slot];
+        if (c.used && memcmp(&c.key, &key, sizeof key) == 0) {
+            *map = c.map;
+            return MQC_OK;
+        }
+    }
     cuuint64_t gd[5], gs[4];
     cuuint32_t bx[5], es[5];
     for (int i = 0; i < rank; ++i) {
@@ -165,6 +212,13 @@ mqc_status encode_codes_map(CUtensorMap *map, const void *base, int rank, const 
                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(MQC_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    if (rank <= 5) {
+        std::lock_guard<std::mutex> lock(g_map_mutex);
+        MapSlot &c = g_map_cache[slot];
+        memcpy(&c.key, &key, sizeof key);
+        c.map = *map;
+        c.used = true;
+    }
     return MQC_OK;
 }
 

@@ -226,3 +226,26 @@ def test_device_wait_timeout_is_reported(mqc):
     assert mqc.get_device_status() == 0
     t = torch.ones(4, device="cuda")
     assert float(t.sum()) == 4.0
+
+
+def test_tensor_map_cache_same_address_other_shape(mqc, orc):
+    """Forwards whose activation codes start at the same device address with
+    other extents (and the first shape again): the library reuses encoded
+    tensor maps keyed by every encoder input, so each call must still see its
+    own geometry."""
+    import torch
+    buf = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    for case in [(2, 32, 8, 8, 32, 3, 3, 1, 1), (4, 32, 6, 10, 32, 3, 3, 1, 1), (2, 32, 8, 8, 32, 3, 3, 1, 1)]:
+        N, C, H, W, K, R, S, st, pad = case
+        x = synth.random_tensor((N, C, H, W), seed=1200 + N * H, dist="student_t")
+        w = synth.random_tensor((K, C, R, S), seed=1201 + W, scale=0.05)
+        xq = mqc.quantize_mx(_dev(x), 0, 2, 0)
+        n = xq.codes.numel()
+        buf[:n].copy_(xq.codes)
+        xs = mqc.Quantized(buf[:n], xq.scales, xq.dims, xq.mx)
+        cv = mqc.conv_desc(N, C, H, W, K, R, S, st, pad)
+        y = mqc.conv2d_fwd(xs, mqc.quantize_mx(_dev(w), 0, 2, 0), cv)
+        xd = orc.dequantize(*orc.quantize(x, 0, 2, 0), x.shape, 0, 2, 0)
+        wd = orc.dequantize(*orc.quantize(w, 0, 2, 0), w.shape, 0, 2, 0)
+        ref, refabs = orc.conv_fwd(xd, wd, st, st, pad, pad)
+        _check(f"fwd {case} at a shared address", _host(y), ref, refabs)
